@@ -1,0 +1,126 @@
+/*
+ * fa_varlen.h -- C ABI of the B200 (sm_100a) variable-length attention
+ * library, libfa_varlen.so.
+ *
+ * What it computes. Exact scaled-dot-product attention over a batch of
+ * sequences packed back to back without padding, addressed by cumulative
+ * offsets, forward and backward, with an optional causal mask:
+ *
+ *   for each sequence b and head h, with Q_b = q[cu_seqlens_q[b] :
+ *   cu_seqlens_q[b+1], h, :] and K_b, V_b taken likewise from cu_seqlens_k,
+ *     S = softmax_scale * Q_b K_b^T, masked entries excluded,
+ *     lse_i = log sum_j exp(S_ij)          (natural log, scaled scores),
+ *     out   = exp(S - lse) V_b.
+ *
+ * Sources: the page "Mecanismo cu_seqlens en FlashAttention" (friki.work),
+ * sections "Estructuras de datos clave" (the offsets arrays hold batch+1
+ * cumulative offsets; [0,128,300] means lengths 128 and 172), "Lógica de
+ * cálculo de longitud" (length = cu[b+1] - cu[b]) and "Optimización de
+ * acceso a memoria" (a sequence starts at packed row cu[b]); the page
+ * "FlashAttention na inferência" (slavadubrov.com), section "Separar o
+ * armazenamento do cálculo" (exact attention: score every visible pair,
+ * normalise, multiply by V; computed here blockwise with an online softmax,
+ * never materialising S in memory); the page "FlashAttention-2 GPU work
+ * partitioning" (iplexlaw.co.kr), section "Bloques pequeños, normalización
+ * global" (global normalisation; results equal up to floating-point order);
+ * the page "Flash-Atención y Flash-Atención-2" (zepes.com), FlashAttention v1
+ * and backward sections (the backward recomputes the probabilities; column
+ * blocks are independent workers and the query gradient is aggregated with
+ * atomic additions).
+ *
+ * Causal mask. Key j of a sequence is visible from its query i iff
+ *   j <= i + (lk - lq)        (bottom-right alignment; for lq == lk this is
+ *                              the usual j <= i).
+ * A query row with no visible key gets out = 0 and lse = -inf.
+ *
+ * Layouts (all row-major, contiguous, device memory):
+ *   q, out, dout, dq : bf16 [total_q, num_heads, head_dim]
+ *   k, v, dk, dv     : bf16 [total_k, num_heads, head_dim]
+ *   softmax_lse      : fp32 [num_heads, total_q]
+ *   cu_seqlens_q/k   : int32 [batch + 1], device memory, cu[0] = 0,
+ *                      non-decreasing, cu[batch] = total_q / total_k.
+ * Element (row, h, c) of a packed tensor is at (row*num_heads + h)*head_dim + c.
+ *
+ * Supported: head_dim 64 or 128 (anything else returns FA_ERR_UNSUPPORTED;
+ * there is no fallback path). q, k, v, out, dout, dq, dk, dv must be 16-byte
+ * aligned. softmax_scale must be finite and > 0.
+ *
+ * Ownership and synchrony. The caller owns every buffer, including the
+ * workspace (size from the *_workspace_size functions, any 256-byte-aligned
+ * device allocation). Calls only enqueue work on `stream` and return; they
+ * never synchronise. The library keeps no state between calls. Calls are
+ * thread-safe; two calls that run concurrently must not share a workspace.
+ *
+ * Errors. The return value reports argument validation and launch errors.
+ * Errors found on the device (malformed cu_seqlens, a wait that timed out)
+ * are written to a status word in the workspace; every kernel of the call
+ * then exits early and the outputs are undefined. fa_get_device_status reads
+ * that word.
+ */
+#ifndef FA_VARLEN_H
+#define FA_VARLEN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Identical to cudaStream_t (the CUDA runtime's stream handle). */
+struct CUstream_st;
+typedef struct CUstream_st* fa_cuda_stream_t;
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARGUMENT = 1, /* null pointer, negative size, bad scale, misaligned pointer */
+  FA_ERR_UNSUPPORTED = 2,      /* head_dim not in {64, 128}, or sizes beyond the limits below */
+  FA_ERR_WORKSPACE = 3,        /* workspace null, misaligned or smaller than required */
+  FA_ERR_CUDA = 4,             /* a CUDA runtime call or launch failed */
+  FA_ERR_BAD_SEQLENS = 5,      /* device: cu_seqlens not monotone, cu[0] != 0, cu[batch] != total,
+                                  or a length above max_seqlen */
+  FA_ERR_DEVICE_TIMEOUT = 6    /* device: a pipeline wait gave up after its time limit */
+} fa_status_t;
+
+/* Limits: batch <= 65535; total_q, total_k < 2^31 / num_heads rows;
+ * num_heads * head_dim <= 65535 * 64. */
+
+/* Workspace bytes needed by fa_varlen_fwd for these sizes. */
+size_t fa_varlen_fwd_workspace_size(int batch, int total_q, int num_heads, int head_dim);
+
+/* Workspace bytes needed by fa_varlen_bwd for these sizes (includes an fp32
+ * dQ accumulator of about total_q * num_heads * head_dim * 4 bytes). */
+size_t fa_varlen_bwd_workspace_size(int batch, int total_q, int total_k, int num_heads, int head_dim);
+
+/* Forward. Writes out and softmax_lse for every row of every sequence.
+ * max_seqlen_q / max_seqlen_k bound the sequence lengths (checked on the
+ * device). Rows of out/softmax_lse outside [0, total_q) are never written. */
+fa_status_t fa_varlen_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                          const int32_t* cu_seqlens_k, int batch, int total_q, int total_k, int max_seqlen_q,
+                          int max_seqlen_k, int num_heads, int head_dim, float softmax_scale, int causal,
+                          void* out, float* softmax_lse, void* workspace, size_t workspace_bytes,
+                          fa_cuda_stream_t stream);
+
+/* Backward of L = sum(out * dout) given the forward's out and softmax_lse.
+ * Recomputes the probabilities from softmax_lse; writes dq, dk, dv.
+ * The query gradient is accumulated with fp32 atomic reductions, so dq may
+ * differ in the last bits between runs. */
+fa_status_t fa_varlen_bwd(const void* dout, const void* q, const void* k, const void* v, const void* out,
+                          const float* softmax_lse, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                          int batch, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int num_heads,
+                          int head_dim, float softmax_scale, int causal, void* dq, void* dk, void* dv,
+                          void* workspace, size_t workspace_bytes, fa_cuda_stream_t stream);
+
+/* Synchronises `stream`, then returns the device-side status of the last
+ * call that used `workspace` (FA_OK, FA_ERR_BAD_SEQLENS or
+ * FA_ERR_DEVICE_TIMEOUT), or FA_ERR_CUDA if the synchronisation failed. */
+fa_status_t fa_get_device_status(const void* workspace, fa_cuda_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char* fa_status_string(fa_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_VARLEN_H */

@@ -49,7 +49,7 @@ class OracleLib:
         lib = ctypes.CDLL(path)
         P = ctypes.c_void_p
         I = ctypes.c_int
-        lib.fa_oracle_fwd.argtypes = [P, P, P, I, P, P, I, I, I, ctypes.c_double, I, I, P, P, P]
+        lib.fa_oracle_fwd.argtypes = [P, P, P, I, P, P, I, I, I, ctypes.c_double, I, I, P, I, P, P]
         lib.fa_oracle_fwd.restype = I
         lib.fa_oracle_bwd.argtypes = [P, P, P, P, I, P, P, I, I, I, ctypes.c_double, I, I, P, P, P, P]
         lib.fa_oracle_bwd.restype = I
@@ -77,9 +77,10 @@ class OracleLib:
         cu = np.ascontiguousarray(cu, dtype=np.int32)
         return int(self.lib.fa_oracle_elem_offset(_ptr(cu), b, r, heads, h, d))
 
-    def fwd(self, q, k, v, cu_q, cu_k, scale: float, causal: bool, units=None):
+    def fwd(self, q, k, v, cu_q, cu_k, scale: float, causal: bool, units=None, row_step: int = 1):
         """Returns (out [Tq,H,d] f64, lse [H,Tq] f64). With ``units`` (list of
-        (b, h)), only those units are computed; other entries are NaN."""
+        (b, h)), only those units are computed; with ``row_step`` > 1 only
+        query rows i % row_step == 0 of each unit. Other entries are NaN."""
         q, dt = _as_input(q)
         k, dtk = _as_input(k)
         v, dtv = _as_input(v)
@@ -92,7 +93,7 @@ class OracleLib:
         n, _keep, up = _units_arg(units)
         rc = self.lib.fa_oracle_fwd(_ptr(q), _ptr(k), _ptr(v), dt, _ptr(cu_q), _ptr(cu_k),
                                     len(cu_q) - 1, H, d, float(scale), int(bool(causal)), n, up,
-                                    _ptr(out), _ptr(lse))
+                                    int(row_step), _ptr(out), _ptr(lse))
         if rc != 0:
             raise MemoryError("oracle forward failed to allocate")
         return out, lse
@@ -156,8 +157,8 @@ def elem_offset(cu, b: int, r: int, heads: int, h: int, d: int) -> int:
     return _load().elem_offset(cu, b, r, heads, h, d)
 
 
-def fwd(q, k, v, cu_q, cu_k, scale: float, causal: bool, units=None):
-    return _load().fwd(q, k, v, cu_q, cu_k, scale, causal, units)
+def fwd(q, k, v, cu_q, cu_k, scale: float, causal: bool, units=None, row_step: int = 1):
+    return _load().fwd(q, k, v, cu_q, cu_k, scale, causal, units, row_step)
 
 
 def bwd(q, k, v, dout, cu_q, cu_k, scale: float, causal: bool, units=None):

@@ -132,10 +132,12 @@ static void unit_at(int64_t u, int H, const int32_t* units, int* b, int* h) {
   }
 }
 
-/* Forward: out = softmax(scale * Q K^T, masked) V per unit; lse per row. */
+/* Forward: out = softmax(scale * Q K^T, masked) V per unit; lse per row.
+ * row_step > 1 computes only query rows i with i % row_step == 0 (rows are
+ * independent in the forward, so a sample of rows is exact). */
 int fa_oracle_fwd(const void* q, const void* k, const void* v, int dtype,
                   const int32_t* cu_q, const int32_t* cu_k, int batch, int H, int d,
-                  double scale, int causal, int n_units, const int32_t* units,
+                  double scale, int causal, int n_units, const int32_t* units, int row_step,
                   double* out, double* lse) {
   const int64_t total_q = cu_q[batch];
   const int64_t nu = unit_count(batch, H, n_units, units);
@@ -154,7 +156,7 @@ int fa_oracle_fwd(const void* q, const void* k, const void* v, int dtype,
       continue;
     }
     for (int64_t j = 0; j < lk; ++j) koffs[j] = fa_oracle_elem_offset(cu_k, b, j, H, h, d);
-    for (int64_t i = 0; i < lq; ++i) {
+    for (int64_t i = 0; i < lq; i += (row_step > 1 ? row_step : 1)) {
       const int64_t qoff = fa_oracle_elem_offset(cu_q, b, i, H, h, d);
       int64_t nvis = score_row(q, k, dtype, qoff, koffs, i, lq, lk, d, scale, causal, s);
       double l = softmax_row(s, lk, nvis);

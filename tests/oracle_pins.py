@@ -322,9 +322,29 @@ def pin_bf16_path(orc):
         assert all(np.array_equal(x, y) for x, y in zip(ga, gb))
 
 
+def pin_row_and_unit_sampling(orc):
+    """A sample of units or of query rows is exactly the full result on the
+    sampled entries (rows of the forward are independent)."""
+    q, k, v, do, cu_q, cu_k = _batch(23, H=3, d=4, lq=[9, 12], lk=[7, 12])
+    for causal in (False, True):
+        full_o, full_l = orc.fwd(q, k, v, cu_q, cu_k, 0.45, causal)
+        o, l = orc.fwd(q, k, v, cu_q, cu_k, 0.45, causal, units=[(1, 2), (0, 0)], row_step=4)
+        for b, h in ((1, 2), (0, 0)):
+            rows = [cu_q[b] + i for i in range(0, cu_q[b + 1] - cu_q[b], 4)]
+            assert np.array_equal(o[rows, h], full_o[rows, h])
+            assert np.array_equal(l[h, rows], full_l[h, rows])
+        assert np.isnan(o[cu_q[0] + 1, 0, 0]) and np.isnan(o[0, 1, 0])
+        g_full = orc.bwd(q, k, v, do, cu_q, cu_k, 0.45, causal)
+        g = orc.bwd(q, k, v, do, cu_q, cu_k, 0.45, causal, units=[(1, 1)])
+        sq, sk = slice(cu_q[1], cu_q[2]), slice(cu_k[1], cu_k[2])
+        assert np.array_equal(g[0][sq, 1], g_full[0][sq, 1])
+        assert np.array_equal(g[1][sk, 1], g_full[1][sk, 1])
+        assert np.array_equal(g[2][sk, 1], g_full[2][sk, 1])
+
+
 ALL_PINS = [
     pin_seqlens_golden, pin_elem_offset, pin_rows_sum_to_one, pin_lse_bounds,
     pin_varlen_independence, pin_single_key, pin_causal_row0, pin_constant_v,
     pin_bruteforce, pin_torch_sdpa, pin_finite_differences, pin_grad_invariants,
-    pin_empty_rows, pin_bf16_path,
+    pin_empty_rows, pin_bf16_path, pin_row_and_unit_sampling,
 ]

@@ -1,0 +1,99 @@
+"""CPU-only checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa_varlen.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from varlen_flashattention_02_b200 import fa_varlen
+
+    return fa_varlen.lib
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("fa_varlen_fwd", "fa_varlen_bwd", "fa_varlen_fwd_workspace_size",
+              "fa_varlen_bwd_workspace_size", "fa_get_device_status", "fa_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), f"{n} declared in the header but not exported"
+
+
+def test_status_strings(lib):
+    assert lib.fa_status_string(0) == b"FA_OK"
+    assert lib.fa_status_string(5) == b"FA_ERR_BAD_SEQLENS"
+    assert lib.fa_status_string(6) == b"FA_ERR_DEVICE_TIMEOUT"
+
+
+def test_workspace_sizes(lib):
+    f = lib.fa_varlen_fwd_workspace_size(2, 1024, 12, 64)
+    assert f >= 256 + 4 * 3 + 8 * (1024 // 128 + 3)
+    b = lib.fa_varlen_bwd_workspace_size(2, 1024, 1024, 12, 64)
+    assert b >= 12 * 1024 * 64 * 4  # holds the fp32 dQ accumulator
+    assert lib.fa_varlen_fwd_workspace_size(0, 10, 1, 64) == 0
+
+
+FAKE = 0x10000  # never dereferenced: validation fails first
+
+
+def _fwd(lib, **over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, cu_q=FAKE, cu_k=FAKE, batch=2, total_q=1024, total_k=1024, max_q=824,
+             max_k=724, H=12, D=64, scale=0.125, causal=0, out=FAKE, lse=FAKE, ws=FAKE, ws_bytes=1 << 30,
+             stream=None)
+    a.update(over)
+    return lib.fa_varlen_fwd(a["q"], a["k"], a["v"], a["cu_q"], a["cu_k"], a["batch"], a["total_q"],
+                             a["total_k"], a["max_q"], a["max_k"], a["H"], a["D"], a["scale"], a["causal"],
+                             a["out"], a["lse"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(D=96), 2), (dict(D=256), 2), (dict(batch=0), 1), (dict(H=0), 1), (dict(total_q=-1), 1),
+    (dict(scale=0.0), 1), (dict(scale=float("inf")), 1), (dict(scale=-1.0), 1), (dict(q=None), 1),
+    (dict(cu_q=None), 1), (dict(q=FAKE + 8), 1), (dict(out=FAKE + 2), 1), (dict(ws=None), 3),
+    (dict(ws=FAKE + 16), 3), (dict(ws_bytes=64), 3),
+], ids=lambda x: str(x))
+def test_fwd_rejects(lib, over, code):
+    assert _fwd(lib, **over) == code
+
+
+def _bwd(lib, **over):
+    a = dict(do=FAKE, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, cu_q=FAKE, cu_k=FAKE, batch=2, total_q=1024,
+             total_k=1024, max_q=824, max_k=724, H=12, D=64, scale=0.125, causal=1, dq=FAKE, dk=FAKE, dv=FAKE,
+             ws=FAKE, ws_bytes=1 << 34, stream=None)
+    a.update(over)
+    return lib.fa_varlen_bwd(a["do"], a["q"], a["k"], a["v"], a["o"], a["lse"], a["cu_q"], a["cu_k"], a["batch"],
+                             a["total_q"], a["total_k"], a["max_q"], a["max_k"], a["H"], a["D"], a["scale"],
+                             a["causal"], a["dq"], a["dk"], a["dv"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(D=32), 2), (dict(batch=-3), 1), (dict(scale=float("nan")), 1), (dict(do=None), 1), (dict(dk=None), 1),
+    (dict(dv=FAKE + 4), 1), (dict(ws_bytes=1024), 3),
+], ids=lambda x: str(x))
+def test_bwd_rejects(lib, over, code):
+    assert _bwd(lib, **over) == code
+
+
+def test_no_cpu_fallback_in_binding():
+    """The binding only marshals arguments: it must not import the oracle or
+    compute attention itself."""
+    src = open(os.path.join(ROOT, "varlen_flashattention_02_b200", "fa_varlen.py")).read()
+    assert "oracle" not in src
+    for forbidden in ("softmax(", "matmul", "einsum", "@ "):
+        assert forbidden not in src

@@ -1,0 +1,63 @@
+"""The device work-list preparation against its CPU restatement, and the
+device-side rejection of malformed cumulative offsets."""
+import numpy as np
+import pytest
+
+from tests import parity_util as pu
+from tests import sched_restatement as sr
+from varlen_flashattention_02_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _read_pairs(ws, backward, batch, total_q, total_k):
+    lay = sr.layout(batch, total_q, total_k, backward)
+    raw = ws.cpu().numpy()
+    status, n_pairs = (int(x) for x in raw[:8].view(np.uint32))
+    pairs = raw[lay["pairs"]:lay["pairs"] + 8 * n_pairs].view(np.int32).reshape(-1, 2)
+    return status, pairs
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("wl", [1, 3, 5])
+def test_fwd_work_list(wl, causal):
+    from varlen_flashattention_02_b200 import fa_varlen
+
+    w = synth.standard_workload(wl)
+    w.causal = causal
+    ws = fa_varlen.new_workspace(fa_varlen.fwd_workspace_size(w.batch, w.total_q, w.heads, w.head_dim), "cuda")
+    pu.run_fwd(w, workspace=ws)
+    status, pairs = _read_pairs(ws, False, w.batch, w.total_q, w.total_k)
+    assert status == 0
+    want = sr.work_list(w.cu_q, w.cu_k, causal)
+    cost = {(b, t): c for b, t, c in want}
+    got = [(int(b), int(t)) for b, t in pairs]
+    assert sorted(got) == sorted(cost)  # same multiset, no padding tiles
+    costs = [cost[p] for p in got]
+    assert all(costs[i] >= costs[i + 1] for i in range(len(costs) - 1))  # longest first
+
+
+@pytest.mark.parametrize("cu_q,cu_k,max_q", [
+    ([0, 10, 5, 20], [0, 10, 15, 20], 64),   # decreasing
+    ([1, 10, 20], [0, 10, 20], 64),          # does not start at 0
+    ([0, 10, 20], [0, 10, 20], 8),           # longer than max_seqlen
+], ids=["decreasing", "nonzero-start", "over-max"])
+def test_bad_seqlens_reported(cu_q, cu_k, max_q):
+    import torch
+
+    from varlen_flashattention_02_b200 import fa_varlen
+
+    H, D = 2, 64
+    Tq, Tk = 20, 20
+    q = torch.randn(Tq, H, D, device="cuda").bfloat16()
+    k = torch.randn(Tk, H, D, device="cuda").bfloat16()
+    v = torch.randn(Tk, H, D, device="cuda").bfloat16()
+    ws = fa_varlen.new_workspace(fa_varlen.fwd_workspace_size(2, Tq, H, D), "cuda")
+    cq = torch.tensor(cu_q, dtype=torch.int32, device="cuda")
+    ck = torch.tensor(cu_k, dtype=torch.int32, device="cuda")
+    fa_varlen.fa_varlen_fwd(q, k, v, cq, ck, max_q, 64, 0.125, False, workspace=ws)
+    assert fa_varlen.device_status(ws) == 5  # FA_ERR_BAD_SEQLENS
+    # The same workspace is usable again afterwards.
+    good = torch.tensor([0, 10, 20], dtype=torch.int32, device="cuda")
+    fa_varlen.fa_varlen_fwd(q, k, v, good, good, 10, 10, 0.125, False, workspace=ws)
+    assert fa_varlen.device_status(ws) == 0

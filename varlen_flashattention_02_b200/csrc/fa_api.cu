@@ -1,0 +1,231 @@
+// fa_api.cu -- the C ABI of libfa_varlen.so (declared in include/fa_varlen.h):
+// argument validation, workspace layout, TMA descriptor encoding and kernel
+// launches. Host code only; it never synchronises except in
+// fa_get_device_status.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fa_varlen.h"
+#include "fa_common.cuh"
+#include "fa_kernels.h"
+
+namespace {
+
+using fa::WsLayout;
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 map over a packed [rows, H*D] tensor: inner dimension H*D
+// elements, row stride H*D*2 bytes, box = 64 columns x box_rows rows,
+// 128-byte swizzle, out-of-range rows read as zero.
+bool encode_map(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+// Shared size checks of both directions.
+fa_status_t check_sizes(int batch, int total_q, int total_k, int max_sq, int max_sk, int H, int D, float scale) {
+  if (batch < 1 || total_q < 0 || total_k < 0 || max_sq < 0 || max_sk < 0 || H < 1) return FA_ERR_INVALID_ARGUMENT;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARGUMENT;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  // Row indices and TMA coordinates are int32; element offsets are 64-bit.
+  const long long hd = static_cast<long long>(H) * D;
+  if (hd > (1ll << 31) - 1 || static_cast<long long>(total_q) + 2 * fa::kFwdBM > (1ll << 31) - 1 ||
+      static_cast<long long>(total_k) + 2 * fa::kFwdBN > (1ll << 31) - 1)
+    return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(total_q / fa::kFwdBM + batch + 1) * H > (1ll << 31) - 1 ||
+      static_cast<long long>(total_k / fa::kBwdBN + batch + 1) * H > (1ll << 31) - 1)
+    return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fa_varlen_fwd_workspace_size(int batch, int total_q, int num_heads, int head_dim) {
+  if (batch < 1 || total_q < 0 || num_heads < 1) return 0;
+  return fa::ws_layout(false, batch, total_q, 0, num_heads, head_dim).total;
+}
+
+size_t fa_varlen_bwd_workspace_size(int batch, int total_q, int total_k, int num_heads, int head_dim) {
+  if (batch < 1 || total_q < 0 || total_k < 0 || num_heads < 1) return 0;
+  return fa::ws_layout(true, batch, total_q, total_k, num_heads, head_dim).total;
+}
+
+const char* fa_status_string(fa_status_t s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARGUMENT: return "FA_ERR_INVALID_ARGUMENT";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_BAD_SEQLENS: return "FA_ERR_BAD_SEQLENS";
+    case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT";
+  }
+  return "FA_ERR_UNKNOWN";
+}
+
+fa_status_t fa_varlen_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                          const int32_t* cu_seqlens_k, int batch, int total_q, int total_k, int max_seqlen_q,
+                          int max_seqlen_k, int num_heads, int head_dim, float softmax_scale, int causal,
+                          void* out, float* softmax_lse, void* workspace, size_t workspace_bytes,
+                          fa_cuda_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  fa_status_t st = check_sizes(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, num_heads, head_dim,
+                               softmax_scale);
+  if (st != FA_OK) return st;
+  if (!cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARGUMENT;
+  if (total_q > 0 && (!q || !out || !softmax_lse || !aligned16(q) || !aligned16(out))) return FA_ERR_INVALID_ARGUMENT;
+  if (total_k > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return FA_ERR_INVALID_ARGUMENT;
+  const WsLayout L = fa::ws_layout(false, batch, total_q, total_k, num_heads, head_dim);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < L.total)
+    return FA_ERR_WORKSPACE;
+
+  fa::SchedArgs sa{cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q, max_seqlen_k,
+                   causal ? 1 : 0, 0, workspace, L.seq_off, L.pairs, L.max_pairs};
+  if (fa::launch_sched_prep(sa, stream) != cudaSuccess) return FA_ERR_CUDA;
+  if (total_q == 0) return FA_OK;
+
+  const int HD = num_heads * head_dim;
+  CUtensorMap tq, tk, tv;
+  // With no keys at all every row is empty and K/V are never read; the maps
+  // then point at q so that they are still well formed.
+  const void* kp = total_k > 0 ? k : q;
+  const void* vp = total_k > 0 ? v : q;
+  const int krows = total_k > 0 ? total_k : total_q;
+  if (!encode_map(&tq, q, total_q, HD, fa::kFwdBM) || !encode_map(&tk, kp, krows, HD, fa::kFwdBN) ||
+      !encode_map(&tv, vp, krows, HD, fa::kFwdBN))
+    return FA_ERR_CUDA;
+
+  const int sms = sm_count();
+  if (sms <= 0) return FA_ERR_CUDA;
+  const long long items = static_cast<long long>(L.max_pairs) * num_heads;
+  fa::FwdArgs fa_args{};
+  fa_args.cu_q = cu_seqlens_q;
+  fa_args.cu_k = cu_seqlens_k;
+  fa_args.out = out;
+  fa_args.lse = softmax_lse;
+  fa_args.workspace = workspace;
+  fa_args.pairs_offset = L.pairs;
+  fa_args.H = num_heads;
+  fa_args.D = head_dim;
+  fa_args.total_q = total_q;
+  fa_args.causal = causal ? 1 : 0;
+  fa_args.scale_log2 = softmax_scale * 1.4426950408889634f;
+  fa_args.grid = static_cast<int>(items < sms ? items : sms);
+  if (fa::launch_fwd(fa_args, tq, tk, tv, stream) != cudaSuccess) return FA_ERR_CUDA;
+  return FA_OK;
+}
+
+fa_status_t fa_varlen_bwd(const void* dout, const void* q, const void* k, const void* v, const void* out,
+                          const float* softmax_lse, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                          int batch, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int num_heads,
+                          int head_dim, float softmax_scale, int causal, void* dq, void* dk, void* dv,
+                          void* workspace, size_t workspace_bytes, fa_cuda_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  fa_status_t st = check_sizes(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, num_heads, head_dim,
+                               softmax_scale);
+  if (st != FA_OK) return st;
+  if (!cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARGUMENT;
+  if (total_q > 0 && (!q || !dout || !out || !softmax_lse || !dq || !aligned16(q) || !aligned16(dout) ||
+                      !aligned16(out) || !aligned16(dq)))
+    return FA_ERR_INVALID_ARGUMENT;
+  if (total_k > 0 && (!k || !v || !dk || !dv || !aligned16(k) || !aligned16(v) || !aligned16(dk) || !aligned16(dv)))
+    return FA_ERR_INVALID_ARGUMENT;
+  const WsLayout L = fa::ws_layout(true, batch, total_q, total_k, num_heads, head_dim);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < L.total)
+    return FA_ERR_WORKSPACE;
+
+  fa::SchedArgs sa{cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q, max_seqlen_k,
+                   causal ? 1 : 0, 1, workspace, L.seq_off, L.pairs, L.max_pairs};
+  if (fa::launch_sched_prep(sa, stream) != cudaSuccess) return FA_ERR_CUDA;
+  if (total_q == 0 && total_k == 0) return FA_OK;
+
+  const int HD = num_heads * head_dim;
+  CUtensorMap tq, tk, tv, tdo;
+  const void* anyp = total_q > 0 ? q : k;
+  const void* qp = total_q > 0 ? q : anyp;
+  const void* dop = total_q > 0 ? dout : anyp;
+  const void* kp = total_k > 0 ? k : anyp;
+  const void* vp = total_k > 0 ? v : anyp;
+  const int qrows = total_q > 0 ? total_q : total_k;
+  const int krows = total_k > 0 ? total_k : total_q;
+  if (!encode_map(&tq, qp, qrows, HD, fa::kBwdBM) || !encode_map(&tdo, dop, qrows, HD, fa::kBwdBM) ||
+      !encode_map(&tk, kp, krows, HD, fa::kBwdBN) || !encode_map(&tv, vp, krows, HD, fa::kBwdBN))
+    return FA_ERR_CUDA;
+
+  const int sms = sm_count();
+  if (sms <= 0) return FA_ERR_CUDA;
+  const long long items = static_cast<long long>(L.max_pairs) * num_heads;
+  fa::BwdArgs b{};
+  b.cu_q = cu_seqlens_q;
+  b.cu_k = cu_seqlens_k;
+  b.dout = dout;
+  b.out = out;
+  b.lse = softmax_lse;
+  b.dq = dq;
+  b.dk = dk;
+  b.dv = dv;
+  b.workspace = workspace;
+  b.pairs_offset = L.pairs;
+  b.dvec_offset = L.dvec;
+  b.dqacc_offset = L.dqacc;
+  b.tq_pad = L.tq_pad;
+  b.H = num_heads;
+  b.D = head_dim;
+  b.total_q = total_q;
+  b.total_k = total_k;
+  b.causal = causal ? 1 : 0;
+  b.scale = softmax_scale;
+  b.scale_log2 = softmax_scale * 1.4426950408889634f;
+  b.grid = static_cast<int>(items < sms ? items : sms);
+  if (fa::launch_bwd(b, tq, tk, tv, tdo, stream) != cudaSuccess) return FA_ERR_CUDA;
+  return FA_OK;
+}
+
+fa_status_t fa_get_device_status(const void* workspace, fa_cuda_stream_t stream_) {
+  if (!workspace) return FA_ERR_INVALID_ARGUMENT;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return FA_ERR_CUDA;
+  uint32_t status = 0;
+  if (cudaMemcpy(&status, workspace, sizeof status, cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_CUDA;
+  return static_cast<fa_status_t>(status);
+}
+
+}  // extern "C"

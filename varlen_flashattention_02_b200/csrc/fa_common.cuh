@@ -1,0 +1,164 @@
+// fa_common.cuh -- pieces shared by the scheduler, forward and backward
+// kernels and the host API: tile sizes, the workspace layout, sequence
+// information from cumulative offsets, visible-tile ranges under the causal
+// mask, and the bounded mbarrier wait.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/fa_varlen.h"
+#include "sm100_ptx.cuh"
+
+namespace fa {
+
+// Forward tiles: a work item is 128 query rows of one (sequence, head);
+// keys stream through in tiles of 128.
+constexpr int kFwdBM = 128;
+constexpr int kFwdBN = 128;
+// Backward tiles: a work item is 128 key rows of one (sequence, head);
+// queries stream through in tiles of 64.
+constexpr int kBwdBN = 128;
+constexpr int kBwdBM = 64;
+
+// Per-call device state at the start of the workspace.
+struct WsHeader {
+  uint32_t status;   // fa_status_t of the device side of the call
+  uint32_t n_pairs;  // number of (sequence, tile) pairs in `pairs`
+  uint32_t reserved[62];
+};
+static_assert(sizeof(WsHeader) == 256, "header is one 256-byte block");
+
+__host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Upper bound on the number of (sequence, tile) pairs: sum_b ceil(len_b / T)
+// <= total / T + batch.
+__host__ __device__ inline int max_pairs(int batch, int total, int tile) { return total / tile + batch + 1; }
+
+// Rows of the padded fp32 dQ accumulator per head: a query tile may run up
+// to kBwdBM - 1 rows past the last token.
+__host__ __device__ inline int dq_rows_padded(int total_q) { return static_cast<int>(align_up(total_q + kBwdBM, 64)); }
+
+struct WsLayout {
+  size_t seq_off;  // int32 [batch + 1]: first pair index of each sequence
+  size_t pairs;    // int2  [max_pairs]: (sequence, tile), longest first
+  size_t dvec;     // fp32  [H, tq_pad] (backward only): rowsum(dO * O)
+  size_t dqacc;    // fp32  [H, tq_pad, D] (backward only)
+  size_t total;
+  int max_pairs;
+  int tq_pad;
+};
+
+__host__ __device__ inline WsLayout ws_layout(bool backward, int batch, int total_q, int total_k, int H, int D) {
+  WsLayout L{};
+  size_t off = sizeof(WsHeader);
+  L.seq_off = off;
+  off = align_up(off + sizeof(int32_t) * (static_cast<size_t>(batch) + 1), 256);
+  L.max_pairs = backward ? max_pairs(batch, total_k, kBwdBN) : max_pairs(batch, total_q, kFwdBM);
+  L.pairs = off;
+  off = align_up(off + 8 * static_cast<size_t>(L.max_pairs), 256);
+  if (backward) {
+    L.tq_pad = dq_rows_padded(total_q);
+    L.dvec = off;
+    off = align_up(off + sizeof(float) * static_cast<size_t>(H) * L.tq_pad, 256);
+    L.dqacc = off;
+    off = align_up(off + sizeof(float) * static_cast<size_t>(H) * L.tq_pad * D, 256);
+  }
+  L.total = off;
+  return L;
+}
+
+// ---------------------------------------------------------------- sequences
+// Page "Mecanismo cu_seqlens en FlashAttention", "Lógica de cálculo de
+// longitud": sequence b starts at packed row cu[b] and has cu[b+1] - cu[b]
+// rows (the cumulative branch; lengths-only and left-padded keys are not
+// supported).
+struct SeqInfo {
+  int q0, lq, k0, lk;
+};
+__device__ __forceinline__ SeqInfo seq_info(const int32_t* cu_q, const int32_t* cu_k, int b) {
+  SeqInfo s;
+  s.q0 = __ldg(cu_q + b);
+  s.lq = __ldg(cu_q + b + 1) - s.q0;
+  s.k0 = __ldg(cu_k + b);
+  s.lk = __ldg(cu_k + b + 1) - s.k0;
+  return s;
+}
+
+// Number of key tiles visible from query tile t (rows t*BM ..), given the
+// bottom-right causal rule j <= i + (lk - lq). Tiles wholly above the
+// diagonal are skipped.
+__host__ __device__ inline int fwd_num_k_tiles(int t, int lq, int lk, bool causal) {
+  if (lk <= 0 || lq <= 0) return 0;
+  const int nk = (lk + kFwdBN - 1) / kFwdBN;
+  if (!causal) return nk;
+  const int rmax = ((t + 1) * kFwdBM < lq ? (t + 1) * kFwdBM : lq) - 1;
+  const long long last = static_cast<long long>(rmax) + lk - lq;
+  if (last < 0) return 0;
+  const long long n = last / kFwdBN + 1;
+  return n < nk ? static_cast<int>(n) : nk;
+}
+
+// Range [begin, end) of backward query tiles (kBwdBM rows) that see at least
+// one key of key tile j (keys j*BN ..).
+__host__ __device__ inline void bwd_q_tiles(int j, int lq, int lk, bool causal, int* begin, int* end) {
+  const int nq = (lq + kBwdBM - 1) / kBwdBM;
+  *end = nq;
+  *begin = 0;
+  if (lk <= 0 || lq <= 0) {
+    *begin = nq;
+    return;
+  }
+  if (causal) {
+    long long first = static_cast<long long>(j) * kBwdBN - (lk - lq);
+    if (first < 0) first = 0;
+    *begin = first >= lq ? nq : static_cast<int>(first / kBwdBM);
+  }
+}
+
+// --------------------------------------------------------- bounded waits
+// Every pipeline wait gives up after this long, records
+// FA_ERR_DEVICE_TIMEOUT in the workspace status and raises the CTA's abort
+// flag so the other roles stop too.
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
+
+struct Abort {
+  volatile int* flag;  // shared memory, one per CTA
+  uint32_t* status;    // workspace status word
+};
+
+__device__ __forceinline__ void raise_abort(const Abort& ab) {
+  *ab.flag = 1;
+  atomicCAS(ab.status, 0u, static_cast<uint32_t>(FA_ERR_DEVICE_TIMEOUT));
+}
+
+static __device__ __noinline__ bool wait_slow(uint32_t addr, uint32_t parity, const Abort& ab) {
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(addr, parity)) return true;
+    if (*ab.flag) return false;
+    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      raise_abort(ab);
+      return false;
+    }
+  }
+}
+
+// Wait for the phase of `bar` with the given parity to complete. Returns
+// false if the CTA is aborting (the caller must stop its role).
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const Abort& ab) {
+  const uint32_t addr = smem_u32(bar);
+  if (mbar_try_wait(addr, parity)) return true;
+  return wait_slow(addr, parity, ab);
+}
+
+// Warp-uniform form for roles whose next step is a .sync.aligned tcgen05
+// instruction: every lane returns the same answer.
+__device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, const Abort& ab) {
+  const bool ok = wait_bar(bar, parity, ab);
+  return __all_sync(0xffffffffu, ok);
+}
+
+}  // namespace fa

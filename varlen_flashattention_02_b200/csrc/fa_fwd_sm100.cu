@@ -1,0 +1,387 @@
+// fa_fwd_sm100.cu -- forward varlen attention for sm_100a.
+//
+// One persistent CTA per SM walks the (sequence, head, query-tile) work list
+// built by the scheduler (longest first). For each item it computes, for
+// 128 query rows of one head of one sequence, exact attention over the
+// sequence's keys with an online softmax:
+//
+//   S_j   = Q K_j^T                      tcgen05.mma, bf16 -> fp32 in TMEM
+//   m'    = max(m, rowmax(S_j) * scale)  registers, one thread per row
+//   P_j   = exp2(S_j*scale*log2e - m')   registers -> bf16 back into TMEM
+//   O     = O * exp2(m - m') + P_j V_j   tcgen05.mma with P read from TMEM
+//   out   = O / l,  lse = (m + log2 l) * ln2
+//
+// Pages: "FlashAttention-2 GPU work partitioning" ("Bloques pequeños,
+// normalización global": the running statistics and partial output are
+// rescaled so that the normalisation stays global; "Tres mejoras": fewer
+// non-matmul operations, parallelism over the sequence, queries split across
+// workers that share K and V); "Flash-Atención y Flash-Atención-2" (tiles of
+// Q, K, V are moved from HBM to on-chip memory and only the output goes
+// back; FlashAttention-2 splits Q, not K, across warps so no cross-warp
+// reduction is needed); "Mecanismo cu_seqlens en FlashAttention" ("Lógica de
+// cálculo de longitud", "Optimización de acceso a memoria": per-sequence
+// offsets and lengths from the cumulative arrays).
+//
+// B200 design, differing from the pages' A100 kernels:
+//  * persistent grid of one CTA per SM over a longest-first work list
+//    instead of one thread block per (batch, head[, q-block]);
+//  * warp specialisation instead of 4-8 symmetric warps: warp 0 issues TMA
+//    loads, one thread of warp 1 issues tcgen05 MMAs, warps 4-7 (128
+//    threads, one per query row and TMEM lane) do the softmax and epilogue;
+//  * accumulators live in tensor memory (S double-buffered so QK^T of tile
+//    j+1 overlaps the softmax of tile j; P overwrites its own S columns as
+//    bf16 and feeds the PV MMA directly from TMEM);
+//  * O is rescaled only when a row maximum grows by more than 2^8 (the
+//    stale maximum stays consistent with l, so the result is exact);
+//  * masking is applied only on the last key tile of a sequence and on
+//    tiles that cross the causal diagonal; tiles wholly above it are never
+//    loaded.
+#include "fa_common.cuh"
+#include "fa_kernels.h"
+
+namespace fa {
+namespace {
+
+constexpr int BM = kFwdBM;
+constexpr int BN = kFwdBN;
+constexpr int kThreads = 256;
+constexpr int kSoftmaxWarp0 = 4;
+constexpr int kChunkBytes = 128 * 128;  // one [128 rows x 64 bf16] swizzled chunk
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+struct FwdSmem {
+  static constexpr int kStages = (D == 64) ? 4 : 2;
+  static constexpr int kChunks = D / 64;
+  static constexpr int kTileBytes = kChunks * kChunkBytes;  // Q, K or V tile
+  static constexpr int kQ = 0;
+  static constexpr int kKV = kQ + kTileBytes;                // stage s: K at kKV + 2s*tile, V after it
+  static constexpr int kBar = kKV + 2 * kStages * kTileBytes;
+  static constexpr int kBytes = kBar + 256;
+  static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
+  static constexpr int kSCol = 0;               // S buffers at columns 0 and 128
+  static constexpr int kOCol = 256;             // O accumulator
+};
+
+struct Bars {
+  uint64_t q_full, q_empty;
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_full, o_empty;
+  uint64_t drain;
+  uint64_t k_full[4], v_full[4], kv_empty[4];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block fits its reserved space");
+
+struct Item {
+  int b, h, t;
+  SeqInfo s;
+  int nk;
+};
+
+__device__ __forceinline__ Item get_item(const FwdArgs& a, const int2* pairs, int idx) {
+  Item it;
+  const int2 pr = pairs[idx / a.H];
+  it.h = idx % a.H;
+  it.b = pr.x;
+  it.t = pr.y;
+  it.s = seq_info(a.cu_q, a.cu_k, it.b);
+  it.nk = fwd_num_k_tiles(it.t, it.s.lq, it.s.lk, a.causal != 0);
+  return it;
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
+  using L = FwdSmem<D>;
+  constexpr int NS = L::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars& bars = *reinterpret_cast<Bars*>(smem + L::kBar);
+
+  auto* hdr = reinterpret_cast<WsHeader*>(a.workspace);
+  const int2* pairs = reinterpret_cast<const int2*>(static_cast<const char*>(a.workspace) + a.pairs_offset);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars.q_full, 1);
+    mbar_init(&bars.q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.s_full[i], 1);
+      mbar_init(&bars.p_full[i], 4);
+    }
+    mbar_init(&bars.o_full, 1);
+    mbar_init(&bars.o_empty, 4);
+    mbar_init(&bars.drain, 1);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&bars.k_full[i], 1);
+      mbar_init(&bars.v_full[i], 1);
+      mbar_init(&bars.kv_empty[i], 1);
+    }
+    bars.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars.tmem_base;
+
+  const Abort ab{&bars.abort_flag, &hdr->status};
+  const int n_items = (hdr->status == FA_OK) ? static_cast<int>(hdr->n_pairs) * a.H : 0;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    uint32_t kv = 0, nq = 0;
+    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+      const Item it = get_item(a, pairs, idx);
+      if (it.nk == 0) continue;
+      if (nq > 0 && !wait_bar(&bars.q_empty, (nq - 1) & 1, ab)) goto producer_done;
+      mbar_arrive_expect_tx(&bars.q_full, L::kTileBytes);
+      for (int c = 0; c < L::kChunks; ++c)
+        tma_load_2d(&tm_q, &bars.q_full, smem + L::kQ + c * kChunkBytes, it.h * D + c * 64, it.s.q0 + it.t * BM);
+      ++nq;
+      for (int j = 0; j < it.nk; ++j, ++kv) {
+        const int st = kv % NS;
+        const uint32_t use = kv / NS;
+        if (use > 0 && !wait_bar(&bars.kv_empty[st], (use - 1) & 1, ab)) goto producer_done;
+        uint8_t* sk = smem + L::kKV + 2 * st * L::kTileBytes;
+        uint8_t* sv = sk + L::kTileBytes;
+        const int row = it.s.k0 + j * BN;
+        mbar_arrive_expect_tx(&bars.k_full[st], L::kTileBytes);
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_2d(&tm_k, &bars.k_full[st], sk + c * kChunkBytes, it.h * D + c * 64, row);
+        mbar_arrive_expect_tx(&bars.v_full[st], L::kTileBytes);
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_2d(&tm_v, &bars.v_full[st], sv + c * kChunkBytes, it.h * D + c * 64, row);
+      }
+    }
+  producer_done:
+    // Never leave TMA writes in flight into shared memory we are about to
+    // give up: wait (bounded) for the last loads issued.
+    if (nq > 0) wait_bar(&bars.q_full, (nq - 1) & 1, ab);
+    for (uint32_t i = (kv > NS ? kv - NS : 0); i < kv; ++i) {
+      wait_bar(&bars.k_full[i % NS], (i / NS) & 1, ab);
+      wait_bar(&bars.v_full[i % NS], (i / NS) & 1, ab);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BN, false, false);
+    constexpr uint32_t kIdescO = idesc_bf16_f32(BM, D, false, true);
+    const uint32_t sq = smem_u32(smem + L::kQ);
+    uint32_t kv = 0, g = 0, nq = 0;
+    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+      const Item it = get_item(a, pairs, idx);
+      if (it.nk == 0) continue;
+      if (!wait_bar(&bars.q_full, nq & 1, ab)) goto mma_done;
+      tc_fence_after();
+      for (int j = 0; j <= it.nk; ++j) {
+        if (j < it.nk) {
+          // S_j = Q K_j^T into S buffer (g + j) & 1.
+          const uint32_t kvj = kv + j;
+          const int st = kvj % NS;
+          if (!wait_bar(&bars.k_full[st], (kvj / NS) & 1, ab)) goto mma_done;
+          tc_fence_after();
+          const uint32_t sk = smem_u32(smem + L::kKV + 2 * st * L::kTileBytes);
+          const uint32_t d_s = tmem + L::kSCol + ((g + j) & 1) * BN;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
+            mma_ss(d_s, smem_desc_sw128(sq + off, 16, 1024), smem_desc_sw128(sk + off, 16, 1024), kIdescS,
+                   kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&bars.s_full[(g + j) & 1]);
+          if (j == it.nk - 1) mma_commit(&bars.q_empty);
+        }
+        if (j > 0) {
+          // O (+)= P_{j-1} V_{j-1}, P read from TMEM.
+          const int jj = j - 1;
+          const uint32_t gj = g + jj, kvj = kv + jj;
+          const int st = kvj % NS;
+          if (!wait_bar(&bars.p_full[gj & 1], (gj >> 1) & 1, ab)) goto mma_done;
+          if (jj == 0 && nq > 0 && !wait_bar(&bars.o_empty, (nq - 1) & 1, ab)) goto mma_done;
+          if (!wait_bar(&bars.v_full[st], (kvj / NS) & 1, ab)) goto mma_done;
+          tc_fence_after();
+          const uint32_t sv = smem_u32(smem + L::kKV + (2 * st + 1) * L::kTileBytes);
+          const uint32_t a_p = tmem + L::kSCol + (gj & 1) * BN;
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            mma_ts(tmem + L::kOCol, a_p + kk * 8, smem_desc_sw128(sv + kk * 2048, kChunkBytes, 1024), kIdescO,
+                   (jj > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&bars.kv_empty[st]);
+          mma_commit(&bars.o_full);
+        }
+      }
+      kv += it.nk;
+      g += it.nk;
+      ++nq;
+    }
+  mma_done:
+    // Make sure every MMA this thread issued has finished before TMEM is freed.
+    mma_commit(&bars.drain);
+    wait_bar(&bars.drain, 0, ab);
+  } else if (warp >= kSoftmaxWarp0) {
+    // ------------------------------------------------------------ softmax
+    const int row = threadIdx.x - kSoftmaxWarp0 * 32;  // query row in tile == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    uint32_t g = 0, nq = 0;
+    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+      const Item it = get_item(a, pairs, idx);
+      const int r = it.t * BM + row;  // row within the sequence
+      const bool row_ok = r < it.s.lq;
+      const size_t orow = (static_cast<size_t>(it.s.q0) + r) * a.H + it.h;
+      if (it.nk == 0) {
+        if (row_ok) {
+          uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + orow * D);
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c) o[c] = make_uint4(0, 0, 0, 0);
+          a.lse[static_cast<size_t>(it.h) * a.total_q + it.s.q0 + r] = -INFINITY;
+        }
+        continue;
+      }
+      float m_used = -INFINITY, l = 0.f;
+      const int diag = it.s.lk - it.s.lq;  // key j visible from row i iff j <= i + diag
+      for (int j = 0; j < it.nk; ++j, ++g) {
+        const uint32_t buf = g & 1;
+        if (!wait_bar_warp(&bars.s_full[buf], (g >> 1) & 1, ab)) goto softmax_done;
+        tc_fence_after();
+        uint32_t sr[BN];
+        const uint32_t t_s = tmem + lane_base + L::kSCol + buf * BN;
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_s + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        tmem_wait_ld();
+        float* s = reinterpret_cast<float*>(sr);
+        const int key0 = j * BN;
+        const bool need_mask = (key0 + BN > it.s.lk) || (CAUSAL && key0 + BN - 1 > it.t * BM + diag);
+        if (need_mask) {
+          int lim = it.s.lk - key0;
+          if (CAUSAL) lim = min(lim, r + diag + 1 - key0);
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (c >= lim) s[c] = -INFINITY;
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+        const float m_new = fmaxf(m_used, mx * a.scale_log2);
+        // The previous PV must be complete before O may be rescaled (and so
+        // that the o_full phase count stays in step).
+        if (j > 0) {
+          if (!wait_bar_warp(&bars.o_full, (g - 1) & 1, ab)) goto softmax_done;
+          tc_fence_after();
+        }
+        float alpha = 1.f;
+        if (m_new > m_used + kRescaleThreshold) {
+          alpha = ex2_approx(m_used - m_new);  // 0 when m_used = -inf
+          l *= alpha;
+          m_used = m_new;
+        }
+        if (__any_sync(0xffffffffu, j > 0 && alpha != 1.f)) {
+          const uint32_t t_o = tmem + lane_base + L::kOCol;
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_o + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(t_o + c * 32, o);
+          }
+          tmem_wait_st();
+        }
+        const float m_ref = (m_used == -INFINITY) ? 0.f : m_used;
+        float lsum = 0.f;
+        uint32_t pk[BN / 2];
+#pragma unroll
+        for (int c = 0; c < BN; c += 2) {
+          const float p0 = ex2_approx(fmaf(s[c], a.scale_log2, -m_ref));
+          const float p1 = ex2_approx(fmaf(s[c + 1], a.scale_log2, -m_ref));
+          lsum += p0 + p1;
+          pk[c / 2] = pack_bf16x2(p0, p1);
+        }
+        l += lsum;
+        // P (bf16, two per column) overwrites the first BN/2 columns of S.
+#pragma unroll
+        for (int c = 0; c < BN / 64; ++c) tmem_st32(t_s + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[c * 32]));
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.p_full[buf]);
+      }
+      // Epilogue: wait for the last PV, normalise, store.
+      if (!wait_bar_warp(&bars.o_full, (g - 1) & 1, ab)) goto softmax_done;
+      tc_fence_after();
+      {
+        const float inv = (l > 0.f) ? 1.f / l : 0.f;
+        const uint32_t t_o = tmem + lane_base + L::kOCol;
+        uint4* o_g = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + orow * D);
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(t_o + c * 32, o);
+          tmem_wait_ld();
+          if (row_ok) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(o[8 * e + 0]) * inv, __uint_as_float(o[8 * e + 1]) * inv);
+              w.y = pack_bf16x2(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv);
+              w.z = pack_bf16x2(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv);
+              w.w = pack_bf16x2(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv);
+              o_g[c * 4 + e] = w;
+            }
+          }
+        }
+        if (row_ok)
+          a.lse[static_cast<size_t>(it.h) * a.total_q + it.s.q0 + r] =
+              (l > 0.f) ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.o_empty);
+      ++nq;
+    }
+  softmax_done:;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D, bool CAUSAL>
+cudaError_t launch_one(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       cudaStream_t stream) {
+  using L = FwdSmem<D>;
+  auto kern = fwd_kernel<D, CAUSAL>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  if (e != cudaSuccess) return e;
+  kern<<<a.grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       cudaStream_t stream) {
+  if (a.D == 64) return a.causal ? launch_one<64, true>(a, tq, tk, tv, stream) : launch_one<64, false>(a, tq, tk, tv, stream);
+  return a.causal ? launch_one<128, true>(a, tq, tk, tv, stream) : launch_one<128, false>(a, tq, tk, tv, stream);
+}
+
+}  // namespace fa

@@ -1,0 +1,68 @@
+// fa_kernels.h -- host-side launchers of the library's kernels (private to
+// libfa_varlen.so; the public interface is include/fa_varlen.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace fa {
+
+// Work-list preparation (one CTA): validates the cumulative offsets, counts
+// the (sequence, tile) pairs and writes them longest-first into the
+// workspace. mode 0: forward query tiles; mode 1: backward key tiles.
+struct SchedArgs {
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int batch, total_q, total_k, max_seqlen_q, max_seqlen_k;
+  int causal;
+  int mode;
+  void* workspace;
+  size_t seq_off_offset, pairs_offset;
+  int max_pairs;
+};
+cudaError_t launch_sched_prep(const SchedArgs& a, cudaStream_t stream);
+
+struct FwdArgs {
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  void* out;         // bf16 [total_q, H, D]
+  float* lse;        // fp32 [H, total_q]
+  void* workspace;   // header + pairs
+  size_t pairs_offset;
+  int H, D, total_q;
+  int causal;
+  float scale_log2;  // softmax_scale * log2(e)
+  int grid;          // persistent CTAs
+};
+// tm_q / tm_k / tm_v: 2-D maps over [rows, H*D] bf16, box 128 rows x 64
+// columns, 128-byte swizzle.
+cudaError_t launch_fwd(const FwdArgs& a, const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                       cudaStream_t stream);
+
+struct BwdArgs {
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  const void* dout;   // bf16 [total_q, H, D]
+  const void* out;    // bf16 [total_q, H, D]
+  const float* lse;   // fp32 [H, total_q]
+  void* dq;           // bf16 [total_q, H, D]
+  void* dk;           // bf16 [total_k, H, D]
+  void* dv;           // bf16 [total_k, H, D]
+  void* workspace;
+  size_t pairs_offset, dvec_offset, dqacc_offset;
+  int tq_pad;
+  int H, D, total_q, total_k;
+  int causal;
+  float scale;        // softmax_scale
+  float scale_log2;   // softmax_scale * log2(e)
+  int grid;
+};
+// Preprocess (rowsum(dO*O), zero the dQ accumulator), main backward, dQ
+// conversion. tm_q / tm_do: box 64 rows x 64 columns; tm_k / tm_v: box 128
+// rows x 64 columns; all 128-byte swizzle.
+cudaError_t launch_bwd(const BwdArgs& a, const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                       const CUtensorMap& tm_do, cudaStream_t stream);
+
+}  // namespace fa

@@ -1,0 +1,155 @@
+"""Python binding of libfa_varlen.so (include/fa_varlen.h).
+
+Argument marshalling only: every step of the attention runs in the CUDA
+kernels of the library. PyTorch provides device memory and the stream. If the
+library is missing, importing this module raises; there is no fallback.
+
+    out, lse = fa_varlen_fwd(q, k, v, cu_q, cu_k, max_q, max_k, scale, causal)
+    dq, dk, dv = fa_varlen_bwd(dout, q, k, v, out, lse, cu_q, cu_k, max_q, max_k,
+                               scale, causal)
+
+q, k, v, dout: bf16 CUDA tensors [total_tokens, heads, head_dim], contiguous.
+cu_q, cu_k: int32 CUDA tensors [batch + 1] of cumulative offsets.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfa_varlen.so")
+
+FA_OK = 0
+STATUS_NAMES = {
+    0: "FA_OK", 1: "FA_ERR_INVALID_ARGUMENT", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_WORKSPACE",
+    4: "FA_ERR_CUDA", 5: "FA_ERR_BAD_SEQLENS", 6: "FA_ERR_DEVICE_TIMEOUT",
+}
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m varlen_flashattention_02_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.fa_varlen_fwd_workspace_size.argtypes = [I, I, I, I]
+    lib.fa_varlen_fwd_workspace_size.restype = S
+    lib.fa_varlen_bwd_workspace_size.argtypes = [I, I, I, I, I]
+    lib.fa_varlen_bwd_workspace_size.restype = S
+    lib.fa_varlen_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, ctypes.c_float, I, P, P, P, S, P]
+    lib.fa_varlen_fwd.restype = I
+    lib.fa_varlen_bwd.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, ctypes.c_float, I,
+                                  P, P, P, P, S, P]
+    lib.fa_varlen_bwd.restype = I
+    lib.fa_get_device_status.argtypes = [P, P]
+    lib.fa_get_device_status.restype = I
+    lib.fa_status_string.argtypes = [I]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    return lib
+
+
+lib = _load()
+
+EXPORTED = ("fa_varlen_fwd_workspace_size", "fa_varlen_bwd_workspace_size", "fa_varlen_fwd",
+            "fa_varlen_bwd", "fa_get_device_status", "fa_status_string")
+
+
+def _p(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_qkv(name, t, H=None, D=None):
+    if t.dtype != torch.bfloat16 or t.dim() != 3 or not t.is_contiguous() or not t.is_cuda:
+        raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor [tokens, heads, head_dim]")
+    if H is not None and (t.shape[1] != H or t.shape[2] != D):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected [*, {H}, {D}]")
+
+
+def _check_cu(name, t):
+    if t.dtype != torch.int32 or t.dim() != 1 or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous int32 CUDA tensor [batch + 1]")
+
+
+def fwd_workspace_size(batch: int, total_q: int, heads: int, head_dim: int) -> int:
+    return int(lib.fa_varlen_fwd_workspace_size(batch, total_q, heads, head_dim))
+
+
+def bwd_workspace_size(batch: int, total_q: int, total_k: int, heads: int, head_dim: int) -> int:
+    return int(lib.fa_varlen_bwd_workspace_size(batch, total_q, total_k, heads, head_dim))
+
+
+def new_workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def fa_varlen_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                  softmax_scale: float, causal: bool, out=None, softmax_lse=None, workspace=None,
+                  stream=None):
+    """Forward. Returns (out bf16 [Tq,H,D], softmax_lse fp32 [H,Tq])."""
+    _check_qkv("q", q)
+    Tq, H, D = q.shape
+    _check_qkv("k", k, H, D)
+    _check_qkv("v", v, H, D)
+    _check_cu("cu_seqlens_q", cu_seqlens_q)
+    _check_cu("cu_seqlens_k", cu_seqlens_k)
+    batch = cu_seqlens_q.numel() - 1
+    if out is None:
+        out = torch.empty_like(q)
+    if softmax_lse is None:
+        softmax_lse = torch.empty((H, Tq), dtype=torch.float32, device=q.device)
+    need = fwd_workspace_size(batch, Tq, H, D)
+    if workspace is None:
+        workspace = new_workspace(need, q.device)
+    rc = lib.fa_varlen_fwd(_p(q), _p(k), _p(v), _p(cu_seqlens_q), _p(cu_seqlens_k), batch, Tq,
+                           k.shape[0], int(max_seqlen_q), int(max_seqlen_k), H, D,
+                           float(softmax_scale), int(bool(causal)), _p(out), _p(softmax_lse),
+                           _p(workspace), workspace.numel(), _stream(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_varlen_fwd")
+    return out, softmax_lse
+
+
+def fa_varlen_bwd(dout, q, k, v, out, softmax_lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
+                  max_seqlen_k: int, softmax_scale: float, causal: bool, dq=None, dk=None, dv=None,
+                  workspace=None, stream=None):
+    """Backward of sum(out * dout). Returns (dq, dk, dv), bf16, shaped like q, k, v."""
+    _check_qkv("q", q)
+    Tq, H, D = q.shape
+    for name, t in (("k", k), ("v", v), ("dout", dout), ("out", out)):
+        _check_qkv(name, t, H, D)
+    _check_cu("cu_seqlens_q", cu_seqlens_q)
+    _check_cu("cu_seqlens_k", cu_seqlens_k)
+    batch = cu_seqlens_q.numel() - 1
+    Tk = k.shape[0]
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = bwd_workspace_size(batch, Tq, Tk, H, D)
+    if workspace is None:
+        workspace = new_workspace(need, q.device)
+    rc = lib.fa_varlen_bwd(_p(dout), _p(q), _p(k), _p(v), _p(out), _p(softmax_lse), _p(cu_seqlens_q),
+                           _p(cu_seqlens_k), batch, Tq, Tk, int(max_seqlen_q), int(max_seqlen_k), H, D,
+                           float(softmax_scale), int(bool(causal)), _p(dq), _p(dk), _p(dv),
+                           _p(workspace), workspace.numel(), _stream(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_varlen_bwd")
+    return dq, dk, dv
+
+
+def device_status(workspace, stream=None) -> int:
+    """Synchronise the stream and return the device status word of the last
+    call that used this workspace."""
+    return int(lib.fa_get_device_status(_p(workspace), _stream(stream)))
