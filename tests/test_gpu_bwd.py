@@ -1,0 +1,106 @@
+"""GPU parity of the backward against the fp64 oracle. The GPU backward is fed
+the GPU forward's own out and logsumexp (as a training step would); the
+oracle recomputes everything from the bf16 inputs alone."""
+import numpy as np
+import pytest
+
+import oracle
+from tests import parity_util as pu
+from varlen_flashattention_02_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    ("one-tile", [100], [100], 2, 128),
+    ("tails-63-64-65-127-128-129-1", [63, 64, 65, 127, 128, 129, 1], [63, 64, 65, 127, 128, 129, 1], 2, 128),
+    ("lq-ne-lk", [200, 64, 300, 17], [300, 64, 130, 250], 2, 64),
+    ("empty-and-one", [0, 5, 1, 0, 130, 3], [3, 0, 1, 0, 257, 300], 2, 128),
+    ("multi-tile-ragged", [513, 260, 384], [513, 260, 384], 2, 64),
+    ("long-ragged", [1000, 45], [1000, 45], 1, 128),
+]
+
+
+def _run_bwd(w):
+    from varlen_flashattention_02_b200 import fa_varlen
+
+    (q, k, v), out, lse = pu.run_fwd(w)
+    do = pu.to_dev(w.tensors()["dout"])
+    dq, dk, dv = fa_varlen.fa_varlen_bwd(do, q, k, v, out, lse, pu.cu_dev(w.cu_q), pu.cu_dev(w.cu_k),
+                                         w.max_seqlen_q, w.max_seqlen_k, w.scale, w.causal)
+    return dq, dk, dv
+
+
+def _check(name, got, want, mask=None):
+    g = pu.bf16_dev_to_f64(got)
+    if mask is not None:
+        g, want = g[mask], want[mask]
+    assert np.all(np.isfinite(g)), f"{name}: non-finite"
+    err = pu.rel_l2(g, want)
+    assert err <= pu.GRAD_REL_L2, f"{name} rel-L2 {err:.3e} > {pu.GRAD_REL_L2}"
+    return err
+
+
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_bwd_small(case, causal):
+    name, lq, lk, H, D = case
+    w = synth.make_workload(name, lq, lk, heads=H, head_dim=D, causal=causal, seed=201 + len(lq))
+    dq, dk, dv = _run_bwd(w)
+    t = w.tensors()
+    rq, rk, rv = oracle.bwd(t["q"], t["k"], t["v"], t["dout"], w.cu_q, w.cu_k, w.scale, w.causal)
+    _check("dq", dq, rq)
+    _check("dk", dk, rk)
+    _check("dv", dv, rv)
+    # Entries the mathematics fixes exactly: zero gradients where nothing is visible.
+    g = pu.bf16_dev_to_f64(dq)
+    assert np.all(g[rq == 0.0] == 0.0)
+    gk, gv = pu.bf16_dev_to_f64(dk), pu.bf16_dev_to_f64(dv)
+    assert np.all(gk[rk == 0.0] == 0.0) and np.all(gv[rv == 0.0] == 0.0)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_bwd_full_size_sampled(D):
+    """The fwd+bwd workload (16384 tokens, lengths U{512..8192}, 16 heads,
+    causal) at full size in the benchmark's launch configuration; whole
+    (sequence, head) units of the shortest sequences are checked against the
+    oracle and every gradient is checked to be finite."""
+    import torch
+
+    w = synth.standard_workload(5)
+    if D != w.head_dim:
+        w = synth.make_workload(w.name + f"-d{D}", np.diff(w.cu_q), heads=w.heads, head_dim=D, causal=True,
+                                seed=w.seed)
+    dq, dk, dv = _run_bwd(w)
+    lens = np.diff(w.cu_q)
+    short = [int(b) for b in np.argsort(lens, kind="stable")[:2]]
+    units = [(b, h) for b in short for h in (0, w.heads - 1)]
+    t = w.tensors()
+    rq, rk, rv = oracle.bwd(t["q"], t["k"], t["v"], t["dout"], w.cu_q, w.cu_k, w.scale, w.causal, units=units)
+    for b, h in units:
+        sq = slice(int(w.cu_q[b]), int(w.cu_q[b + 1]))
+        sk = slice(int(w.cu_k[b]), int(w.cu_k[b + 1]))
+        _check(f"dq[{b},{h}]", dq[sq, h], rq[sq, h])
+        _check(f"dk[{b},{h}]", dk[sk, h], rk[sk, h])
+        _check(f"dv[{b},{h}]", dv[sk, h], rv[sk, h])
+    for x in (dq, dk, dv):
+        assert bool(torch.isfinite(x.float()).all())
+
+
+def test_bwd_gradient_sums():
+    """Properties that hold at any size: per (sequence, head), the rows of dS
+    sum to zero so sum_j dK_j = 0, and the rows of P sum to one so
+    sum_j dV_j = sum_i dO_i (every query row of a causal lq == lk sequence
+    sees at least one key)."""
+    import torch
+
+    w = synth.make_workload("sums", [700, 300, 1024], heads=2, head_dim=128, causal=True, seed=9)
+    dq, dk, dv = _run_bwd(w)
+    do = torch.from_numpy(synth.bf16_bits_to_f32(w.tensors()["dout"])).double()
+    for b in range(w.batch):
+        sk = slice(int(w.cu_k[b]), int(w.cu_k[b + 1]))
+        sq = slice(int(w.cu_q[b]), int(w.cu_q[b + 1]))
+        dvs = dv[sk].double().sum(0).cpu()
+        dos = do[sq].sum(0)
+        assert float((dvs - dos).norm() / dos.norm()) < 2e-2
+        dks = dk[sk].double().sum(0).cpu()
+        assert float(dks.norm() / dk[sk].double().norm().cpu()) < 5e-2

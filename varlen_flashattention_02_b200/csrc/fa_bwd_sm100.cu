@@ -1,8 +1,551 @@
+// fa_bwd_sm100.cu -- backward varlen attention for sm_100a.
+//
+// Three kernels per call, after the work-list preparation (key-tile mode):
+//  1. preprocess: Dv_i = sum_c dO_ic * O_ic (fp32, [H, rows]) and zero the
+//     fp32 dQ accumulator;
+//  2. main: one persistent CTA per SM walks (sequence, head, key-tile)
+//     items, longest first. For 128 keys K_j, V_j of one head it loops over
+//     the 64-row query tiles that see them, recomputing the probabilities
+//     from the saved logsumexp instead of storing them:
+//        S^T  = K_j Q_i^T,  P^T = exp2(S^T*scale*log2e - lse_i*log2e)
+//        dP^T = V_j dO_i^T, dS^T = P^T * (dP^T - Dv_i)
+//        dV_j += P^T dO_i,  dK_j += dS^T Q_i      (accumulated in TMEM)
+//        dQ_i^T = K_j^T dS^T -> added to the fp32 accumulator in global
+//                               memory with bulk reductions
+//     and finally writes dK_j = scale * dK_j and dV_j as bf16;
+//  3. convert: dQ = bf16(scale * dQacc).
+//
+// Pages: "Flash-Atención y Flash-Atención-2", FlashAttention v1 section
+// (tiling and recomputation: probabilities are recomputed in the backward)
+// and backward paragraph (each worker owns a block of columns of the
+// attention matrix, i.e. a key tile; workers aggregate the query gradient
+// with atomic operations, which beats row parallelism that would have to
+// aggregate dK and dV); "Mecanismo cu_seqlens en FlashAttention" (per-
+// sequence offsets and lengths from the cumulative arrays). The gradient
+// formulas are the chain rule of softmax attention (the pages print none).
+//
+// B200 design: persistent longest-first scheduling; warp specialisation
+// (warp 0 TMA, warp 1 MMA issue, warps 2-3 stage logsumexp/Dv rows,
+// warps 4-7 compute P^T and dS^T with one thread per key row, warps 8-11
+// drain dQ^T from TMEM into bulk fp32 reductions and write dK/dV); dK, dV
+// and the per-step S^T, dP^T tiles live in TMEM (S^T and dP^T double-
+// buffered so the next step's QK^T overlaps this step's softmax); P^T goes
+// back to TMEM as bf16 and feeds the dV MMA directly; dS^T is written once to
+// shared memory in a layout that serves both the dK MMA (K-major A) and the
+// dQ^T MMA (MN-major B).
 #include "fa_common.cuh"
 #include "fa_kernels.h"
+
 namespace fa {
-cudaError_t launch_bwd(const BwdArgs&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                       const CUtensorMap&, cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+constexpr int BN = kBwdBN;  // keys per item
+constexpr int BM = kBwdBM;  // queries per step
+constexpr int kThreads = 384;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kColDK = 0, kColDV = 128, kColS = 256, kColDP = 384;  // TMEM column map
+
+template <int D>
+struct BwdSmem {
+  static constexpr int kChunks = D / 64;
+  static constexpr int kKChunk = BN * 128;  // [128 rows x 64 bf16] swizzled chunk
+  static constexpr int kQChunk = BM * 128;  // [ 64 rows x 64 bf16]
+  static constexpr int kKTile = kChunks * kKChunk;
+  static constexpr int kQTile = kChunks * kQChunk;
+  static constexpr int kDsTile = BN * BM * 2;  // dS^T [128 keys x 64 queries] bf16
+  static constexpr int kK = 0;
+  static constexpr int kV = kK + kKTile;
+  static constexpr int kQdo = kV + kKTile;  // stage s: Q at kQdo + 2s*QTile, dO after it
+  static constexpr int kDs = kQdo + 4 * kQTile;
+  static constexpr int kStage = kDs + 2 * kDsTile;   // fp32 dQ [64 x D]
+  static constexpr int kLd = kStage + BM * D * 4;    // 2 slots x (lse[64], dv[64]) fp32
+  static constexpr int kBar = kLd + 2 * 2 * BM * 4;
+  static constexpr int kBytes = kBar + 512;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+struct Bars {
+  uint64_t kv_full, kv_empty;
+  uint64_t qdo_full[2], qdo_empty[2];
+  uint64_t st_full[2];
+  uint64_t ds_full[2], ds_empty[2];
+  uint64_t dq_full[2], dq_empty[2];
+  uint64_t dkv_full, dkv_empty;
+  uint64_t ld_full[2], ld_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+static_assert(sizeof(Bars) <= 512, "barrier block fits its reserved space");
+
+struct Item {
+  int b, h, j;
+  SeqInfo s;
+  int i0, n;  // first query tile and number of steps
+};
+
+__device__ __forceinline__ Item get_item(const BwdArgs& a, const int2* pairs, int idx) {
+  Item it;
+  const int2 pr = pairs[idx / a.H];
+  it.h = idx % a.H;
+  it.b = pr.x;
+  it.j = pr.y;
+  it.s = seq_info(a.cu_q, a.cu_k, it.b);
+  int e;
+  bwd_q_tiles(it.j, it.s.lq, it.s.lk, a.causal != 0, &it.i0, &e);
+  it.n = e - it.i0;
+  return it;
 }
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+               const BwdArgs a) {
+  using L = BwdSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars& bars = *reinterpret_cast<Bars*>(smem + L::kBar);
+  auto* hdr = reinterpret_cast<WsHeader*>(a.workspace);
+  const int2* pairs = reinterpret_cast<const int2*>(static_cast<const char*>(a.workspace) + a.pairs_offset);
+  const float* dvec = reinterpret_cast<const float*>(static_cast<const char*>(a.workspace) + a.dvec_offset);
+  float* dqacc = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + a.dqacc_offset);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars.kv_full, 1);
+    mbar_init(&bars.kv_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.qdo_full[i], 1);
+      mbar_init(&bars.qdo_empty[i], 1);
+      mbar_init(&bars.st_full[i], 1);
+      mbar_init(&bars.ds_full[i], 4);
+      mbar_init(&bars.ds_empty[i], 1);
+      mbar_init(&bars.dq_full[i], 1);
+      mbar_init(&bars.dq_empty[i], 4);
+      mbar_init(&bars.ld_full[i], 2);
+      mbar_init(&bars.ld_empty[i], 4);
+    }
+    mbar_init(&bars.dkv_full, 1);
+    mbar_init(&bars.dkv_empty, 4);
+    mbar_init(&bars.drain, 1);
+    bars.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_do);
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars.tmem_base;
+  const Abort ab{&bars.abort_flag, &hdr->status};
+  const int n_items = (hdr->status == FA_OK) ? static_cast<int>(hdr->n_pairs) * a.H : 0;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- producer
+      uint32_t m = 0, p = 0;
+      for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+        const Item it = get_item(a, pairs, idx);
+        if (it.n == 0) continue;
+        if (m > 0 && !wait_bar(&bars.kv_empty, (m - 1) & 1, ab)) goto producer_done;
+        const int krow = it.s.k0 + it.j * BN;
+        mbar_arrive_expect_tx(&bars.kv_full, 2 * L::kKTile);
+        for (int c = 0; c < L::kChunks; ++c) {
+          tma_load_2d(&tm_k, &bars.kv_full, smem + L::kK + c * L::kKChunk, it.h * D + c * 64, krow);
+          tma_load_2d(&tm_v, &bars.kv_full, smem + L::kV + c * L::kKChunk, it.h * D + c * 64, krow);
+        }
+        for (int s = 0; s < it.n; ++s, ++p) {
+          const int st = p & 1;
+          if (p >= 2 && !wait_bar(&bars.qdo_empty[st], ((p >> 1) - 1) & 1, ab)) goto producer_done;
+          const int qrow = it.s.q0 + (it.i0 + s) * BM;
+          uint8_t* sq = smem + L::kQdo + 2 * st * L::kQTile;
+          uint8_t* sdo = sq + L::kQTile;
+          mbar_arrive_expect_tx(&bars.qdo_full[st], 2 * L::kQTile);
+          for (int c = 0; c < L::kChunks; ++c) {
+            tma_load_2d(&tm_q, &bars.qdo_full[st], sq + c * L::kQChunk, it.h * D + c * 64, qrow);
+            tma_load_2d(&tm_do, &bars.qdo_full[st], sdo + c * L::kQChunk, it.h * D + c * 64, qrow);
+          }
+        }
+        ++m;
+      }
+    producer_done:
+      if (m > 0) wait_bar(&bars.kv_full, (m - 1) & 1, ab);
+      for (uint32_t i = (p > 2 ? p - 2 : 0); i < p; ++i) wait_bar(&bars.qdo_full[i & 1], (i >> 1) & 1, ab);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      constexpr uint32_t kIdS = idesc_bf16_f32(BN, BM, false, false);   // S^T, dP^T: 128 x 64, K = D
+      constexpr uint32_t kIdKV = idesc_bf16_f32(BN, D, false, true);    // dV, dK: 128 x D, K = 64
+      constexpr uint32_t kIdQ = idesc_bf16_f32(128, BM, true, true);    // dQ^T: 128 (>= D) x 64, K = 128
+      const uint32_t sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
+      uint32_t m = 0, p = 0;
+      for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+        const Item it = get_item(a, pairs, idx);
+        if (it.n == 0) continue;
+        if (!wait_bar(&bars.kv_full, m & 1, ab)) goto mma_done;
+        tc_fence_after();
+        for (int s = 0; s <= it.n; ++s) {
+          if (s < it.n) {
+            const uint32_t ps = p + s;
+            const int st = ps & 1;
+            if (!wait_bar(&bars.qdo_full[st], (ps >> 1) & 1, ab)) goto mma_done;
+            if (ps >= 2 && !wait_bar(&bars.dq_empty[st], ((ps >> 1) - 1) & 1, ab)) goto mma_done;
+            tc_fence_after();
+            const uint32_t sq = smem_u32(smem + L::kQdo + 2 * st * L::kQTile);
+            const uint32_t sdo = sq + L::kQTile;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t oa = (kk >> 2) * L::kKChunk + (kk & 3) * 32;
+              const uint32_t ob = (kk >> 2) * L::kQChunk + (kk & 3) * 32;
+              mma_ss(tmem + kColS + st * BM, smem_desc_sw128(sK + oa, 16, 1024), smem_desc_sw128(sq + ob, 16, 1024),
+                     kIdS, kk > 0);
+            }
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t oa = (kk >> 2) * L::kKChunk + (kk & 3) * 32;
+              const uint32_t ob = (kk >> 2) * L::kQChunk + (kk & 3) * 32;
+              mma_ss(tmem + kColDP + st * BM, smem_desc_sw128(sV + oa, 16, 1024),
+                     smem_desc_sw128(sdo + ob, 16, 1024), kIdS, kk > 0);
+            }
+            mma_commit(&bars.st_full[st]);
+          }
+          if (s > 0) {
+            const uint32_t pp = p + s - 1;
+            const int pb = pp & 1;
+            if (!wait_bar(&bars.ds_full[pb], (pp >> 1) & 1, ab)) goto mma_done;
+            if (s == 1 && m > 0 && !wait_bar(&bars.dkv_empty, (m - 1) & 1, ab)) goto mma_done;
+            tc_fence_after();
+            const uint32_t sq = smem_u32(smem + L::kQdo + 2 * pb * L::kQTile);
+            const uint32_t sdo = sq + L::kQTile;
+            const uint32_t sds = smem_u32(smem + L::kDs + pb * L::kDsTile);
+            const uint32_t acc = (s > 1) ? 1u : 0u;
+            // dV += P^T dO (P^T from TMEM, dO MN-major); dK += dS^T Q.
+#pragma unroll
+            for (int kk = 0; kk < BM / 16; ++kk) {
+              mma_ts(tmem + kColDV, tmem + kColS + pb * BM + kk * 8,
+                     smem_desc_sw128(sdo + kk * 2048, L::kQChunk, 1024), kIdKV, (acc | kk) ? 1u : 0u);
+            }
+#pragma unroll
+            for (int kk = 0; kk < BM / 16; ++kk) {
+              mma_ss(tmem + kColDK, smem_desc_sw128(sds + kk * 32, 16, 1024),
+                     smem_desc_sw128(sq + kk * 2048, L::kQChunk, 1024), kIdKV, (acc | kk) ? 1u : 0u);
+            }
+            // dQ^T = K^T dS^T into the dP^T columns of this step.
+#pragma unroll
+            for (int kk = 0; kk < BN / 16; ++kk) {
+              mma_ss(tmem + kColDP + pb * BM, smem_desc_sw128(sK + kk * 2048, D == 128 ? L::kKChunk : 0, 1024),
+                     smem_desc_sw128(sds + kk * 2048, 0, 1024), kIdQ, kk > 0);
+            }
+            mma_commit(&bars.dq_full[pb]);
+            mma_commit(&bars.qdo_empty[pb]);
+            mma_commit(&bars.ds_empty[pb]);
+          }
+        }
+        mma_commit(&bars.dkv_full);
+        mma_commit(&bars.kv_empty);
+        p += it.n;
+        ++m;
+      }
+    mma_done:
+      mma_commit(&bars.drain);
+      wait_bar(&bars.drain, 0, ab);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ lse / Dv rows
+    const int r = threadIdx.x - 64;  // query row within the tile, 0..63
+    uint32_t p = 0;
+    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+      const Item it = get_item(a, pairs, idx);
+      for (int s = 0; s < it.n; ++s, ++p) {
+        const int slot = p & 1;
+        if (p >= 2 && !wait_bar_warp(&bars.ld_empty[slot], ((p >> 1) - 1) & 1, ab)) goto loader_done;
+        const int qi = (it.i0 + s) * BM + r;  // row within the sequence
+        float lse2 = INFINITY, dv = 0.f;      // +inf logsumexp => P = 0 for rows outside the sequence
+        if (qi < it.s.lq) {
+          const size_t gq = static_cast<size_t>(it.s.q0) + qi;
+          const float l = __ldg(a.lse + static_cast<size_t>(it.h) * a.total_q + gq);
+          if (l != -INFINITY) {
+            lse2 = l * 1.4426950408889634f;
+            dv = __ldg(dvec + static_cast<size_t>(it.h) * a.tq_pad + gq);
+          }
+        }
+        float* ld = reinterpret_cast<float*>(smem + L::kLd) + slot * 2 * BM;
+        ld[r] = lse2;
+        ld[BM + r] = dv;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.ld_full[slot]);
+      }
+    }
+  loader_done:;
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ P^T, dS^T
+    const int kr = threadIdx.x - 128;  // key row in the tile == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    uint32_t p = 0;
+    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+      const Item it = get_item(a, pairs, idx);
+      const int kg = it.j * BN + kr;  // key index within the sequence
+      const bool key_ok = kg < it.s.lk;
+      const int diag = it.s.lk - it.s.lq;
+      for (int s = 0; s < it.n; ++s, ++p) {
+        const int pb = p & 1;
+        if (!wait_bar_warp(&bars.st_full[pb], (p >> 1) & 1, ab)) goto compute_done;
+        if (!wait_bar_warp(&bars.ld_full[pb], (p >> 1) & 1, ab)) goto compute_done;
+        if (p >= 2 && !wait_bar_warp(&bars.ds_empty[pb], ((p >> 1) - 1) & 1, ab)) goto compute_done;
+        tc_fence_after();
+        const float* ld = reinterpret_cast<const float*>(smem + L::kLd) + pb * 2 * BM;
+        const int row0 = (it.i0 + s) * BM;  // first query row of the step
+        // Visible iff kg <= row + diag, i.e. e >= kg - diag - row0; keys past
+        // the sequence see nothing.
+        int e_min = CAUSAL ? kg - diag - row0 : 0;
+        if (!key_ok) e_min = BM;
+        uint8_t* ds_row = smem + L::kDs + pb * L::kDsTile + kr * 128;
+#pragma unroll
+        for (int c = 0; c < BM / 32; ++c) {
+          uint32_t sv[32], dpv[32];
+          tmem_ld32(tmem + lane_base + kColS + pb * BM + c * 32, sv);
+          tmem_ld32(tmem + lane_base + kColDP + pb * BM + c * 32, dpv);
+          tmem_wait_ld();
+          uint32_t pk[16], dsk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int q = c * 32 + e;
+            float p0 = ex2_approx(fmaf(__uint_as_float(sv[e]), a.scale_log2, -ld[q]));
+            float p1 = ex2_approx(fmaf(__uint_as_float(sv[e + 1]), a.scale_log2, -ld[q + 1]));
+            if (q < e_min) p0 = 0.f;
+            if (q + 1 < e_min) p1 = 0.f;
+            const float d0 = p0 * (__uint_as_float(dpv[e]) - ld[BM + q]);
+            const float d1 = p1 * (__uint_as_float(dpv[e + 1]) - ld[BM + q + 1]);
+            pk[e / 2] = pack_bf16x2(p0, p1);
+            dsk[e / 2] = pack_bf16x2(d0, d1);
+          }
+          // P^T (bf16 pairs) into the first 32 columns of this step's S^T.
+          tmem_st16(tmem + lane_base + kColS + pb * BM + c * 16, pk);
+          // dS^T row kr, queries c*32 .. c*32+31: four 16-byte chunks, 128-byte swizzle.
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int chunk = (c * 4 + u) ^ (kr & 7);
+            *reinterpret_cast<uint4*>(ds_row + chunk * 16) =
+                make_uint4(dsk[4 * u], dsk[4 * u + 1], dsk[4 * u + 2], dsk[4 * u + 3]);
+          }
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bars.ds_full[pb]);
+          mbar_arrive(&bars.ld_empty[pb]);
+        }
+      }
+    }
+  compute_done:;
+  } else {
+    // ------------------------------------------------------------ dQ drain, dK/dV
+    const int t = threadIdx.x - 256;  // 0..127: TMEM lane (d for dQ^T, key row for dK/dV)
+    const int q4 = warp & 3;
+    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    float* stage = reinterpret_cast<float*>(smem + L::kStage);
+    uint32_t p = 0, m = 0;
+    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+      const Item it = get_item(a, pairs, idx);
+      const int kg = it.j * BN + t;
+      const bool key_ok = kg < it.s.lk;
+      const size_t krow = (static_cast<size_t>(it.s.k0) + kg) * a.H + it.h;
+      if (it.n == 0) {
+        if (key_ok) {
+          uint4* dk = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.dk) + krow * D);
+          uint4* dv = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.dv) + krow * D);
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c) dk[c] = dv[c] = make_uint4(0, 0, 0, 0);
+        }
+        continue;
+      }
+      for (int s = 0; s < it.n; ++s, ++p) {
+        const int pb = p & 1;
+        if (!wait_bar_warp(&bars.dq_full[pb], (p >> 1) & 1, ab)) goto drain_done;
+        tc_fence_after();
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tmem + lane_base + kColDP + pb * BM, v0);
+        tmem_ld32(tmem + lane_base + kColDP + pb * BM + 32, v1);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.dq_empty[pb]);
+        // The previous bulk reduction must have finished reading the stage.
+        if (t == 0) bulk_wait_group_read0();
+        named_bar_sync(1, 128);
+        if (t < D) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) stage[e * D + t] = __uint_as_float(v0[e]);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) stage[(32 + e) * D + t] = __uint_as_float(v1[e]);
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (t == 0) {
+          const size_t q0 = static_cast<size_t>(it.s.q0) + static_cast<size_t>(it.i0 + s) * BM;
+          bulk_reduce_add_f32(dqacc + (static_cast<size_t>(it.h) * a.tq_pad + q0) * D, stage, BM * D * 4);
+          bulk_commit_group();
+        }
+      }
+      // dK, dV of this key tile.
+      if (!wait_bar_warp(&bars.dkv_full, m & 1, ab)) goto drain_done;
+      tc_fence_after();
+      {
+        uint4* dk = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.dk) + krow * D);
+        uint4* dv = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.dv) + krow * D);
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t x[32], y[32];
+          tmem_ld32(tmem + lane_base + kColDK + c * 32, x);
+          tmem_ld32(tmem + lane_base + kColDV + c * 32, y);
+          tmem_wait_ld();
+          if (key_ok) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              uint4 wk, wv;
+              wk.x = pack_bf16x2(__uint_as_float(x[8 * e + 0]) * a.scale, __uint_as_float(x[8 * e + 1]) * a.scale);
+              wk.y = pack_bf16x2(__uint_as_float(x[8 * e + 2]) * a.scale, __uint_as_float(x[8 * e + 3]) * a.scale);
+              wk.z = pack_bf16x2(__uint_as_float(x[8 * e + 4]) * a.scale, __uint_as_float(x[8 * e + 5]) * a.scale);
+              wk.w = pack_bf16x2(__uint_as_float(x[8 * e + 6]) * a.scale, __uint_as_float(x[8 * e + 7]) * a.scale);
+              wv.x = pack_bf16x2(__uint_as_float(y[8 * e + 0]), __uint_as_float(y[8 * e + 1]));
+              wv.y = pack_bf16x2(__uint_as_float(y[8 * e + 2]), __uint_as_float(y[8 * e + 3]));
+              wv.z = pack_bf16x2(__uint_as_float(y[8 * e + 4]), __uint_as_float(y[8 * e + 5]));
+              wv.w = pack_bf16x2(__uint_as_float(y[8 * e + 6]), __uint_as_float(y[8 * e + 7]));
+              dk[c * 4 + e] = wk;
+              dv[c * 4 + e] = wv;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.dkv_empty);
+      ++m;
+    }
+  drain_done:
+    // Bulk reductions still reading the stage must finish before exit.
+    if (t == 0) bulk_wait_group0();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Dv[h, r] = sum_c dO[r, h, c] * O[r, h, c] in fp32, and dQacc[h, r, :] = 0.
+// One warp per (row, head).
+template <int D>
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdArgs a) {
+  const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= static_cast<long long>(a.total_q) * a.H) return;
+  const int row = static_cast<int>(w / a.H), h = static_cast<int>(w % a.H);
+  const size_t base = static_cast<size_t>(w) * D;
+  constexpr int E = D / 32;  // bf16 elements per lane
+  const __nv_bfloat16* o = static_cast<const __nv_bfloat16*>(a.out) + base + lane * E;
+  const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(a.dout) + base + lane * E;
+  float acc = 0.f;
+  if constexpr (E == 4) {
+    const uint2 ov = *reinterpret_cast<const uint2*>(o), gv = *reinterpret_cast<const uint2*>(g);
+    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const float2 x = __bfloat1622float2(o2[i]), y = __bfloat1622float2(g2[i]);
+      acc = fmaf(x.x, y.x, acc);
+      acc = fmaf(x.y, y.y, acc);
+    }
+  } else {
+    const uint32_t ov = *reinterpret_cast<const uint32_t*>(o), gv = *reinterpret_cast<const uint32_t*>(g);
+    const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ov));
+    const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv));
+    acc = fmaf(x.x, y.x, acc);
+    acc = fmaf(x.y, y.y, acc);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  float* dvec = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + a.dvec_offset);
+  float* dqacc = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + a.dqacc_offset);
+  if (lane == 0) dvec[static_cast<size_t>(h) * a.tq_pad + row] = acc;
+  float4* z = reinterpret_cast<float4*>(dqacc + (static_cast<size_t>(h) * a.tq_pad + row) * D);
+  for (int i = lane; i < D / 4; i += 32) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// dQ[r, h, :] = bf16(scale * dQacc[h, r, :]). One warp per (row, head).
+template <int D>
+__global__ void __launch_bounds__(256) bwd_convert_kernel(const BwdArgs a) {
+  const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= static_cast<long long>(a.total_q) * a.H) return;
+  const int row = static_cast<int>(w / a.H), h = static_cast<int>(w % a.H);
+  const float* src = reinterpret_cast<const float*>(static_cast<const char*>(a.workspace) + a.dqacc_offset) +
+                     (static_cast<size_t>(h) * a.tq_pad + row) * D;
+  __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.dq) + static_cast<size_t>(w) * D;
+  constexpr int E = D / 32;
+  if constexpr (E == 4) {
+    const float4 v = reinterpret_cast<const float4*>(src)[lane];
+    uint2 o;
+    o.x = pack_bf16x2(v.x * a.scale, v.y * a.scale);
+    o.y = pack_bf16x2(v.z * a.scale, v.w * a.scale);
+    reinterpret_cast<uint2*>(dst)[lane] = o;
+  } else {
+    const float2 v = reinterpret_cast<const float2*>(src)[lane];
+    reinterpret_cast<uint32_t*>(dst)[lane] = pack_bf16x2(v.x * a.scale, v.y * a.scale);
+  }
+}
+
+template <int D, bool CAUSAL>
+cudaError_t launch_main(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const CUtensorMap& tdo, cudaStream_t stream) {
+  using L = BwdSmem<D>;
+  auto kern = bwd_kernel<D, CAUSAL>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  if (e != cudaSuccess) return e;
+  kern<<<a.grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, tdo, a);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_all(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, cudaStream_t stream) {
+  const long long warps = static_cast<long long>(a.total_q) * a.H;
+  const unsigned blocks = static_cast<unsigned>((warps + 7) / 8);
+  if (blocks > 0) {
+    bwd_preprocess_kernel<D><<<blocks, 256, 0, stream>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  cudaError_t e = a.causal ? launch_main<D, true>(a, tq, tk, tv, tdo, stream)
+                           : launch_main<D, false>(a, tq, tk, tv, tdo, stream);
+  if (e != cudaSuccess) return e;
+  if (blocks > 0) {
+    bwd_convert_kernel<D><<<blocks, 256, 0, stream>>>(a);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+}  // namespace
+
+cudaError_t launch_bwd(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, cudaStream_t stream) {
+  return a.D == 64 ? launch_all<64>(a, tq, tk, tv, tdo, stream) : launch_all<128>(a, tq, tk, tv, tdo, stream);
+}
+
 }  // namespace fa
