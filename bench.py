@@ -1,0 +1,495 @@
+#!/usr/bin/env python
+"""Benchmark of the varlen attention hot path on B200.
+
+One step = the whole path on one batch: work-list preparation, forward
+(out, logsumexp), then backward (preprocess, dQ/dK/dV, dQ conversion), on the
+fwd+bwd workload: 16384 packed tokens, lengths U{512..8192} (seed 5, last
+clipped), 16 heads, head_dim 128, causal, bf16 inputs ~N(0,1).
+
+FLOPs: F_fwd = 4 * sum_b lq_b * lk_b * heads * head_dim, halved for causal;
+backward = 2.5 * F_fwd; the headline fwd+bwd figure uses 3.5 * F_fwd (the
+literal 2.5 * F_fwd / step time is reported beside it, labelled).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs the same workload shape on its own
+seeded data (weak scaling, no collective on the data path); timing is the
+max over ranks. Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import random
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from varlen_flashattention_02_b200 import synth  # noqa: E402
+
+METRIC = "attention TFLOP/s (fwd, fwd+bwd) at 1 B200 and % of dense BF16 peak"
+UNIT = "TFLOP/s"
+WORKLOAD = ("varlen fwd+bwd: 16384 total tokens, lengths uniform int [512,8192] from seed 5 (last clipped), "
+            "16 heads, head_dim 128, bf16 Q/K/V/dO ~N(0,1), causal, LSE saved fwd, outputs dQ/dK/dV")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 256 << 20
+
+
+def fwd_flops(cu_q, cu_k, heads, head_dim, causal, units=None):
+    lq = np.diff(np.asarray(cu_q, dtype=np.int64))
+    lk = np.diff(np.asarray(cu_k, dtype=np.int64))
+    if units is None:
+        total = float(np.sum(lq * lk)) * heads
+    else:
+        total = float(sum(lq[b] * lk[b] for b, _ in units))
+    f = 4.0 * total * head_dim
+    return f / 2 if causal else f
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-f", self.path],
+                                         stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for ln in f:
+                parts = [x.strip() for x in ln.split(",")]
+                if len(parts) < 9:
+                    continue
+                if self.uuid and parts[0] != self.uuid:
+                    continue
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "", 1).isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "", 1).isdigit()]
+        reasons = sorted({name for r in rows for name, val in zip(self.REASONS, r[5:9]) if val == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------- our arm
+def kernel_traffic(kernel_file: str):
+    """Per-launch DRAM bytes of the dominant kernel from the committed ncu
+    summary, if it was taken on the current source of that kernel."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    src = os.path.join(ROOT, "varlen_flashattention_02_b200", "csrc", kernel_file)
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    ent = d.get(kernel_file)
+    if not ent or ent.get("source_sha256_16") != h:
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from varlen_flashattention_02_b200 import fa_varlen
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = synth.standard_workload(5)
+    w.seed = w.seed + 1000 * rank  # same shape, own data per rank
+    t = w.tensors()
+    H, D = w.heads, w.head_dim
+
+    def dev_bf16(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q, k, v, do = (dev_bf16(t[n]) for n in ("q", "k", "v", "dout"))
+    cu_q = torch.from_numpy(w.cu_q).to(dev)
+    cu_k = torch.from_numpy(w.cu_k).to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((H, w.total_q), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_f = fa_varlen.new_workspace(fa_varlen.fwd_workspace_size(w.batch, w.total_q, H, D), dev)
+    ws_b = fa_varlen.new_workspace(fa_varlen.bwd_workspace_size(w.batch, w.total_q, w.total_k, H, D), dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    lib = fa_varlen.lib
+
+    def fwd():
+        fa_varlen.fa_varlen_fwd(q, k, v, cu_q, cu_k, w.max_seqlen_q, w.max_seqlen_k, w.scale, w.causal,
+                                out=out, softmax_lse=lse, workspace=ws_f, stream=stream)
+
+    def bwd():
+        fa_varlen.fa_varlen_bwd(do, q, k, v, out, lse, cu_q, cu_k, w.max_seqlen_q, w.max_seqlen_k, w.scale,
+                                w.causal, dq=dq, dk=dk, dv=dv, workspace=ws_b, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        fwd()
+        bwd()
+    torch.cuda.synchronize(dev)
+    if fa_varlen.device_status(ws_f) != 0 or fa_varlen.device_status(ws_b) != 0:
+        raise RuntimeError("device status not OK after warm-up")
+
+    def mk():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)  # materialise the handle
+        return e
+
+    K = args.steps
+    step_ev = [(mk(), mk()) for _ in range(K)]
+    fwd_ev = [[mk() for _ in range(4)] for _ in range(K)]   # prep, attention
+    bwd_ev = [[mk() for _ in range(8)] for _ in range(K)]   # prep, preprocess, main, convert
+    import ctypes
+
+    fwd_arr = [(ctypes.c_void_p * 4)(*[e.cuda_event for e in evs]) for evs in fwd_ev]
+    bwd_arr = [(ctypes.c_void_p * 8)(*[e.cuda_event for e in evs]) for evs in bwd_ev]
+    torch.cuda.synchronize(dev)
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    wall0 = time.perf_counter()
+    for i in range(K):
+        flush.zero_()
+        step_ev[i][0].record(stream)
+        lib.fa_set_kernel_events(fwd_arr[i], 2)
+        fwd()
+        lib.fa_set_kernel_events(bwd_arr[i], 4)
+        bwd()
+        lib.fa_set_kernel_events(None, 0)
+        step_ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    wall1 = time.perf_counter()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    if fa_varlen.device_status(ws_f) != 0 or fa_varlen.device_status(ws_b) != 0:
+        raise RuntimeError("device status not OK after the timed steps")
+
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    fwd_call_ms = [evs[0].elapsed_time(evs[3]) for evs in fwd_ev]
+    fwd_kern_ms = [evs[2].elapsed_time(evs[3]) for evs in fwd_ev]
+    bwd_call_ms = [evs[0].elapsed_time(evs[7]) for evs in bwd_ev]
+    bwd_main_ms = [evs[4].elapsed_time(evs[5]) for evs in bwd_ev]
+    per_kernel = {
+        "sched_prep_fwd": statistics.mean(evs[0].elapsed_time(evs[1]) for evs in fwd_ev),
+        "fwd_attention": statistics.mean(fwd_kern_ms),
+        "sched_prep_bwd": statistics.mean(evs[0].elapsed_time(evs[1]) for evs in bwd_ev),
+        "bwd_preprocess": statistics.mean(evs[2].elapsed_time(evs[3]) for evs in bwd_ev),
+        "bwd_attention": statistics.mean(bwd_main_ms),
+        "bwd_dq_convert": statistics.mean(evs[6].elapsed_time(evs[7]) for evs in bwd_ev),
+    }
+    tot_ms = sum(step_ms)
+    if world > 1:
+        tm = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+        tot_ms = float(tm.item())
+    F = fwd_flops(w.cu_q, w.cu_k, H, D, w.causal)
+    ms_step = tot_ms / K
+    value = world * 3.5 * F / (ms_step * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers (pinned)
+    host_in = {n: torch.from_numpy(t[n].view(np.int16)).view(torch.bfloat16).pin_memory()
+               for n in ("q", "k", "v", "dout")}
+    host_cu = (torch.from_numpy(w.cu_q).pin_memory(), torch.from_numpy(w.cu_k).pin_memory())
+    host_out = [torch.empty(x.shape, dtype=torch.bfloat16).pin_memory() for x in (dq, dk, dv)]
+    h2d = sum(x.numel() * x.element_size() for x in host_in.values()) + sum(x.numel() * 4 for x in host_cu)
+    d2h = sum(x.numel() * x.element_size() for x in host_out)
+    e2e_steps = max(3, min(K, 10))
+    e2e_ev = [(mk(), mk()) for _ in range(e2e_steps)]
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    for i in range(e2e_steps):
+        flush.zero_()
+        e2e_ev[i][0].record(stream)
+        q.copy_(host_in["q"], non_blocking=True)
+        k.copy_(host_in["k"], non_blocking=True)
+        v.copy_(host_in["v"], non_blocking=True)
+        do.copy_(host_in["dout"], non_blocking=True)
+        cu_q.copy_(host_cu[0], non_blocking=True)
+        cu_k.copy_(host_cu[1], non_blocking=True)
+        fwd()
+        bwd()
+        host_out[0].copy_(dq, non_blocking=True)
+        host_out[1].copy_(dk, non_blocking=True)
+        host_out[2].copy_(dv, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / e2e_steps
+    if world > 1:
+        tm = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tm.item())
+        dist.barrier()
+    e2e = {"value": world * 3.5 * F / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    bwd_main = statistics.mean(bwd_main_ms)
+    achieved = 2.5 * F / (bwd_main * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "bwd_attention (fa_bwd_sm100.cu, bwd_kernel<128,causal>)",
+                "achieved": achieved, "peak": peak, "peak_source": f"{peak_src} bf16_tflops (burst)",
+                "unit": UNIT, "frac": achieved / peak,
+                "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
+                "traffic": kernel_traffic("fa_bwd_sm100.cu"),
+                "algorithmic": "2.5 * F_fwd FLOPs per launch (5 bf16 matmuls over visible tiles, causal halved)"}
+    fwd_k = statistics.mean(fwd_kern_ms)
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded bf16 N(0,1); lengths from numpy default_rng)",
+        "config": {"workload": WORKLOAD, "total_tokens": w.total_q, "batch": w.batch, "heads": H,
+                   "head_dim": D, "causal": True, "max_seqlen": w.max_seqlen_q,
+                   "flops_fwd": F, "flop_convention": "fwd+bwd = 3.5 * F_fwd (bwd = 2.5 * F_fwd); causal halved",
+                   "l2": "256 MiB buffer written between steps (and step inputs exceed L2)",
+                   "parallelism": f"weak: {world} independent replicas of the workload, no data-path collective"},
+        "fwd_tflops": F / (statistics.mean(fwd_call_ms) * 1e-3) / 1e12,
+        "bwd_tflops": 2.5 * F / (statistics.mean(bwd_call_ms) * 1e-3) / 1e12,
+        "fwd_bwd_tflops_literal_2p5": world * 2.5 * F / (ms_step * 1e-3) / 1e12,
+        "fwd_kernel_tflops": F / (fwd_k * 1e-3) / 1e12,
+        "pct_of_peak": {"fwd_bwd": 100 * value / world / peak,
+                        "fwd": 100 * F / (statistics.mean(fwd_call_ms) * 1e-3) / 1e12 / peak,
+                        "bwd": 100 * 2.5 * F / (statistics.mean(bwd_call_ms) * 1e-3) / 1e12 / peak,
+                        "denominator": f"{peak} TFLOP/s ({peak_src} bf16 burst)"},
+        "kernel_ms": per_kernel,
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": 6 * K,
+        "clocks": clocks,
+        "wall_s_timed_region": wall1 - wall0,
+    }
+    if rank == 0 and not args.no_aux:
+        result["fwd_by_workload"] = fwd_only_workloads(dev, stream, flush, peak)
+    return result, w
+
+
+def fwd_only_workloads(dev, stream, flush, peak, iters=10):
+    """Forward TFLOP/s of the other standard workloads (same launch path)."""
+    import torch
+
+    from varlen_flashattention_02_b200 import fa_varlen
+
+    res = {}
+    specs = [("varlen-2seq-h12-d64 (cu_q=[0,200,1024], cu_k=[0,300,1024])", 1, {}),
+             ("fixed-8x2048-h16-d128 non-causal", 2, {"causal": False}),
+             ("fixed-8x2048-h16-d128 causal", 2, {"causal": True}),
+             ("packed-16k-U128..4096-h32-d128 causal", 3, {}),
+             ("long-1x16384-h16-d64 causal", 4, {"head_dim": 64}),
+             ("long-1x16384-h16-d128 causal", 4, {"head_dim": 128})]
+    for name, n, kw in specs:
+        w = synth.standard_workload(n, **kw)
+        t = w.tensors()
+        mk = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)
+        q, k, v = mk(t["q"]), mk(t["k"]), mk(t["v"])
+        cq, ck = torch.from_numpy(w.cu_q).to(dev), torch.from_numpy(w.cu_k).to(dev)
+        out = torch.empty_like(q)
+        lse = torch.empty((w.heads, w.total_q), dtype=torch.float32, device=dev)
+        ws = fa_varlen.new_workspace(fa_varlen.fwd_workspace_size(w.batch, w.total_q, w.heads, w.head_dim), dev)
+        call = lambda: fa_varlen.fa_varlen_fwd(q, k, v, cq, ck, w.max_seqlen_q, w.max_seqlen_k, w.scale,
+                                               w.causal, out=out, softmax_lse=lse, workspace=ws, stream=stream)
+        for _ in range(3):
+            call()
+        evs = []
+        for _ in range(iters):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            call()
+            b.record(stream)
+            evs.append((a, b))
+        torch.cuda.synchronize(dev)
+        ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+        F = fwd_flops(w.cu_q, w.cu_k, w.heads, w.head_dim, w.causal)
+        res[name] = {"ms": ms, "tflops": F / (ms * 1e-3) / 1e12, "pct_of_peak": 100 * F / (ms * 1e-3) / 1e12 / peak}
+        del q, k, v, out, lse, ws
+    return res
+
+
+# ------------------------------------------------------------- oracle (CPU)
+def oracle_sample(w, budget_s: float, seed: int = 0):
+    """Pick (sequence, head) units of ``w`` whose oracle fwd+bwd takes about
+    ``budget_s`` on this host, calibrated on a first small batch."""
+    import oracle
+
+    t = w.tensors()
+    cores = oracle.num_threads()
+    rng = random.Random(seed)
+    units = [(b, h) for b in range(w.batch) for h in range(w.heads)]
+    rng.shuffle(units)
+    lens = np.diff(w.cu_q)
+    shortest = int(np.argmin(lens))
+    calib = [(shortest, h % w.heads) for h in range(max(cores, 1))]
+    t0 = time.perf_counter()
+    oracle.fwd(t["q"], t["k"], t["v"], w.cu_q, w.cu_k, w.scale, w.causal, units=calib)
+    oracle.bwd(t["q"], t["k"], t["v"], t["dout"], w.cu_q, w.cu_k, w.scale, w.causal, units=calib)
+    dt = time.perf_counter() - t0
+    rate = 3.5 * fwd_flops(w.cu_q, w.cu_k, w.heads, w.head_dim, w.causal, calib) / max(dt, 1e-6)
+    pick, fl = [], 0.0
+    for u in units:
+        f = 3.5 * fwd_flops(w.cu_q, w.cu_k, w.heads, w.head_dim, w.causal, [u])
+        if pick and fl + f > rate * budget_s:
+            continue
+        pick.append(u)
+        fl += f
+        if fl >= rate * budget_s:
+            break
+    return pick, cores
+
+
+def time_oracle(w, units):
+    import oracle
+
+    t = w.tensors()
+    t0 = time.perf_counter()
+    oracle.fwd(t["q"], t["k"], t["v"], w.cu_q, w.cu_k, w.scale, w.causal, units=units)
+    oracle.bwd(t["q"], t["k"], t["v"], t["dout"], w.cu_q, w.cu_k, w.scale, w.causal, units=units)
+    dt = time.perf_counter() - t0
+    fl = 3.5 * fwd_flops(w.cu_q, w.cu_k, w.heads, w.head_dim, w.causal, units)
+    return fl / dt / 1e12, dt, fl
+
+
+def describe_sample(w, units):
+    seqs = sorted({b for b, _ in units})
+    return (f"{len(units)} (sequence, head) units of the workload (sequences {seqs[:8]}{'...' if len(seqs) > 8 else ''}, "
+            f"lengths {[int(np.diff(w.cu_q)[b]) for b in seqs[:8]]}), fp64 fwd+bwd, value scaled by the sample's "
+            f"3.5*F_fwd FLOPs")
+
+
+def cpu_baseline(w, budget_s=15.0):
+    units, cores = oracle_sample(w, budget_s)
+    tf, dt, _ = time_oracle(w, units)
+    return {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle", "seconds": dt,
+            "sample": describe_sample(w, units)}
+
+
+def run_reference(args):
+    """The oracle as it stands, on bounded samples of the same workload."""
+    w = synth.standard_workload(5)
+    per_step = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    units, cores = oracle_sample(w, per_step)
+    for _ in range(args.warmup):
+        time_oracle(w, units)
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        _, dt, fl = time_oracle(w, units)
+        times.append(dt)
+        flops = fl
+    ms = 1e3 * statistics.mean(times)
+    value = flops / (ms * 1e-3) / 1e12
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded bf16 N(0,1) inputs, widened exactly)",
+        "config": {"workload": WORKLOAD, "total_tokens": w.total_q, "heads": w.heads, "head_dim": w.head_dim,
+                   "causal": True},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": describe_sample(w, units)},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-aux", action="store_true", help="skip the forward-only workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            sys.exit("--gpus N > 1 must be launched with torchrun (one process per GPU)")
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    import torch
+
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        result, w = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                result["cpu_baseline"] = cpu_baseline(w)
+            print(json.dumps(result), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

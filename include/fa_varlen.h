@@ -116,6 +116,16 @@ fa_status_t fa_varlen_bwd(const void* dout, const void* q, const void* k, const 
  * FA_ERR_DEVICE_TIMEOUT), or FA_ERR_CUDA if the synchronisation failed. */
 fa_status_t fa_get_device_status(const void* workspace, fa_cuda_stream_t stream);
 
+/* Measurement hook for benchmarks; normal callers never need it. With
+ * `events` non-null, every later fa_varlen_fwd / fa_varlen_bwd call made from
+ * the calling host thread records, on its stream, events[2i] just before and
+ * events[2i+1] just after the i-th kernel it launches (i counts from 0 in each
+ * call; forward: 0 work-list preparation, 1 attention; backward: 0 work-list
+ * preparation, 1 preprocess, 2 attention gradients, 3 dQ conversion), for
+ * i < n_pairs. `events` holds cudaEvent_t handles created by the caller and
+ * must stay valid while the hook is on. Pass NULL to turn it off. */
+void fa_set_kernel_events(void* const* events, int n_pairs);
+
 /* Static, human-readable name of a status code. */
 const char* fa_status_string(fa_status_t status);
 

@@ -48,6 +48,29 @@ bool encode_map(CUtensorMap* map, const void* base, int rows, int cols, int box_
   return r == CUDA_SUCCESS;
 }
 
+// Measurement hook state (per host thread): events recorded around each
+// kernel launch of the next calls.
+struct KernelEvents {
+  void* const* events = nullptr;
+  int n_pairs = 0;
+  int next = 0;
+};
+thread_local KernelEvents t_events;
+
+// Runs one launch, bracketed by the caller's timing events when the hook is on.
+template <class F>
+cudaError_t timed_launch(cudaStream_t stream, F&& launch) {
+  KernelEvents& ev = t_events;
+  const int i = ev.next++;
+  const bool on = ev.events && i < ev.n_pairs;
+  if (on && cudaEventRecord(static_cast<cudaEvent_t>(ev.events[2 * i]), stream) != cudaSuccess) return cudaErrorUnknown;
+  cudaError_t e = launch();
+  if (e != cudaSuccess) return e;
+  if (on && cudaEventRecord(static_cast<cudaEvent_t>(ev.events[2 * i + 1]), stream) != cudaSuccess)
+    return cudaErrorUnknown;
+  return cudaSuccess;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int sm_count() {
@@ -117,9 +140,10 @@ fa_status_t fa_varlen_fwd(const void* q, const void* k, const void* v, const int
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < L.total)
     return FA_ERR_WORKSPACE;
 
+  t_events.next = 0;
   fa::SchedArgs sa{cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q, max_seqlen_k,
                    causal ? 1 : 0, 0, workspace, L.seq_off, L.pairs, L.max_pairs};
-  if (fa::launch_sched_prep(sa, stream) != cudaSuccess) return FA_ERR_CUDA;
+  if (timed_launch(stream, [&] { return fa::launch_sched_prep(sa, stream); }) != cudaSuccess) return FA_ERR_CUDA;
   if (total_q == 0) return FA_OK;
 
   const int HD = num_heads * head_dim;
@@ -149,7 +173,8 @@ fa_status_t fa_varlen_fwd(const void* q, const void* k, const void* v, const int
   fa_args.causal = causal ? 1 : 0;
   fa_args.scale_log2 = softmax_scale * 1.4426950408889634f;
   fa_args.grid = static_cast<int>(items < sms ? items : sms);
-  if (fa::launch_fwd(fa_args, tq, tk, tv, stream) != cudaSuccess) return FA_ERR_CUDA;
+  if (timed_launch(stream, [&] { return fa::launch_fwd(fa_args, tq, tk, tv, stream); }) != cudaSuccess)
+    return FA_ERR_CUDA;
   return FA_OK;
 }
 
@@ -172,9 +197,10 @@ fa_status_t fa_varlen_bwd(const void* dout, const void* q, const void* k, const 
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < L.total)
     return FA_ERR_WORKSPACE;
 
+  t_events.next = 0;
   fa::SchedArgs sa{cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q, max_seqlen_k,
                    causal ? 1 : 0, 1, workspace, L.seq_off, L.pairs, L.max_pairs};
-  if (fa::launch_sched_prep(sa, stream) != cudaSuccess) return FA_ERR_CUDA;
+  if (timed_launch(stream, [&] { return fa::launch_sched_prep(sa, stream); }) != cudaSuccess) return FA_ERR_CUDA;
   if (total_q == 0 && total_k == 0) return FA_OK;
 
   const int HD = num_heads * head_dim;
@@ -215,8 +241,17 @@ fa_status_t fa_varlen_bwd(const void* dout, const void* q, const void* k, const 
   b.scale = softmax_scale;
   b.scale_log2 = softmax_scale * 1.4426950408889634f;
   b.grid = static_cast<int>(items < sms ? items : sms);
-  if (fa::launch_bwd(b, tq, tk, tv, tdo, stream) != cudaSuccess) return FA_ERR_CUDA;
+  if (timed_launch(stream, [&] { return fa::launch_bwd_preprocess(b, stream); }) != cudaSuccess ||
+      timed_launch(stream, [&] { return fa::launch_bwd_main(b, tq, tk, tv, tdo, stream); }) != cudaSuccess ||
+      timed_launch(stream, [&] { return fa::launch_bwd_convert(b, stream); }) != cudaSuccess)
+    return FA_ERR_CUDA;
   return FA_OK;
+}
+
+void fa_set_kernel_events(void* const* events, int n_pairs) {
+  t_events.events = events;
+  t_events.n_pairs = events ? n_pairs : 0;
+  t_events.next = 0;
 }
 
 fa_status_t fa_get_device_status(const void* workspace, fa_cuda_stream_t stream_) {

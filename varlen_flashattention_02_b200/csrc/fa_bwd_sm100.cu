@@ -521,31 +521,37 @@ cudaError_t launch_main(const BwdArgs& a, const CUtensorMap& tq, const CUtensorM
   return cudaGetLastError();
 }
 
-template <int D>
-cudaError_t launch_all(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, cudaStream_t stream) {
-  const long long warps = static_cast<long long>(a.total_q) * a.H;
-  const unsigned blocks = static_cast<unsigned>((warps + 7) / 8);
-  if (blocks > 0) {
-    bwd_preprocess_kernel<D><<<blocks, 256, 0, stream>>>(a);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  cudaError_t e = a.causal ? launch_main<D, true>(a, tq, tk, tv, tdo, stream)
-                           : launch_main<D, false>(a, tq, tk, tv, tdo, stream);
-  if (e != cudaSuccess) return e;
-  if (blocks > 0) {
-    bwd_convert_kernel<D><<<blocks, 256, 0, stream>>>(a);
-    e = cudaGetLastError();
-  }
-  return e;
-}
-
 }  // namespace
 
-cudaError_t launch_bwd(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, cudaStream_t stream) {
-  return a.D == 64 ? launch_all<64>(a, tq, tk, tv, tdo, stream) : launch_all<128>(a, tq, tk, tv, tdo, stream);
+cudaError_t launch_bwd_preprocess(const BwdArgs& a, cudaStream_t stream) {
+  const long long warps = static_cast<long long>(a.total_q) * a.H;
+  const unsigned blocks = static_cast<unsigned>((warps + 7) / 8);
+  if (blocks == 0) return cudaSuccess;
+  if (a.D == 64)
+    bwd_preprocess_kernel<64><<<blocks, 256, 0, stream>>>(a);
+  else
+    bwd_preprocess_kernel<128><<<blocks, 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_main(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, cudaStream_t stream) {
+  if (a.D == 64)
+    return a.causal ? launch_main<64, true>(a, tq, tk, tv, tdo, stream)
+                    : launch_main<64, false>(a, tq, tk, tv, tdo, stream);
+  return a.causal ? launch_main<128, true>(a, tq, tk, tv, tdo, stream)
+                  : launch_main<128, false>(a, tq, tk, tv, tdo, stream);
+}
+
+cudaError_t launch_bwd_convert(const BwdArgs& a, cudaStream_t stream) {
+  const long long warps = static_cast<long long>(a.total_q) * a.H;
+  const unsigned blocks = static_cast<unsigned>((warps + 7) / 8);
+  if (blocks == 0) return cudaSuccess;
+  if (a.D == 64)
+    bwd_convert_kernel<64><<<blocks, 256, 0, stream>>>(a);
+  else
+    bwd_convert_kernel<128><<<blocks, 256, 0, stream>>>(a);
+  return cudaGetLastError();
 }
 
 }  // namespace fa

@@ -59,10 +59,12 @@ struct BwdArgs {
   float scale_log2;   // softmax_scale * log2(e)
   int grid;
 };
-// Preprocess (rowsum(dO*O), zero the dQ accumulator), main backward, dQ
-// conversion. tm_q / tm_do: box 64 rows x 64 columns; tm_k / tm_v: box 128
-// rows x 64 columns; all 128-byte swizzle.
-cudaError_t launch_bwd(const BwdArgs& a, const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                       const CUtensorMap& tm_do, cudaStream_t stream);
+// Backward in three launches: preprocess (rowsum(dO*O) and zero the dQ
+// accumulator), main, dQ conversion. tm_q / tm_do: box 64 rows x 64 columns;
+// tm_k / tm_v: box 128 rows x 64 columns; all 128-byte swizzle.
+cudaError_t launch_bwd_preprocess(const BwdArgs& a, cudaStream_t stream);
+cudaError_t launch_bwd_main(const BwdArgs& a, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                            const CUtensorMap& tm_v, const CUtensorMap& tm_do, cudaStream_t stream);
+cudaError_t launch_bwd_convert(const BwdArgs& a, cudaStream_t stream);
 
 }  // namespace fa

@@ -51,6 +51,8 @@ def _load():
     lib.fa_varlen_bwd.restype = I
     lib.fa_get_device_status.argtypes = [P, P]
     lib.fa_get_device_status.restype = I
+    lib.fa_set_kernel_events.argtypes = [P, I]
+    lib.fa_set_kernel_events.restype = None
     lib.fa_status_string.argtypes = [I]
     lib.fa_status_string.restype = ctypes.c_char_p
     return lib
@@ -59,7 +61,7 @@ def _load():
 lib = _load()
 
 EXPORTED = ("fa_varlen_fwd_workspace_size", "fa_varlen_bwd_workspace_size", "fa_varlen_fwd",
-            "fa_varlen_bwd", "fa_get_device_status", "fa_status_string")
+            "fa_varlen_bwd", "fa_get_device_status", "fa_set_kernel_events", "fa_status_string")
 
 
 def _p(t):
