@@ -178,8 +178,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++m;
       }
     producer_done:
-      if (m > 0) wait_bar(&bars.kv_full, (m - 1) & 1, ab);
-      for (uint32_t i = (p > 2 ? p - 2 : 0); i < p; ++i) wait_bar(&bars.qdo_full[i & 1], (i >> 1) & 1, ab);
+      if (m > 0) wait_bar_final(&bars.kv_full, (m - 1) & 1, ab);
+      for (uint32_t i = (p > 2 ? p - 2 : 0); i < p; ++i) wait_bar_final(&bars.qdo_full[i & 1], (i >> 1) & 1, ab);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     mma_done:
       mma_commit(&bars.drain);
-      wait_bar(&bars.drain, 0, ab);
+      wait_bar_final(&bars.drain, 0, ab);
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ lse / Dv rows
@@ -373,7 +373,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int s = 0; s < it.n; ++s, ++p) {
         const int pb = p & 1;
-        if (!wait_bar_warp(&bars.dq_full[pb], (p >> 1) & 1, ab)) goto drain_done;
+        // Group-wide decision: every warp of this group reaches the vote, so
+        // none is left waiting on the named barriers below.
+        if (!named_bar_and(1, 128, wait_bar(&bars.dq_full[pb], (p >> 1) & 1, ab))) goto drain_done;
         tc_fence_after();
         uint32_t v0[32], v1[32];
         tmem_ld32(tmem + lane_base + kColDP + pb * BM, v0);
@@ -400,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // dK, dV of this key tile.
-      if (!wait_bar_warp(&bars.dkv_full, m & 1, ab)) goto drain_done;
+      if (!named_bar_and(1, 128, wait_bar(&bars.dkv_full, m & 1, ab))) goto drain_done;
       tc_fence_after();
       {
         uint4* dk = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.dk) + krow * D);

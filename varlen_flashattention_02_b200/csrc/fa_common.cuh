@@ -154,6 +154,22 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const A
   return wait_slow(addr, parity, ab);
 }
 
+// Exit-path wait for work this thread itself put in flight (TMA loads,
+// MMAs): ignores the abort flag and gives up only after the time limit.
+__device__ __noinline__ static bool wait_bar_final(uint64_t* bar, uint32_t parity, const Abort& ab) {
+  const uint32_t addr = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(addr, parity)) return true;
+    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      raise_abort(ab);
+      return false;
+    }
+  }
+}
+
 // Warp-uniform form for roles whose next step is a .sync.aligned tcgen05
 // instruction: every lane returns the same answer.
 __device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, const Abort& ab) {

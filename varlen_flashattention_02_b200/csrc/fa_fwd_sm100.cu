@@ -170,10 +170,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   producer_done:
     // Never leave TMA writes in flight into shared memory we are about to
     // give up: wait (bounded) for the last loads issued.
-    if (nq > 0) wait_bar(&bars.q_full, (nq - 1) & 1, ab);
+    if (nq > 0) wait_bar_final(&bars.q_full, (nq - 1) & 1, ab);
     for (uint32_t i = (kv > NS ? kv - NS : 0); i < kv; ++i) {
-      wait_bar(&bars.k_full[i % NS], (i / NS) & 1, ab);
-      wait_bar(&bars.v_full[i % NS], (i / NS) & 1, ab);
+      wait_bar_final(&bars.k_full[i % NS], (i / NS) & 1, ab);
+      wait_bar_final(&bars.v_full[i % NS], (i / NS) & 1, ab);
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   mma_done:
     // Make sure every MMA this thread issued has finished before TMEM is freed.
     mma_commit(&bars.drain);
-    wait_bar(&bars.drain, 0, ab);
+    wait_bar_final(&bars.drain, 0, ab);
   } else if (warp >= kSoftmaxWarp0) {
     // ------------------------------------------------------------ softmax
     const int row = threadIdx.x - kSoftmaxWarp0 * 32;  // query row in tile == TMEM lane
