@@ -67,53 +67,64 @@ def load_peaks():
 
 # --------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples every 200 ms while the timed region runs."""
+    """Samples the SM clock and the clock-event reasons of one GPU through NVML
+    every 5 ms on a background thread while the timed region runs (read-only;
+    no setting of the GPU is touched)."""
 
-    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown", 0x8),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap", 0x4),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80))
 
     def __init__(self, uuid: str | None):
-        self.uuid = uuid
-        self.proc = None
-        self.path = None
+        self.samples = []
+        self.handle = None
+        self.thread = None
+        self.stop_flag = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(uuid) if uuid else pynvml.nvmlDeviceGetHandleByIndex(0)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.handle = None
+
+    def _run(self):
+        nv = self.nvml
+        while not self.stop_flag:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((sm, rs))
+            except Exception:
+                pass
+            time.sleep(0.005)
 
     def start(self):
-        try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "200", "-f", self.path],
-                                         stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+        if self.handle is None:
+            return
+        import threading
+
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if self.handle is None or self.thread is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = []
-        with open(self.path) as f:
-            for ln in f:
-                parts = [x.strip() for x in ln.split(",")]
-                if len(parts) < 9:
-                    continue
-                if self.uuid and parts[0] != self.uuid:
-                    continue
-                rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
+        self.stop_flag = True
+        self.thread.join()
+        if not self.samples:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "", 1).isdigit()]
-        smax = [float(r[2]) for r in rows if r[2].replace(".", "", 1).isdigit()]
-        reasons = sorted({name for r in rows for name, val in zip(self.REASONS, r[5:9]) if val == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(rows)}
+        reasons = set()
+        for _, rs in self.samples:
+            for name, attr, default in self.REASONS:
+                if rs & getattr(self.nvml, attr, default):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s for s, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.samples), "source": "NVML, 5 ms period"}
 
 
 # ----------------------------------------------------------------- our arm
@@ -133,6 +144,16 @@ def kernel_traffic(kernel_file: str):
     return ent.get("dram_bytes_per_launch")
 
 
+def bench_workload(tokens: int):
+    """The fwd+bwd workload; ``tokens`` < 16384 gives the same recipe on fewer
+    tokens (used only for small profiling captures)."""
+    if tokens == synth.TOTAL_TOKENS:
+        return synth.standard_workload(5)
+    lens = synth.lengths_uniform(5, tokens, 512, 8192)
+    return synth.make_workload(f"varlen-{tokens}-U512..8192-h16-d128-causal", lens, heads=16, head_dim=128,
+                               causal=True, seed=5, with_grad=True)
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -141,7 +162,7 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = synth.standard_workload(5)
+    w = bench_workload(args.tokens)
     w.seed = w.seed + 1000 * rank  # same shape, own data per rank
     t = w.tensors()
     H, D = w.heads, w.head_dim
@@ -249,7 +270,7 @@ def run_ours(args, rank, world, local_rank):
     host_out = [torch.empty(x.shape, dtype=torch.bfloat16).pin_memory() for x in (dq, dk, dv)]
     h2d = sum(x.numel() * x.element_size() for x in host_in.values()) + sum(x.numel() * 4 for x in host_cu)
     d2h = sum(x.numel() * x.element_size() for x in host_out)
-    e2e_steps = max(3, min(K, 10))
+    e2e_steps = 0 if args.no_e2e else max(3, min(K, 10))
     e2e_ev = [(mk(), mk()) for _ in range(e2e_steps)]
     torch.cuda.synchronize(dev)
     if world > 1:
@@ -270,14 +291,15 @@ def run_ours(args, rank, world, local_rank):
         host_out[2].copy_(dv, non_blocking=True)
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / e2e_steps
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / e2e_steps if e2e_steps else float("nan")
     if world > 1:
         tm = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(tm, op=dist.ReduceOp.MAX)
         e2e_ms = float(tm.item())
         dist.barrier()
-    e2e = {"value": world * 3.5 * F / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+    e2e = None if not e2e_steps else {
+        "value": world * 3.5 * F / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     peaks, peak_src = load_peaks()
     peak = float(peaks["bf16_tflops"])
@@ -364,14 +386,13 @@ def fwd_only_workloads(dev, stream, flush, peak, iters=10):
 # ------------------------------------------------------------- oracle (CPU)
 def oracle_sample(w, budget_s: float, seed: int = 0):
     """Pick (sequence, head) units of ``w`` whose oracle fwd+bwd takes about
-    ``budget_s`` on this host, calibrated on a first small batch."""
+    ``budget_s`` on this host. The oracle runs one unit per thread, so the
+    estimate is max(total work / cores, largest unit) at the single-thread
+    rate measured on a first batch of one unit per core."""
     import oracle
 
     t = w.tensors()
     cores = oracle.num_threads()
-    rng = random.Random(seed)
-    units = [(b, h) for b in range(w.batch) for h in range(w.heads)]
-    rng.shuffle(units)
     lens = np.diff(w.cu_q)
     shortest = int(np.argmin(lens))
     calib = [(shortest, h % w.heads) for h in range(max(cores, 1))]
@@ -379,16 +400,21 @@ def oracle_sample(w, budget_s: float, seed: int = 0):
     oracle.fwd(t["q"], t["k"], t["v"], w.cu_q, w.cu_k, w.scale, w.causal, units=calib)
     oracle.bwd(t["q"], t["k"], t["v"], t["dout"], w.cu_q, w.cu_k, w.scale, w.causal, units=calib)
     dt = time.perf_counter() - t0
-    rate = 3.5 * fwd_flops(w.cu_q, w.cu_k, w.heads, w.head_dim, w.causal, calib) / max(dt, 1e-6)
-    pick, fl = [], 0.0
+    unit_f = lambda u: 3.5 * fwd_flops(w.cu_q, w.cu_k, w.heads, w.head_dim, w.causal, [u])
+    r1 = unit_f(calib[0]) / max(dt, 1e-6)  # one thread's rate
+    units = [(b, h) for b in range(w.batch) for h in range(w.heads)]
+    random.Random(seed).shuffle(units)
+    pick, total, biggest = [], 0.0, 0.0
     for u in units:
-        f = 3.5 * fwd_flops(w.cu_q, w.cu_k, w.heads, w.head_dim, w.causal, [u])
-        if pick and fl + f > rate * budget_s:
+        f = unit_f(u)
+        est = max((total + f) / (cores * r1), max(biggest, f) / r1)
+        if est > budget_s:
             continue
         pick.append(u)
-        fl += f
-        if fl >= rate * budget_s:
-            break
+        total += f
+        biggest = max(biggest, f)
+    if not pick:
+        pick = calib
     return pick, cores
 
 
@@ -452,6 +478,9 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-aux", action="store_true", help="skip the forward-only workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--tokens", type=int, default=synth.TOTAL_TOKENS,
+                    help="total tokens of the workload (default 16384; smaller only for profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
