@@ -45,6 +45,25 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 FLUSH_BYTES = 256 << 20
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process
+    group). Works with NCCL (CUDA tensor) and gloo (CPU tensor)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(world: int, flops_per_rank: float, max_ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: every rank did ``flops_per_rank`` per step; the job's
+    step time is the slowest rank's."""
+    return world * flops_per_rank / (max_ms_per_step * 1e-3) / 1e12
+
+
 def fwd_flops(cu_q, cu_k, heads, head_dim, causal, units=None):
     lq = np.diff(np.asarray(cu_q, dtype=np.int64))
     lk = np.diff(np.asarray(cu_k, dtype=np.int64))
@@ -254,14 +273,10 @@ def run_ours(args, rank, world, local_rank):
         "bwd_attention": statistics.mean(bwd_main_ms),
         "bwd_dq_convert": statistics.mean(evs[6].elapsed_time(evs[7]) for evs in bwd_ev),
     }
-    tot_ms = sum(step_ms)
-    if world > 1:
-        tm = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-        tot_ms = float(tm.item())
+    tot_ms = max_over_ranks(sum(step_ms), dev)
     F = fwd_flops(w.cu_q, w.cu_k, H, D, w.causal)
     ms_step = tot_ms / K
-    value = world * 3.5 * F / (ms_step * 1e-3) / 1e12
+    value = weak_scaling_value(world, 3.5 * F, ms_step)
 
     # ---- end to end through the public API with host buffers (pinned)
     host_in = {n: torch.from_numpy(t[n].view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -292,13 +307,11 @@ def run_ours(args, rank, world, local_rank):
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / e2e_steps if e2e_steps else float("nan")
+    e2e_ms = max_over_ranks(e2e_ms, dev)
     if world > 1:
-        tm = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tm.item())
         dist.barrier()
     e2e = None if not e2e_steps else {
-        "value": world * 3.5 * F / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "value": weak_scaling_value(world, 3.5 * F, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
         "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     peaks, peak_src = load_peaks()
@@ -323,7 +336,7 @@ def run_ours(args, rank, world, local_rank):
                    "parallelism": f"weak: {world} independent replicas of the workload, no data-path collective"},
         "fwd_tflops": F / (statistics.mean(fwd_call_ms) * 1e-3) / 1e12,
         "bwd_tflops": 2.5 * F / (statistics.mean(bwd_call_ms) * 1e-3) / 1e12,
-        "fwd_bwd_tflops_literal_2p5": world * 2.5 * F / (ms_step * 1e-3) / 1e12,
+        "fwd_bwd_tflops_literal_2p5": weak_scaling_value(world, 2.5 * F, ms_step),
         "fwd_kernel_tflops": F / (fwd_k * 1e-3) / 1e12,
         "pct_of_peak": {"fwd_bwd": 100 * value / world / peak,
                         "fwd": 100 * F / (statistics.mean(fwd_call_ms) * 1e-3) / 1e12 / peak,

@@ -47,6 +47,7 @@ constexpr int kColDK = 0, kColDV = 128, kColS = 256, kColDP = 384;  // TMEM colu
 
 template <int D>
 struct BwdSmem {
+  static constexpr int kQStages = 3;  // Q/dO stages (and logsumexp/Dv slots) in flight
   static constexpr int kChunks = D / 64;
   static constexpr int kKChunk = BN * 128;  // [128 rows x 64 bf16] swizzled chunk
   static constexpr int kQChunk = BM * 128;  // [ 64 rows x 64 bf16]
@@ -56,22 +57,22 @@ struct BwdSmem {
   static constexpr int kK = 0;
   static constexpr int kV = kK + kKTile;
   static constexpr int kQdo = kV + kKTile;  // stage s: Q at kQdo + 2s*QTile, dO after it
-  static constexpr int kDs = kQdo + 4 * kQTile;
+  static constexpr int kDs = kQdo + 2 * kQStages * kQTile;
   static constexpr int kStage = kDs + 2 * kDsTile;   // fp32 dQ [64 x D]
-  static constexpr int kLd = kStage + BM * D * 4;    // 2 slots x (lse[64], dv[64]) fp32
-  static constexpr int kBar = kLd + 2 * 2 * BM * 4;
+  static constexpr int kLd = kStage + BM * D * 4;    // kQStages slots x (lse[64], dv[64]) fp32
+  static constexpr int kBar = kLd + kQStages * 2 * BM * 4;
   static constexpr int kBytes = kBar + 512;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
 struct Bars {
   uint64_t kv_full, kv_empty;
-  uint64_t qdo_full[2], qdo_empty[2];
+  uint64_t qdo_full[3], qdo_empty[3];
   uint64_t st_full[2];
   uint64_t ds_full[2], ds_empty[2];
   uint64_t dq_full[2], dq_empty[2];
   uint64_t dkv_full, dkv_empty;
-  uint64_t ld_full[2], ld_empty[2];
+  uint64_t ld_full[3], ld_empty[3];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -103,6 +104,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                const BwdArgs a) {
   using L = BwdSmem<D>;
+  constexpr int NQ = L::kQStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars& bars = *reinterpret_cast<Bars*>(smem + L::kBar);
@@ -115,16 +117,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(&bars.kv_full, 1);
     mbar_init(&bars.kv_empty, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < L::kQStages; ++i) {
       mbar_init(&bars.qdo_full[i], 1);
       mbar_init(&bars.qdo_empty[i], 1);
+      mbar_init(&bars.ld_full[i], 2);
+      mbar_init(&bars.ld_empty[i], 4);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.st_full[i], 1);
       mbar_init(&bars.ds_full[i], 4);
       mbar_init(&bars.ds_empty[i], 1);
       mbar_init(&bars.dq_full[i], 1);
       mbar_init(&bars.dq_empty[i], 4);
-      mbar_init(&bars.ld_full[i], 2);
-      mbar_init(&bars.ld_empty[i], 4);
     }
     mbar_init(&bars.dkv_full, 1);
     mbar_init(&bars.dkv_empty, 4);
@@ -164,8 +168,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(&tm_v, &bars.kv_full, smem + L::kV + c * L::kKChunk, it.h * D + c * 64, krow);
         }
         for (int s = 0; s < it.n; ++s, ++p) {
-          const int st = p & 1;
-          if (p >= 2 && !wait_bar(&bars.qdo_empty[st], ((p >> 1) - 1) & 1, ab)) goto producer_done;
+          const int st = p % NQ;
+          if (p >= NQ && !wait_bar(&bars.qdo_empty[st], ((p / NQ) - 1) & 1, ab)) goto producer_done;
           const int qrow = it.s.q0 + (it.i0 + s) * BM;
           uint8_t* sq = smem + L::kQdo + 2 * st * L::kQTile;
           uint8_t* sdo = sq + L::kQTile;
@@ -179,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     producer_done:
       if (m > 0) wait_bar_final(&bars.kv_full, (m - 1) & 1, ab);
-      for (uint32_t i = (p > 2 ? p - 2 : 0); i < p; ++i) wait_bar_final(&bars.qdo_full[i & 1], (i >> 1) & 1, ab);
+      for (uint32_t i = (p > NQ ? p - NQ : 0); i < p; ++i) wait_bar_final(&bars.qdo_full[i % NQ], (i / NQ) & 1, ab);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -197,11 +201,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s <= it.n; ++s) {
           if (s < it.n) {
             const uint32_t ps = p + s;
-            const int st = ps & 1;
-            if (!wait_bar(&bars.qdo_full[st], (ps >> 1) & 1, ab)) goto mma_done;
+            const int st = ps & 1;      // TMEM S^T / dP^T buffer
+            const int qs = ps % NQ;     // Q/dO stage
+            if (!wait_bar(&bars.qdo_full[qs], (ps / NQ) & 1, ab)) goto mma_done;
             if (ps >= 2 && !wait_bar(&bars.dq_empty[st], ((ps >> 1) - 1) & 1, ab)) goto mma_done;
             tc_fence_after();
-            const uint32_t sq = smem_u32(smem + L::kQdo + 2 * st * L::kQTile);
+            const uint32_t sq = smem_u32(smem + L::kQdo + 2 * qs * L::kQTile);
             const uint32_t sdo = sq + L::kQTile;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
@@ -222,10 +227,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (s > 0) {
             const uint32_t pp = p + s - 1;
             const int pb = pp & 1;
+            const int qs = pp % NQ;
             if (!wait_bar(&bars.ds_full[pb], (pp >> 1) & 1, ab)) goto mma_done;
             if (s == 1 && m > 0 && !wait_bar(&bars.dkv_empty, (m - 1) & 1, ab)) goto mma_done;
             tc_fence_after();
-            const uint32_t sq = smem_u32(smem + L::kQdo + 2 * pb * L::kQTile);
+            const uint32_t sq = smem_u32(smem + L::kQdo + 2 * qs * L::kQTile);
             const uint32_t sdo = sq + L::kQTile;
             const uint32_t sds = smem_u32(smem + L::kDs + pb * L::kDsTile);
             const uint32_t acc = (s > 1) ? 1u : 0u;
@@ -247,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      smem_desc_sw128(sds + kk * 2048, 0, 1024), kIdQ, kk > 0);
             }
             mma_commit(&bars.dq_full[pb]);
-            mma_commit(&bars.qdo_empty[pb]);
+            mma_commit(&bars.qdo_empty[qs]);
             mma_commit(&bars.ds_empty[pb]);
           }
         }
@@ -267,8 +273,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
       const Item it = get_item(a, pairs, idx);
       for (int s = 0; s < it.n; ++s, ++p) {
-        const int slot = p & 1;
-        if (p >= 2 && !wait_bar_warp(&bars.ld_empty[slot], ((p >> 1) - 1) & 1, ab)) goto loader_done;
+        const int slot = p % NQ;
+        if (p >= NQ && !wait_bar_warp(&bars.ld_empty[slot], ((p / NQ) - 1) & 1, ab)) goto loader_done;
         const int qi = (it.i0 + s) * BM + r;  // row within the sequence
         float lse2 = INFINITY, dv = 0.f;      // +inf logsumexp => P = 0 for rows outside the sequence
         if (qi < it.s.lq) {
@@ -300,10 +306,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < it.n; ++s, ++p) {
         const int pb = p & 1;
         if (!wait_bar_warp(&bars.st_full[pb], (p >> 1) & 1, ab)) goto compute_done;
-        if (!wait_bar_warp(&bars.ld_full[pb], (p >> 1) & 1, ab)) goto compute_done;
+        const int slot = p % NQ;
+        if (!wait_bar_warp(&bars.ld_full[slot], (p / NQ) & 1, ab)) goto compute_done;
         if (p >= 2 && !wait_bar_warp(&bars.ds_empty[pb], ((p >> 1) - 1) & 1, ab)) goto compute_done;
         tc_fence_after();
-        const float* ld = reinterpret_cast<const float*>(smem + L::kLd) + pb * 2 * BM;
+        const float* ld = reinterpret_cast<const float*>(smem + L::kLd) + slot * 2 * BM;
         const int row0 = (it.i0 + s) * BM;  // first query row of the step
         // Visible iff kg <= row + diag, i.e. e >= kg - diag - row0; keys past
         // the sequence see nothing.
@@ -345,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&bars.ds_full[pb]);
-          mbar_arrive(&bars.ld_empty[pb]);
+          mbar_arrive(&bars.ld_empty[slot]);
         }
       }
     }

@@ -25,8 +25,9 @@
 // B200 design, differing from the pages' A100 kernels:
 //  * persistent grid of one CTA per SM over a longest-first work list
 //    instead of one thread block per (batch, head[, q-block]);
-//  * warp specialisation instead of 4-8 symmetric warps: warp 0 issues TMA
-//    loads, one thread of warp 1 issues tcgen05 MMAs, warps 4-7 (128
+//  * warp specialisation instead of 4-8 symmetric warps: warp 0 issues the
+//    Q and K TMA loads, warp 2 the V loads (separate rings, so K can run
+//    ahead of V), one thread of warp 1 issues tcgen05 MMAs, warps 4-7 (128
 //    threads, one per query row and TMEM lane) do the softmax and epilogue;
 //  * accumulators live in tensor memory (S double-buffered so QK^T of tile
 //    j+1 overlaps the softmax of tile j; P overwrites its own S columns as
@@ -52,12 +53,16 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int D>
 struct FwdSmem {
-  static constexpr int kStages = (D == 64) ? 4 : 2;
+  // K and V have rings of their own: a K stage is released as soon as QK^T
+  // has read it, a V stage only after PV, so K runs further ahead.
+  static constexpr int kKStages = (D == 64) ? 4 : 3;
+  static constexpr int kVStages = (D == 64) ? 4 : 2;
   static constexpr int kChunks = D / 64;
   static constexpr int kTileBytes = kChunks * kChunkBytes;  // Q, K or V tile
   static constexpr int kQ = 0;
-  static constexpr int kKV = kQ + kTileBytes;                // stage s: K at kKV + 2s*tile, V after it
-  static constexpr int kBar = kKV + 2 * kStages * kTileBytes;
+  static constexpr int kK = kQ + kTileBytes;                 // K stage s at kK + s*tile
+  static constexpr int kV = kK + kKStages * kTileBytes;      // V stage s at kV + s*tile
+  static constexpr int kBar = kV + kVStages * kTileBytes;
   static constexpr int kBytes = kBar + 256;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
   static constexpr int kSCol = 0;               // S buffers at columns 0 and 128
@@ -69,7 +74,7 @@ struct Bars {
   uint64_t s_full[2], p_full[2];
   uint64_t o_full, o_empty;
   uint64_t drain;
-  uint64_t k_full[4], v_full[4], kv_empty[4];
+  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -97,7 +102,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
   using L = FwdSmem<D>;
-  constexpr int NS = L::kStages;
+  constexpr int NK = L::kKStages, NV = L::kVStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars& bars = *reinterpret_cast<Bars*>(smem + L::kBar);
@@ -116,10 +121,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars.o_full, 1);
     mbar_init(&bars.o_empty, 4);
     mbar_init(&bars.drain, 1);
-    for (int i = 0; i < NS; ++i) {
+    for (int i = 0; i < NK; ++i) {
       mbar_init(&bars.k_full[i], 1);
+      mbar_init(&bars.k_empty[i], 1);
+    }
+    for (int i = 0; i < NV; ++i) {
       mbar_init(&bars.v_full[i], 1);
-      mbar_init(&bars.kv_empty[i], 1);
+      mbar_init(&bars.v_empty[i], 1);
     }
     bars.abort_flag = 0;
     fence_mbar_init();
@@ -142,39 +150,48 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_items = (hdr->status == FA_OK) ? static_cast<int>(hdr->n_pairs) * a.H : 0;
 
   if (warp == 0 && lane == 0) {
-    // ------------------------------------------------------------ producer
-    uint32_t kv = 0, nq = 0;
+    // ------------------------------------------------------------ Q and K producer
+    uint32_t kc = 0, nq = 0;
     for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
       const Item it = get_item(a, pairs, idx);
       if (it.nk == 0) continue;
-      if (nq > 0 && !wait_bar(&bars.q_empty, (nq - 1) & 1, ab)) goto producer_done;
+      if (nq > 0 && !wait_bar(&bars.q_empty, (nq - 1) & 1, ab)) goto kproducer_done;
       mbar_arrive_expect_tx(&bars.q_full, L::kTileBytes);
       for (int c = 0; c < L::kChunks; ++c)
         tma_load_2d(&tm_q, &bars.q_full, smem + L::kQ + c * kChunkBytes, it.h * D + c * 64, it.s.q0 + it.t * BM);
       ++nq;
-      for (int j = 0; j < it.nk; ++j, ++kv) {
-        const int st = kv % NS;
-        const uint32_t use = kv / NS;
-        if (use > 0 && !wait_bar(&bars.kv_empty[st], (use - 1) & 1, ab)) goto producer_done;
-        uint8_t* sk = smem + L::kKV + 2 * st * L::kTileBytes;
-        uint8_t* sv = sk + L::kTileBytes;
-        const int row = it.s.k0 + j * BN;
+      for (int j = 0; j < it.nk; ++j, ++kc) {
+        const int st = kc % NK;
+        const uint32_t use = kc / NK;
+        if (use > 0 && !wait_bar(&bars.k_empty[st], (use - 1) & 1, ab)) goto kproducer_done;
         mbar_arrive_expect_tx(&bars.k_full[st], L::kTileBytes);
         for (int c = 0; c < L::kChunks; ++c)
-          tma_load_2d(&tm_k, &bars.k_full[st], sk + c * kChunkBytes, it.h * D + c * 64, row);
-        mbar_arrive_expect_tx(&bars.v_full[st], L::kTileBytes);
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_2d(&tm_v, &bars.v_full[st], sv + c * kChunkBytes, it.h * D + c * 64, row);
+          tma_load_2d(&tm_k, &bars.k_full[st], smem + L::kK + st * L::kTileBytes + c * kChunkBytes,
+                      it.h * D + c * 64, it.s.k0 + j * BN);
       }
     }
-  producer_done:
+  kproducer_done:
     // Never leave TMA writes in flight into shared memory we are about to
     // give up: wait (bounded) for the last loads issued.
     if (nq > 0) wait_bar_final(&bars.q_full, (nq - 1) & 1, ab);
-    for (uint32_t i = (kv > NS ? kv - NS : 0); i < kv; ++i) {
-      wait_bar_final(&bars.k_full[i % NS], (i / NS) & 1, ab);
-      wait_bar_final(&bars.v_full[i % NS], (i / NS) & 1, ab);
+    for (uint32_t i = (kc > NK ? kc - NK : 0); i < kc; ++i) wait_bar_final(&bars.k_full[i % NK], (i / NK) & 1, ab);
+  } else if (warp == 2 && lane == 0) {
+    // ------------------------------------------------------------ V producer
+    uint32_t vc = 0;
+    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+      const Item it = get_item(a, pairs, idx);
+      for (int j = 0; j < it.nk; ++j, ++vc) {
+        const int st = vc % NV;
+        const uint32_t use = vc / NV;
+        if (use > 0 && !wait_bar(&bars.v_empty[st], (use - 1) & 1, ab)) goto vproducer_done;
+        mbar_arrive_expect_tx(&bars.v_full[st], L::kTileBytes);
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_2d(&tm_v, &bars.v_full[st], smem + L::kV + st * L::kTileBytes + c * kChunkBytes,
+                      it.h * D + c * 64, it.s.k0 + j * BN);
+      }
     }
+  vproducer_done:
+    for (uint32_t i = (vc > NV ? vc - NV : 0); i < vc; ++i) wait_bar_final(&bars.v_full[i % NV], (i / NV) & 1, ab);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BN, false, false);
@@ -190,10 +207,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j < it.nk) {
           // S_j = Q K_j^T into S buffer (g + j) & 1.
           const uint32_t kvj = kv + j;
-          const int st = kvj % NS;
-          if (!wait_bar(&bars.k_full[st], (kvj / NS) & 1, ab)) goto mma_done;
+          const int st = kvj % NK;
+          if (!wait_bar(&bars.k_full[st], (kvj / NK) & 1, ab)) goto mma_done;
           tc_fence_after();
-          const uint32_t sk = smem_u32(smem + L::kKV + 2 * st * L::kTileBytes);
+          const uint32_t sk = smem_u32(smem + L::kK + st * L::kTileBytes);
           const uint32_t d_s = tmem + L::kSCol + ((g + j) & 1) * BN;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -202,25 +219,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                    kk > 0 ? 1u : 0u);
           }
           mma_commit(&bars.s_full[(g + j) & 1]);
+          mma_commit(&bars.k_empty[st]);
           if (j == it.nk - 1) mma_commit(&bars.q_empty);
         }
         if (j > 0) {
           // O (+)= P_{j-1} V_{j-1}, P read from TMEM.
           const int jj = j - 1;
           const uint32_t gj = g + jj, kvj = kv + jj;
-          const int st = kvj % NS;
+          const int st = kvj % NV;
           if (!wait_bar(&bars.p_full[gj & 1], (gj >> 1) & 1, ab)) goto mma_done;
           if (jj == 0 && nq > 0 && !wait_bar(&bars.o_empty, (nq - 1) & 1, ab)) goto mma_done;
-          if (!wait_bar(&bars.v_full[st], (kvj / NS) & 1, ab)) goto mma_done;
+          if (!wait_bar(&bars.v_full[st], (kvj / NV) & 1, ab)) goto mma_done;
           tc_fence_after();
-          const uint32_t sv = smem_u32(smem + L::kKV + (2 * st + 1) * L::kTileBytes);
+          const uint32_t sv = smem_u32(smem + L::kV + st * L::kTileBytes);
           const uint32_t a_p = tmem + L::kSCol + (gj & 1) * BN;
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
             mma_ts(tmem + L::kOCol, a_p + kk * 8, smem_desc_sw128(sv + kk * 2048, kChunkBytes, 1024), kIdescO,
                    (jj > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(&bars.kv_empty[st]);
+          mma_commit(&bars.v_empty[st]);
           mma_commit(&bars.o_full);
         }
       }
@@ -272,9 +290,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < BN; ++c)
             if (c >= lim) s[c] = -INFINITY;
         }
-        float mx = s[0];
+        // Row maximum with 8 independent partial maxima (short dependency chains).
+        float mx8[8];
 #pragma unroll
-        for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+        for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+#pragma unroll
+        for (int c = 8; c < BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mx8[i] = fmaxf(mx8[i], mx8[i + 4]);
+        const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3]));
         const float m_new = fmaxf(m_used, mx * a.scale_log2);
         // The previous PV must be complete before O may be rescaled (and so
         // that the o_full phase count stays in step).
@@ -302,16 +326,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_st();
         }
         const float m_ref = (m_used == -INFINITY) ? 0.f : m_used;
-        float lsum = 0.f;
+        float ls4[4] = {0.f, 0.f, 0.f, 0.f};  // partial row sums
         uint32_t pk[BN / 2];
 #pragma unroll
         for (int c = 0; c < BN; c += 2) {
           const float p0 = ex2_approx(fmaf(s[c], a.scale_log2, -m_ref));
           const float p1 = ex2_approx(fmaf(s[c + 1], a.scale_log2, -m_ref));
-          lsum += p0 + p1;
+          ls4[(c >> 1) & 3] += p0 + p1;
           pk[c / 2] = pack_bf16x2(p0, p1);
         }
-        l += lsum;
+        l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
         // P (bf16, two per column) overwrites the first BN/2 columns of S.
 #pragma unroll
         for (int c = 0; c < BN / 64; ++c) tmem_st32(t_s + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[c * 32]));
