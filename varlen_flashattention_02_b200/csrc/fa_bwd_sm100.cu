@@ -186,86 +186,96 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (uint32_t i = (p > NQ ? p - NQ : 0); i < p; ++i) wait_bar_final(&bars.qdo_full[i % NQ], (i / NQ) & 1, ab);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------------------------------------------------- MMA issuer
-      constexpr uint32_t kIdS = idesc_bf16_f32(BN, BM, false, false);   // S^T, dP^T: 128 x 64, K = D
-      constexpr uint32_t kIdKV = idesc_bf16_f32(BN, D, false, true);    // dV, dK: 128 x D, K = 64
-      constexpr uint32_t kIdQ = idesc_bf16_f32(128, BM, true, true);    // dQ^T: 128 (>= D) x 64, K = 128
-      const uint32_t sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
-      uint32_t m = 0, p = 0;
-      for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
-        const Item it = get_item(a, pairs, idx);
-        if (it.n == 0) continue;
-        if (!wait_bar(&bars.kv_full, m & 1, ab)) goto mma_done;
-        tc_fence_after();
-        for (int s = 0; s <= it.n; ++s) {
-          if (s < it.n) {
-            const uint32_t ps = p + s;
-            const int st = ps & 1;      // TMEM S^T / dP^T buffer
-            const int qs = ps % NQ;     // Q/dO stage
-            if (!wait_bar(&bars.qdo_full[qs], (ps / NQ) & 1, ab)) goto mma_done;
-            if (ps >= 2 && !wait_bar(&bars.dq_empty[st], ((ps >> 1) - 1) & 1, ab)) goto mma_done;
-            tc_fence_after();
-            const uint32_t sq = smem_u32(smem + L::kQdo + 2 * qs * L::kQTile);
-            const uint32_t sdo = sq + L::kQTile;
+    // ------------------------------------------------------------ MMA issuer
+    // The whole warp runs this loop converged; one elected lane issues each
+    // group of MMAs and the commits. Descriptors are built once and advanced
+    // by constant offsets.
+    constexpr uint32_t kIdS = idesc_bf16_f32(BN, BM, false, false);   // S^T, dP^T: 128 x 64, K = D
+    constexpr uint32_t kIdKV = idesc_bf16_f32(BN, D, false, true);    // dV, dK: 128 x D, K = 64
+    constexpr uint32_t kIdQ = idesc_bf16_f32(128, BM, true, true);    // dQ^T: 128 (>= D) x 64, K = 128
+    const uint64_t k_kmaj = smem_desc_sw128(smem_u32(smem + L::kK), 16, 1024);
+    const uint64_t v_kmaj = smem_desc_sw128(smem_u32(smem + L::kV), 16, 1024);
+    const uint64_t k_mn = smem_desc_sw128(smem_u32(smem + L::kK), D == 128 ? L::kKChunk : 0, 1024);
+    const uint64_t qdo_kmaj0 = smem_desc_sw128(smem_u32(smem + L::kQdo), 16, 1024);
+    const uint64_t qdo_mn0 = smem_desc_sw128(smem_u32(smem + L::kQdo), L::kQChunk, 1024);
+    const uint64_t ds_kmaj0 = smem_desc_sw128(smem_u32(smem + L::kDs), 16, 1024);
+    const uint64_t ds_mn0 = smem_desc_sw128(smem_u32(smem + L::kDs), 0, 1024);
+    constexpr uint64_t kQTileD = L::kQTile >> 4;    // descriptor step between Q and dO of a stage
+    uint32_t m = 0, p = 0;
+    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+      const Item it = get_item(a, pairs, idx);
+      if (it.n == 0) continue;
+      if (!wait_bar_warp(&bars.kv_full, m & 1, ab)) goto mma_done;
+      tc_fence_after();
+      for (int s = 0; s <= it.n; ++s) {
+        if (s < it.n) {
+          const uint32_t ps = p + s;
+          const int st = ps & 1;      // TMEM S^T / dP^T buffer
+          const int qs = ps % NQ;     // Q/dO stage
+          if (!wait_bar_warp(&bars.qdo_full[qs], (ps / NQ) & 1, ab)) goto mma_done;
+          if (ps >= 2 && !wait_bar_warp(&bars.dq_empty[st], ((ps >> 1) - 1) & 1, ab)) goto mma_done;
+          tc_fence_after();
+          const uint64_t q_desc = qdo_kmaj0 + static_cast<uint64_t>((2 * qs * L::kQTile) >> 4);
+          if (elect_one()) {
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t oa = (kk >> 2) * L::kKChunk + (kk & 3) * 32;
-              const uint32_t ob = (kk >> 2) * L::kQChunk + (kk & 3) * 32;
-              mma_ss(tmem + kColS + st * BM, smem_desc_sw128(sK + oa, 16, 1024), smem_desc_sw128(sq + ob, 16, 1024),
-                     kIdS, kk > 0);
+              const uint64_t oa = ((kk >> 2) * L::kKChunk + (kk & 3) * 32) >> 4;
+              const uint64_t ob = ((kk >> 2) * L::kQChunk + (kk & 3) * 32) >> 4;
+              mma_ss(tmem + kColS + st * BM, k_kmaj + oa, q_desc + ob, kIdS, kk > 0);
             }
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t oa = (kk >> 2) * L::kKChunk + (kk & 3) * 32;
-              const uint32_t ob = (kk >> 2) * L::kQChunk + (kk & 3) * 32;
-              mma_ss(tmem + kColDP + st * BM, smem_desc_sw128(sV + oa, 16, 1024),
-                     smem_desc_sw128(sdo + ob, 16, 1024), kIdS, kk > 0);
+              const uint64_t oa = ((kk >> 2) * L::kKChunk + (kk & 3) * 32) >> 4;
+              const uint64_t ob = ((kk >> 2) * L::kQChunk + (kk & 3) * 32) >> 4;
+              mma_ss(tmem + kColDP + st * BM, v_kmaj + oa, q_desc + kQTileD + ob, kIdS, kk > 0);
             }
             mma_commit(&bars.st_full[st]);
           }
-          if (s > 0) {
-            const uint32_t pp = p + s - 1;
-            const int pb = pp & 1;
-            const int qs = pp % NQ;
-            if (!wait_bar(&bars.ds_full[pb], (pp >> 1) & 1, ab)) goto mma_done;
-            if (s == 1 && m > 0 && !wait_bar(&bars.dkv_empty, (m - 1) & 1, ab)) goto mma_done;
-            tc_fence_after();
-            const uint32_t sq = smem_u32(smem + L::kQdo + 2 * qs * L::kQTile);
-            const uint32_t sdo = sq + L::kQTile;
-            const uint32_t sds = smem_u32(smem + L::kDs + pb * L::kDsTile);
-            const uint32_t acc = (s > 1) ? 1u : 0u;
+          __syncwarp();
+        }
+        if (s > 0) {
+          const uint32_t pp = p + s - 1;
+          const int pb = pp & 1;
+          const int qs = pp % NQ;
+          if (!wait_bar_warp(&bars.ds_full[pb], (pp >> 1) & 1, ab)) goto mma_done;
+          if (s == 1 && m > 0 && !wait_bar_warp(&bars.dkv_empty, (m - 1) & 1, ab)) goto mma_done;
+          tc_fence_after();
+          const uint64_t q_mn = qdo_mn0 + static_cast<uint64_t>((2 * qs * L::kQTile) >> 4);
+          const uint64_t ds_k = ds_kmaj0 + static_cast<uint64_t>((pb * L::kDsTile) >> 4);
+          const uint64_t ds_mn = ds_mn0 + static_cast<uint64_t>((pb * L::kDsTile) >> 4);
+          const uint32_t acc = (s > 1) ? 1u : 0u;
+          if (elect_one()) {
             // dV += P^T dO (P^T from TMEM, dO MN-major); dK += dS^T Q.
 #pragma unroll
-            for (int kk = 0; kk < BM / 16; ++kk) {
-              mma_ts(tmem + kColDV, tmem + kColS + pb * BM + kk * 8,
-                     smem_desc_sw128(sdo + kk * 2048, L::kQChunk, 1024), kIdKV, (acc | kk) ? 1u : 0u);
-            }
+            for (int kk = 0; kk < BM / 16; ++kk)
+              mma_ts(tmem + kColDV, tmem + kColS + pb * BM + kk * 8, q_mn + kQTileD + ((kk * 2048) >> 4), kIdKV,
+                     (acc | kk) ? 1u : 0u);
 #pragma unroll
-            for (int kk = 0; kk < BM / 16; ++kk) {
-              mma_ss(tmem + kColDK, smem_desc_sw128(sds + kk * 32, 16, 1024),
-                     smem_desc_sw128(sq + kk * 2048, L::kQChunk, 1024), kIdKV, (acc | kk) ? 1u : 0u);
-            }
+            for (int kk = 0; kk < BM / 16; ++kk)
+              mma_ss(tmem + kColDK, ds_k + ((kk * 32) >> 4), q_mn + ((kk * 2048) >> 4), kIdKV, (acc | kk) ? 1u : 0u);
             // dQ^T = K^T dS^T into the dP^T columns of this step.
 #pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk) {
-              mma_ss(tmem + kColDP + pb * BM, smem_desc_sw128(sK + kk * 2048, D == 128 ? L::kKChunk : 0, 1024),
-                     smem_desc_sw128(sds + kk * 2048, 0, 1024), kIdQ, kk > 0);
-            }
+            for (int kk = 0; kk < BN / 16; ++kk)
+              mma_ss(tmem + kColDP + pb * BM, k_mn + ((kk * 2048) >> 4), ds_mn + ((kk * 2048) >> 4), kIdQ, kk > 0);
             mma_commit(&bars.dq_full[pb]);
             mma_commit(&bars.qdo_empty[qs]);
             mma_commit(&bars.ds_empty[pb]);
           }
+          __syncwarp();
         }
+      }
+      if (elect_one()) {
         mma_commit(&bars.dkv_full);
         mma_commit(&bars.kv_empty);
-        p += it.n;
-        ++m;
       }
-    mma_done:
-      mma_commit(&bars.drain);
-      wait_bar_final(&bars.drain, 0, ab);
+      __syncwarp();
+      p += it.n;
+      ++m;
     }
+  mma_done:
+    if (elect_one()) mma_commit(&bars.drain);
+    __syncwarp();
+    wait_bar_final(&bars.drain, 0, ab);
   } else if (warp < 4) {
     // ------------------------------------------------------------ lse / Dv rows
     const int r = threadIdx.x - 64;  // query row within the tile, 0..63

@@ -72,7 +72,7 @@ struct FwdSmem {
 struct Bars {
   uint64_t q_full, q_empty;
   uint64_t s_full[2], p_full[2];
-  uint64_t o_full, o_empty;
+  uint64_t o_full[2], o_empty;
   uint64_t drain;
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
   uint32_t tmem_base;
@@ -118,7 +118,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.s_full[i], 1);
       mbar_init(&bars.p_full[i], 4);
     }
-    mbar_init(&bars.o_full, 1);
+    mbar_init(&bars.o_full[0], 1);
+    mbar_init(&bars.o_full[1], 1);
     mbar_init(&bars.o_empty, 4);
     mbar_init(&bars.drain, 1);
     for (int i = 0; i < NK; ++i) {
@@ -192,54 +193,63 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   vproducer_done:
     for (uint32_t i = (vc > NV ? vc - NV : 0); i < vc; ++i) wait_bar_final(&bars.v_full[i % NV], (i / NV) & 1, ab);
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // The whole warp runs this loop converged (all values warp-uniform);
+    // one elected lane issues each group of MMAs and the commits. Shared
+    // memory descriptors are built once and advanced by constant offsets.
     constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BN, false, false);
     constexpr uint32_t kIdescO = idesc_bf16_f32(BM, D, false, true);
-    const uint32_t sq = smem_u32(smem + L::kQ);
+    const uint64_t q_desc = smem_desc_sw128(smem_u32(smem + L::kQ), 16, 1024);
+    const uint64_t k_desc0 = smem_desc_sw128(smem_u32(smem + L::kK), 16, 1024);
+    const uint64_t v_desc0 = smem_desc_sw128(smem_u32(smem + L::kV), kChunkBytes, 1024);
     uint32_t kv = 0, g = 0, nq = 0;
     for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
       const Item it = get_item(a, pairs, idx);
       if (it.nk == 0) continue;
-      if (!wait_bar(&bars.q_full, nq & 1, ab)) goto mma_done;
+      if (!wait_bar_warp(&bars.q_full, nq & 1, ab)) goto mma_done;
       tc_fence_after();
       for (int j = 0; j <= it.nk; ++j) {
         if (j < it.nk) {
           // S_j = Q K_j^T into S buffer (g + j) & 1.
           const uint32_t kvj = kv + j;
           const int st = kvj % NK;
-          if (!wait_bar(&bars.k_full[st], (kvj / NK) & 1, ab)) goto mma_done;
+          if (!wait_bar_warp(&bars.k_full[st], (kvj / NK) & 1, ab)) goto mma_done;
           tc_fence_after();
-          const uint32_t sk = smem_u32(smem + L::kK + st * L::kTileBytes);
+          const uint64_t k_desc = k_desc0 + static_cast<uint64_t>((st * L::kTileBytes) >> 4);
           const uint32_t d_s = tmem + L::kSCol + ((g + j) & 1) * BN;
+          if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-            mma_ss(d_s, smem_desc_sw128(sq + off, 16, 1024), smem_desc_sw128(sk + off, 16, 1024), kIdescS,
-                   kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+              mma_ss(d_s, q_desc + off, k_desc + off, kIdescS, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&bars.s_full[(g + j) & 1]);
+            mma_commit(&bars.k_empty[st]);
+            if (j == it.nk - 1) mma_commit(&bars.q_empty);
           }
-          mma_commit(&bars.s_full[(g + j) & 1]);
-          mma_commit(&bars.k_empty[st]);
-          if (j == it.nk - 1) mma_commit(&bars.q_empty);
+          __syncwarp();
         }
         if (j > 0) {
           // O (+)= P_{j-1} V_{j-1}, P read from TMEM.
           const int jj = j - 1;
           const uint32_t gj = g + jj, kvj = kv + jj;
           const int st = kvj % NV;
-          if (!wait_bar(&bars.p_full[gj & 1], (gj >> 1) & 1, ab)) goto mma_done;
-          if (jj == 0 && nq > 0 && !wait_bar(&bars.o_empty, (nq - 1) & 1, ab)) goto mma_done;
-          if (!wait_bar(&bars.v_full[st], (kvj / NV) & 1, ab)) goto mma_done;
+          if (!wait_bar_warp(&bars.p_full[gj & 1], (gj >> 1) & 1, ab)) goto mma_done;
+          if (jj == 0 && nq > 0 && !wait_bar_warp(&bars.o_empty, (nq - 1) & 1, ab)) goto mma_done;
+          if (!wait_bar_warp(&bars.v_full[st], (kvj / NV) & 1, ab)) goto mma_done;
           tc_fence_after();
-          const uint32_t sv = smem_u32(smem + L::kV + st * L::kTileBytes);
+          const uint64_t v_desc = v_desc0 + static_cast<uint64_t>((st * L::kTileBytes) >> 4);
           const uint32_t a_p = tmem + L::kSCol + (gj & 1) * BN;
+          if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            mma_ts(tmem + L::kOCol, a_p + kk * 8, smem_desc_sw128(sv + kk * 2048, kChunkBytes, 1024), kIdescO,
-                   (jj > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BN / 16; ++kk)
+              mma_ts(tmem + L::kOCol, a_p + kk * 8, v_desc + static_cast<uint64_t>((kk * 2048) >> 4), kIdescO,
+                     (jj > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&bars.v_empty[st]);
+            mma_commit(&bars.o_full[gj & 1]);
           }
-          mma_commit(&bars.v_empty[st]);
-          mma_commit(&bars.o_full);
+          __syncwarp();
         }
       }
       kv += it.nk;
@@ -247,8 +257,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++nq;
     }
   mma_done:
-    // Make sure every MMA this thread issued has finished before TMEM is freed.
-    mma_commit(&bars.drain);
+    // Make sure every MMA this warp issued has finished before TMEM is freed.
+    if (elect_one()) mma_commit(&bars.drain);
+    __syncwarp();
     wait_bar_final(&bars.drain, 0, ab);
   } else if (warp >= kSoftmaxWarp0) {
     // ------------------------------------------------------------ softmax
@@ -300,12 +311,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 4; ++i) mx8[i] = fmaxf(mx8[i], mx8[i + 4]);
         const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3]));
         const float m_new = fmaxf(m_used, mx * a.scale_log2);
-        // The previous PV must be complete before O may be rescaled (and so
-        // that the o_full phase count stays in step).
-        if (j > 0) {
-          if (!wait_bar_warp(&bars.o_full, (g - 1) & 1, ab)) goto softmax_done;
-          tc_fence_after();
-        }
         float alpha = 1.f;
         if (m_new > m_used + kRescaleThreshold) {
           alpha = ex2_approx(m_used - m_new);  // 0 when m_used = -inf
@@ -313,6 +318,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_used = m_new;
         }
         if (__any_sync(0xffffffffu, j > 0 && alpha != 1.f)) {
+          // O may be rescaled only once the previous PV (global index g-1)
+          // has completed. PV completions alternate between two barriers, so
+          // the phase waited for is unambiguous: S_g done implies PV_{g-2}
+          // done, and PV_{g+1} cannot start before this tile's P exists.
+          if (!wait_bar_warp(&bars.o_full[(g - 1) & 1], ((g - 1) >> 1) & 1, ab)) goto softmax_done;
+          tc_fence_after();
           const uint32_t t_o = tmem + lane_base + L::kOCol;
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
@@ -344,8 +355,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.p_full[buf]);
       }
-      // Epilogue: wait for the last PV, normalise, store.
-      if (!wait_bar_warp(&bars.o_full, (g - 1) & 1, ab)) goto softmax_done;
+      // Epilogue: wait for the last PV (global index g-1), normalise, store.
+      if (!wait_bar_warp(&bars.o_full[(g - 1) & 1], ((g - 1) >> 1) & 1, ab)) goto softmax_done;
       tc_fence_after();
       {
         const float inv = (l > 0.f) ? 1.f / l : 0.f;
