@@ -3,8 +3,8 @@
 // Three kernels per call, after the work-list preparation (key-tile mode):
 //  1. preprocess: Dv_i = sum_c dO_ic * O_ic (fp32, [H, rows]) and zero the
 //     fp32 dQ accumulator;
-//  2. main: one persistent CTA per SM walks (sequence, head, key-tile)
-//     items, longest first. For 128 keys K_j, V_j of one head it loops over
+//  2. main: one persistent CTA per SM takes (sequence, head, key-tile)
+//     items, longest first, from a global counter. For 128 keys K_j, V_j of one head it loops over
 //     the 64-row query tiles that see them, recomputing the probabilities
 //     from the saved logsumexp instead of storing them:
 //        S^T  = K_j Q_i^T,  P^T = exp2(S^T*scale*log2e - lse_i*log2e)
@@ -74,6 +74,7 @@ struct Bars {
   uint64_t dkv_full, dkv_empty;
   uint64_t ld_full[3], ld_empty[3];
   uint64_t drain;
+  ItemRing items;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -133,6 +134,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars.dkv_full, 1);
     mbar_init(&bars.dkv_empty, 4);
     mbar_init(&bars.drain, 1);
+    // Item consumers: MMA warp (1), row loaders (2), P/dS warps (4), drain warps (4).
+    item_ring_init(bars.items, 11);
     bars.abort_flag = 0;
     fence_mbar_init();
   }
@@ -156,8 +159,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------------------------------------------------- producer
-      uint32_t m = 0, p = 0;
-      for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+      uint32_t m = 0, p = 0, ni = 0;
+      for (;;) {
+        int idx;
+        if (!publish_item(bars.items, ni, &hdr->work_counter, n_items, idx, ab)) goto producer_done;
+        if (idx < 0) break;
         const Item it = get_item(a, pairs, idx);
         if (it.n == 0) continue;
         if (m > 0 && !wait_bar(&bars.kv_empty, (m - 1) & 1, ab)) goto producer_done;
@@ -201,8 +207,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t ds_kmaj0 = smem_desc_sw128(smem_u32(smem + L::kDs), 16, 1024);
     const uint64_t ds_mn0 = smem_desc_sw128(smem_u32(smem + L::kDs), 0, 1024);
     constexpr uint64_t kQTileD = L::kQTile >> 4;    // descriptor step between Q and dO of a stage
-    uint32_t m = 0, p = 0;
-    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+    uint32_t m = 0, p = 0, ni = 0;
+    for (;;) {
+      int slot;
+      const int idx = consume_item<true>(bars.items, ni, slot, ab);
+      if (idx < 0) break;
+      if (elect_one()) mbar_arrive(&bars.items.empty[slot]);
+      __syncwarp();
       const Item it = get_item(a, pairs, idx);
       if (it.n == 0) continue;
       if (!wait_bar_warp(&bars.kv_full, m & 1, ab)) goto mma_done;
@@ -279,8 +290,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < 4) {
     // ------------------------------------------------------------ lse / Dv rows
     const int r = threadIdx.x - 64;  // query row within the tile, 0..63
-    uint32_t p = 0;
-    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+    uint32_t p = 0, ni = 0;
+    for (;;) {
+      int islot;
+      const int idx = consume_item<true>(bars.items, ni, islot, ab);
+      if (idx < 0) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.items.empty[islot]);
       const Item it = get_item(a, pairs, idx);
       for (int s = 0; s < it.n; ++s, ++p) {
         const int slot = p % NQ;
@@ -307,8 +323,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ P^T, dS^T
     const int kr = threadIdx.x - 128;  // key row in the tile == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    uint32_t p = 0;
-    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+    uint32_t p = 0, ni = 0;
+    for (;;) {
+      int islot;
+      const int idx = consume_item<true>(bars.items, ni, islot, ab);
+      if (idx < 0) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.items.empty[islot]);
       const Item it = get_item(a, pairs, idx);
       const int kg = it.j * BN + kr;  // key index within the sequence
       const bool key_ok = kg < it.s.lk;
@@ -373,8 +394,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q4 = warp & 3;
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     float* stage = reinterpret_cast<float*>(smem + L::kStage);
-    uint32_t p = 0, m = 0;
-    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+    uint32_t p = 0, m = 0, ni = 0;
+    for (;;) {
+      int islot;
+      const int idx = consume_item<true>(bars.items, ni, islot, ab);
+      // Group-uniform: this group uses named barriers, so all four warps
+      // must leave together (end of work, or an abort seen by any warp).
+      if (!named_bar_and(1, 128, idx >= 0)) break;
+      if (lane == 0) mbar_arrive(&bars.items.empty[islot]);
       const Item it = get_item(a, pairs, idx);
       const int kg = it.j * BN + t;
       const bool key_ok = kg < it.s.lk;

@@ -23,9 +23,10 @@ constexpr int kBwdBM = 64;
 
 // Per-call device state at the start of the workspace.
 struct WsHeader {
-  uint32_t status;   // fa_status_t of the device side of the call
-  uint32_t n_pairs;  // number of (sequence, tile) pairs in `pairs`
-  uint32_t reserved[62];
+  uint32_t status;        // fa_status_t of the device side of the call
+  uint32_t n_pairs;       // number of (sequence, tile) pairs in `pairs`
+  uint32_t work_counter;  // next work item to hand out (reset by the scheduler)
+  uint32_t reserved[61];
 };
 static_assert(sizeof(WsHeader) == 256, "header is one 256-byte block");
 
@@ -175,6 +176,52 @@ __device__ __noinline__ static bool wait_bar_final(uint64_t* bar, uint32_t parit
 __device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, const Abort& ab) {
   const bool ok = wait_bar(bar, parity, ab);
   return __all_sync(0xffffffffu, ok);
+}
+
+// ------------------------------------------------------- dynamic work items
+// Persistent CTAs take work items (in the scheduler's longest-first order)
+// from a global counter. One thread per CTA claims each item and publishes
+// its index to the CTA's other roles through this ring; -1 means "no more".
+constexpr int kItemSlots = 4;
+struct ItemRing {
+  uint64_t full[kItemSlots];   // count 1: the publishing thread
+  uint64_t empty[kItemSlots];  // count = number of consuming arrivals per item
+  int idx[kItemSlots];
+};
+
+__device__ __forceinline__ void item_ring_init(ItemRing& r, uint32_t consumers) {
+  for (int i = 0; i < kItemSlots; ++i) {
+    mbar_init(&r.full[i], 1);
+    mbar_init(&r.empty[i], consumers);
+  }
+}
+
+// Publisher (one thread): claim the next item and publish it. Returns false
+// if the CTA is aborting.
+__device__ __forceinline__ bool publish_item(ItemRing& r, uint32_t& n, uint32_t* counter, int n_items, int& idx,
+                                             const Abort& ab) {
+  const int slot = n % kItemSlots;
+  if (n >= kItemSlots && !wait_bar(&r.empty[slot], ((n / kItemSlots) - 1) & 1, ab)) return false;
+  int v = static_cast<int>(atomicAdd(counter, 1u));
+  if (v >= n_items) v = -1;
+  *reinterpret_cast<volatile int*>(&r.idx[slot]) = v;
+  mbar_arrive(&r.full[slot]);
+  ++n;
+  idx = v;
+  return true;
+}
+
+// Consumer: wait for the n-th published item; returns its index, or -1 when
+// there is no more work (or the CTA is aborting). `slot` receives the ring
+// slot, on whose `empty` barrier the caller arrives once it has the index.
+template <bool WARP>
+__device__ __forceinline__ int consume_item(ItemRing& r, uint32_t& n, int& slot, const Abort& ab) {
+  slot = n % kItemSlots;
+  const uint32_t par = (n / kItemSlots) & 1;
+  const bool ok = WARP ? wait_bar_warp(&r.full[slot], par, ab) : wait_bar(&r.full[slot], par, ab);
+  ++n;
+  if (!ok) return -2;
+  return *reinterpret_cast<volatile int*>(&r.idx[slot]);
 }
 
 }  // namespace fa

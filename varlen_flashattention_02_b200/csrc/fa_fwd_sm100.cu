@@ -1,7 +1,7 @@
 // fa_fwd_sm100.cu -- forward varlen attention for sm_100a.
 //
-// One persistent CTA per SM walks the (sequence, head, query-tile) work list
-// built by the scheduler (longest first). For each item it computes, for
+// One persistent CTA per SM takes (sequence, head, query-tile) items from the
+// scheduler's longest-first list through a global counter. For each item it computes, for
 // 128 query rows of one head of one sequence, exact attention over the
 // sequence's keys with an online softmax:
 //
@@ -63,7 +63,7 @@ struct FwdSmem {
   static constexpr int kK = kQ + kTileBytes;                 // K stage s at kK + s*tile
   static constexpr int kV = kK + kKStages * kTileBytes;      // V stage s at kV + s*tile
   static constexpr int kBar = kV + kVStages * kTileBytes;
-  static constexpr int kBytes = kBar + 256;
+  static constexpr int kBytes = kBar + 512;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
   static constexpr int kSCol = 0;               // S buffers at columns 0 and 128
   static constexpr int kOCol = 256;             // O accumulator
@@ -75,10 +75,11 @@ struct Bars {
   uint64_t o_full[2], o_empty;
   uint64_t drain;
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
+  ItemRing items;
   uint32_t tmem_base;
   int abort_flag;
 };
-static_assert(sizeof(Bars) <= 256, "barrier block fits its reserved space");
+static_assert(sizeof(Bars) <= 512, "barrier block fits its reserved space");
 
 struct Item {
   int b, h, t;
@@ -130,6 +131,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.v_full[i], 1);
       mbar_init(&bars.v_empty[i], 1);
     }
+    // Item consumers: V producer (1), MMA warp (1), softmax warps (4).
+    item_ring_init(bars.items, 6);
     bars.abort_flag = 0;
     fence_mbar_init();
   }
@@ -152,8 +155,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ Q and K producer
-    uint32_t kc = 0, nq = 0;
-    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+    uint32_t kc = 0, nq = 0, ni = 0;
+    for (;;) {
+      int idx;
+      if (!publish_item(bars.items, ni, &hdr->work_counter, n_items, idx, ab)) goto kproducer_done;
+      if (idx < 0) break;
       const Item it = get_item(a, pairs, idx);
       if (it.nk == 0) continue;
       if (nq > 0 && !wait_bar(&bars.q_empty, (nq - 1) & 1, ab)) goto kproducer_done;
@@ -178,8 +184,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (uint32_t i = (kc > NK ? kc - NK : 0); i < kc; ++i) wait_bar_final(&bars.k_full[i % NK], (i / NK) & 1, ab);
   } else if (warp == 2 && lane == 0) {
     // ------------------------------------------------------------ V producer
-    uint32_t vc = 0;
-    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+    uint32_t vc = 0, ni = 0;
+    for (;;) {
+      int slot;
+      const int idx = consume_item<false>(bars.items, ni, slot, ab);
+      if (idx < 0) break;
+      mbar_arrive(&bars.items.empty[slot]);
       const Item it = get_item(a, pairs, idx);
       for (int j = 0; j < it.nk; ++j, ++vc) {
         const int st = vc % NV;
@@ -203,8 +213,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t q_desc = smem_desc_sw128(smem_u32(smem + L::kQ), 16, 1024);
     const uint64_t k_desc0 = smem_desc_sw128(smem_u32(smem + L::kK), 16, 1024);
     const uint64_t v_desc0 = smem_desc_sw128(smem_u32(smem + L::kV), kChunkBytes, 1024);
-    uint32_t kv = 0, g = 0, nq = 0;
-    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+    uint32_t kv = 0, g = 0, nq = 0, ni = 0;
+    for (;;) {
+      int slot;
+      const int idx = consume_item<true>(bars.items, ni, slot, ab);
+      if (idx < 0) break;
+      if (elect_one()) mbar_arrive(&bars.items.empty[slot]);
+      __syncwarp();
       const Item it = get_item(a, pairs, idx);
       if (it.nk == 0) continue;
       if (!wait_bar_warp(&bars.q_full, nq & 1, ab)) goto mma_done;
@@ -265,8 +280,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ softmax
     const int row = threadIdx.x - kSoftmaxWarp0 * 32;  // query row in tile == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    uint32_t g = 0, nq = 0;
-    for (int idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
+    uint32_t g = 0, nq = 0, ni = 0;
+    for (;;) {
+      int slot;
+      const int idx = consume_item<true>(bars.items, ni, slot, ab);
+      if (idx < 0) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.items.empty[slot]);
       const Item it = get_item(a, pairs, idx);
       const int r = it.t * BM + row;  // row within the sequence
       const bool row_ok = r < it.s.lq;
@@ -339,12 +359,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m_ref = (m_used == -INFINITY) ? 0.f : m_used;
         float ls4[4] = {0.f, 0.f, 0.f, 0.f};  // partial row sums
         uint32_t pk[BN / 2];
+        if (need_mask) {
+          // Masked entries are -inf and must give exactly 0: MUFU only.
 #pragma unroll
-        for (int c = 0; c < BN; c += 2) {
-          const float p0 = ex2_approx(fmaf(s[c], a.scale_log2, -m_ref));
-          const float p1 = ex2_approx(fmaf(s[c + 1], a.scale_log2, -m_ref));
-          ls4[(c >> 1) & 3] += p0 + p1;
-          pk[c / 2] = pack_bf16x2(p0, p1);
+          for (int c = 0; c < BN; c += 2) {
+            const float p0 = ex2_approx(fmaf(s[c], a.scale_log2, -m_ref));
+            const float p1 = ex2_approx(fmaf(s[c + 1], a.scale_log2, -m_ref));
+            ls4[(c >> 1) & 3] += p0 + p1;
+            pk[c / 2] = pack_bf16x2(p0, p1);
+          }
+        } else {
+          // Every fourth pair of columns on the FMA pipe, the rest on MUFU.
+#pragma unroll
+          for (int c = 0; c < BN; c += 2) {
+            const float x0 = fmaf(s[c], a.scale_log2, -m_ref);
+            const float x1 = fmaf(s[c + 1], a.scale_log2, -m_ref);
+            const bool poly = ((c >> 1) & 3) == 3;
+            const float p0 = poly ? exp2_poly3(x0) : ex2_approx(x0);
+            const float p1 = poly ? exp2_poly3(x1) : ex2_approx(x1);
+            ls4[(c >> 1) & 3] += p0 + p1;
+            pk[c / 2] = pack_bf16x2(p0, p1);
+          }
         }
         l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
         // P (bf16, two per column) overwrites the first BN/2 columns of S.

@@ -82,6 +82,7 @@ __global__ void __launch_bounds__(kThreads) sched_prep_kernel(SchedArgs a) {
   if (tid == 0) {
     s_err = 0;
     s_total = 0;
+    hdr->work_counter = 0;
     if (a.cu_q[0] != 0 || a.cu_k[0] != 0 || a.cu_q[a.batch] != a.total_q || a.cu_k[a.batch] != a.total_k)
       s_err = 1;
   }
