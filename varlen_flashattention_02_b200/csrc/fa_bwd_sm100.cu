@@ -302,17 +302,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int slot = p % NQ;
         if (p >= NQ && !wait_bar_warp(&bars.ld_empty[slot], ((p / NQ) - 1) & 1, ab)) goto loader_done;
         const int qi = (it.i0 + s) * BM + r;  // row within the sequence
-        float lse2 = INFINITY, dv = 0.f;      // +inf logsumexp => P = 0 for rows outside the sequence
+        // Stored negated and in base 2: -lse*log2(e); -inf for rows outside
+        // the sequence or without a visible key, which makes their P exactly 0.
+        float nlse2 = -INFINITY, dv = 0.f;
         if (qi < it.s.lq) {
           const size_t gq = static_cast<size_t>(it.s.q0) + qi;
           const float l = __ldg(a.lse + static_cast<size_t>(it.h) * a.total_q + gq);
           if (l != -INFINITY) {
-            lse2 = l * 1.4426950408889634f;
+            nlse2 = -l * 1.4426950408889634f;
             dv = __ldg(dvec + static_cast<size_t>(it.h) * a.tq_pad + gq);
           }
         }
         float* ld = reinterpret_cast<float*>(smem + L::kLd) + slot * 2 * BM;
-        ld[r] = lse2;
+        ld[r] = nlse2;
         ld[BM + r] = dv;
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.ld_full[slot]);
@@ -348,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int e_min = CAUSAL ? kg - diag - row0 : 0;
         if (!key_ok) e_min = BM;
         uint8_t* ds_row = smem + L::kDs + pb * L::kDsTile + kr * 128;
+        const uint64_t sc2 = f2_make(a.scale_log2, a.scale_log2);
 #pragma unroll
         for (int c = 0; c < BM / 32; ++c) {
           uint32_t sv[32], dpv[32];
@@ -358,12 +361,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const int q = c * 32 + e;
-            float p0 = ex2_approx(fmaf(__uint_as_float(sv[e]), a.scale_log2, -ld[q]));
-            float p1 = ex2_approx(fmaf(__uint_as_float(sv[e + 1]), a.scale_log2, -ld[q + 1]));
+            // Pairs of query columns share packed f32x2 arithmetic.
+            const uint64_t nl2 = *reinterpret_cast<const uint64_t*>(ld + q);
+            const uint64_t dv2 = *reinterpret_cast<const uint64_t*>(ld + BM + q);
+            float x0, x1;
+            f2_split(f2_fma(f2_make(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sc2, nl2), x0, x1);
+            float p0 = ex2_approx(x0);
+            float p1 = ex2_approx(x1);
             if (q < e_min) p0 = 0.f;
             if (q + 1 < e_min) p1 = 0.f;
-            const float d0 = p0 * (__uint_as_float(dpv[e]) - ld[BM + q]);
-            const float d1 = p1 * (__uint_as_float(dpv[e + 1]) - ld[BM + q + 1]);
+            const uint64_t p2 = f2_make(p0, p1);
+            float d0, d1;
+            f2_split(f2_mul(p2, f2_sub(f2_make(__uint_as_float(dpv[e]), __uint_as_float(dpv[e + 1])), dv2)), d0, d1);
             pk[e / 2] = pack_bf16x2(p0, p1);
             dsk[e / 2] = pack_bf16x2(d0, d1);
           }

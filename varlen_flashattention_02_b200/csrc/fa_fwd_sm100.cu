@@ -321,15 +321,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < BN; ++c)
             if (c >= lim) s[c] = -INFINITY;
         }
-        // Row maximum with 8 independent partial maxima (short dependency chains).
-        float mx8[8];
+        // Row maximum: four independent chains of three-input maxima.
+        float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx8[i] = s[i];
-#pragma unroll
-        for (int c = 8; c < BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) mx8[i] = fmaxf(mx8[i], mx8[i + 4]);
-        const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3]));
+        for (int c = 4; c + 8 <= BN; c += 8) {
+          m0 = fmax3(m0, s[c], s[c + 1]);
+          m1 = fmax3(m1, s[c + 2], s[c + 3]);
+          m2 = fmax3(m2, s[c + 4], s[c + 5]);
+          m3 = fmax3(m3, s[c + 6], s[c + 7]);
+        }
+        m0 = fmax3(m0, s[BN - 4], s[BN - 3]);
+        m1 = fmax3(m1, s[BN - 2], s[BN - 1]);
+        const float mx = fmax3(m0, m1, fmaxf(m2, m3));
         const float m_new = fmaxf(m_used, mx * a.scale_log2);
         float alpha = 1.f;
         if (m_new > m_used + kRescaleThreshold) {
@@ -357,29 +360,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_st();
         }
         const float m_ref = (m_used == -INFINITY) ? 0.f : m_used;
-        float ls4[4] = {0.f, 0.f, 0.f, 0.f};  // partial row sums
+        // p = exp2(s * scale * log2e - m): pairs of columns share one packed
+        // FMA and one packed add into the partial row sums.
+        const uint64_t sc2 = f2_make(a.scale_log2, a.scale_log2);
+        const uint64_t nm2 = f2_make(-m_ref, -m_ref);
+        uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
         uint32_t pk[BN / 2];
-        if (need_mask) {
-          // Masked entries are -inf and must give exactly 0: MUFU only.
 #pragma unroll
-          for (int c = 0; c < BN; c += 2) {
-            const float p0 = ex2_approx(fmaf(s[c], a.scale_log2, -m_ref));
-            const float p1 = ex2_approx(fmaf(s[c + 1], a.scale_log2, -m_ref));
-            ls4[(c >> 1) & 3] += p0 + p1;
-            pk[c / 2] = pack_bf16x2(p0, p1);
-          }
-        } else {
-          // Every fourth pair of columns on the FMA pipe, the rest on MUFU.
-#pragma unroll
-          for (int c = 0; c < BN; c += 2) {
-            const float x0 = fmaf(s[c], a.scale_log2, -m_ref);
-            const float x1 = fmaf(s[c + 1], a.scale_log2, -m_ref);
-            const bool poly = ((c >> 1) & 3) == 3;
-            const float p0 = poly ? exp2_poly3(x0) : ex2_approx(x0);
-            const float p1 = poly ? exp2_poly3(x1) : ex2_approx(x1);
-            ls4[(c >> 1) & 3] += p0 + p1;
-            pk[c / 2] = pack_bf16x2(p0, p1);
-          }
+        for (int c = 0; c < BN; c += 2) {
+          float x0, x1;
+          f2_split(f2_fma(f2_make(s[c], s[c + 1]), sc2, nm2), x0, x1);
+          const float p0 = ex2_approx(x0);
+          const float p1 = ex2_approx(x1);
+          ls2[(c >> 1) & 3] = f2_add(ls2[(c >> 1) & 3], f2_make(p0, p1));
+          pk[c / 2] = pack_bf16x2(p0, p1);
+        }
+        float ls4[4];
+        {
+          float a0, a1, b0, b1;
+          f2_split(f2_add(ls2[0], ls2[1]), a0, a1);
+          f2_split(f2_add(ls2[2], ls2[3]), b0, b1);
+          ls4[0] = a0;
+          ls4[1] = a1;
+          ls4[2] = b0;
+          ls4[3] = b1;
         }
         l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
         // P (bf16, two per column) overwrites the first BN/2 columns of S.
