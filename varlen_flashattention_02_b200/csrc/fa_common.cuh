@@ -133,7 +133,7 @@ __device__ __forceinline__ void raise_abort(const Abort& ab) {
   atomicCAS(ab.status, 0u, static_cast<uint32_t>(FA_ERR_DEVICE_TIMEOUT));
 }
 
-static __device__ __noinline__ bool wait_slow(uint32_t addr, uint32_t parity, const Abort& ab) {
+static __device__ __forceinline__ bool wait_slow(uint32_t addr, uint32_t parity, const Abort& ab) {
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
 #pragma unroll 1
@@ -157,7 +157,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const A
 
 // Exit-path wait for work this thread itself put in flight (TMA loads,
 // MMAs): ignores the abort flag and gives up only after the time limit.
-__device__ __noinline__ static bool wait_bar_final(uint64_t* bar, uint32_t parity, const Abort& ab) {
+__device__ __forceinline__ static bool wait_bar_final(uint64_t* bar, uint32_t parity, const Abort& ab) {
   const uint32_t addr = smem_u32(bar);
   const uint64_t t0 = globaltimer_ns();
   for (;;) {

@@ -230,22 +230,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-// 2^x on the FMA pipe, for x in [-126, 64], to offload the MUFU unit.
-// Range reduction: adding 1.5 * 2^23 rounds x to the nearest integer n in the
-// low mantissa bits of t; f = x - n lies in [-0.5, 0.5]. 2^f is a degree-3
-// polynomial fitted for this library by the Remez exchange algorithm
-// (minimax in relative error, max 7.5e-5 in fp32 Horner form); the result is
-// scaled by 2^n by adding n to the exponent field. Inputs below -126 are
-// clamped (the result is then ~1.2e-38 instead of smaller).
-__device__ __forceinline__ float exp2_poly3(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  const float p = fmaf(fmaf(fmaf(0.0551716685295105f, f, 0.2426111251115799f), f, 0.6932609677314758f), f,
-                       0.9999280571937561f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 // Packed pairs of fp32 (sm_100 f32x2 arithmetic: one instruction, two lanes
 // of work).
 __device__ __forceinline__ uint64_t f2_make(float lo, float hi) {
