@@ -111,6 +111,37 @@ fa_status_t fa_varlen_bwd(const void* dout, const void* q, const void* k, const 
                           int head_dim, float softmax_scale, int causal, void* dq, void* dk, void* dv,
                           void* workspace, size_t workspace_bytes, fa_cuda_stream_t stream);
 
+/* Forward for callers that cannot allocate device memory. The pages have no
+ * counterpart of this entry point; it exists for the library's users.
+ *
+ * Same arguments and results as fa_varlen_fwd, without the workspace. Some
+ * callers cannot call cudaMalloc: code running inside another framework's
+ * plugin or operator interface that receives only input and output pointers
+ * (allocating outside that framework's pool breaks its accounting), or
+ * latency-critical paths where a device allocation, which may synchronise
+ * the device, is not allowed. This entry point allocates nothing: its scratch
+ * is a library-owned device buffer of FA_NOALLOC_SCRATCH_BYTES (256 KiB) that
+ * every GPU loading the library holds until the process exits.
+ *
+ * - Returns FA_ERR_WORKSPACE, before any CUDA call, when the sizes need more
+ *   scratch than that (fa_varlen_fwd_workspace_size(batch, total_q,
+ *   num_heads, head_dim) > FA_NOALLOC_SCRATCH_BYTES; roughly
+ *   total_q / 128 + batch must stay below about 32000).
+ * - The first call on each device looks up the buffer's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ * - All calls on a device share the one buffer, which keeps the last call's
+ *   contents: calls that can overlap on the GPU (different streams, or
+ *   different host threads) race and must be serialised by the caller.
+ * - Errors found on the device (malformed cu_seqlens) cannot be read back:
+ *   the outputs are then undefined. */
+#define FA_NOALLOC_SCRATCH_BYTES (256u * 1024u)
+fa_status_t fa_varlen_fwd_noalloc(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                                  const int32_t* cu_seqlens_k, int batch, int total_q, int total_k,
+                                  int max_seqlen_q, int max_seqlen_k, int num_heads, int head_dim,
+                                  float softmax_scale, int causal, void* out, float* softmax_lse,
+                                  fa_cuda_stream_t stream);
+
 /* Synchronises `stream`, then returns the device-side status of the last
  * call that used `workspace` (FA_OK, FA_ERR_BAD_SEQLENS or
  * FA_ERR_DEVICE_TIMEOUT), or FA_ERR_CUDA if the synchronisation failed. */

@@ -51,6 +51,8 @@ def _load():
     lib.fa_varlen_bwd.restype = I
     lib.fa_get_device_status.argtypes = [P, P]
     lib.fa_get_device_status.restype = I
+    lib.fa_varlen_fwd_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, ctypes.c_float, I, P, P, P]
+    lib.fa_varlen_fwd_noalloc.restype = I
     lib.fa_set_kernel_events.argtypes = [P, I]
     lib.fa_set_kernel_events.restype = None
     lib.fa_status_string.argtypes = [I]
@@ -61,7 +63,8 @@ def _load():
 lib = _load()
 
 EXPORTED = ("fa_varlen_fwd_workspace_size", "fa_varlen_bwd_workspace_size", "fa_varlen_fwd",
-            "fa_varlen_bwd", "fa_get_device_status", "fa_set_kernel_events", "fa_status_string")
+            "fa_varlen_bwd", "fa_varlen_fwd_noalloc", "fa_get_device_status", "fa_set_kernel_events",
+            "fa_status_string")
 
 
 def _p(t):
@@ -149,6 +152,31 @@ def fa_varlen_bwd(dout, q, k, v, out, softmax_lse, cu_seqlens_q, cu_seqlens_k, m
     if rc != FA_OK:
         raise FaError(rc, "fa_varlen_bwd")
     return dq, dk, dv
+
+
+def fa_varlen_fwd_noalloc(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                          softmax_scale: float, causal: bool, out=None, softmax_lse=None, stream=None):
+    """Forward without a workspace, for callers that cannot allocate device
+    memory: the library's own device buffer serves as scratch. Calls that can
+    overlap on the GPU must be serialised by the caller (they share it)."""
+    _check_qkv("q", q)
+    Tq, H, D = q.shape
+    _check_qkv("k", k, H, D)
+    _check_qkv("v", v, H, D)
+    _check_cu("cu_seqlens_q", cu_seqlens_q)
+    _check_cu("cu_seqlens_k", cu_seqlens_k)
+    batch = cu_seqlens_q.numel() - 1
+    if out is None:
+        out = torch.empty_like(q)
+    if softmax_lse is None:
+        softmax_lse = torch.empty((H, Tq), dtype=torch.float32, device=q.device)
+    rc = lib.fa_varlen_fwd_noalloc(_p(q), _p(k), _p(v), _p(cu_seqlens_q), _p(cu_seqlens_k), batch, Tq,
+                                   k.shape[0], int(max_seqlen_q), int(max_seqlen_k), H, D,
+                                   float(softmax_scale), int(bool(causal)), _p(out), _p(softmax_lse),
+                                   _stream(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_varlen_fwd_noalloc")
+    return out, softmax_lse
 
 
 def device_status(workspace, stream=None) -> int:
