@@ -82,8 +82,9 @@ typedef enum {
   FA_ERR_DEVICE_TIMEOUT = 6    /* device: a pipeline wait gave up after its time limit */
 } fa_status_t;
 
-/* Limits: batch <= 65535; total_q, total_k < 2^31 / num_heads rows;
- * num_heads * head_dim <= 65535 * 64. */
+/* Limits (FA_ERR_UNSUPPORTED beyond them): num_heads * head_dim < 2^31;
+ * total_q and total_k below 2^31 - 256; (total_q / 128 + batch + 1) *
+ * num_heads and (total_k / 128 + batch + 1) * num_heads below 2^31. */
 
 /* Workspace bytes needed by fa_varlen_fwd for these sizes. */
 size_t fa_varlen_fwd_workspace_size(int batch, int total_q, int num_heads, int head_dim);
@@ -126,7 +127,7 @@ fa_status_t fa_varlen_bwd(const void* dout, const void* q, const void* k, const 
  * - Returns FA_ERR_WORKSPACE, before any CUDA call, when the sizes need more
  *   scratch than that (fa_varlen_fwd_workspace_size(batch, total_q,
  *   num_heads, head_dim) > FA_NOALLOC_SCRATCH_BYTES; roughly
- *   total_q / 128 + batch must stay below about 32000).
+ *   total_q / 256 + 1.5 * batch must stay below about 32600).
  * - The first call on each device looks up the buffer's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
  *   before any stream capture.

@@ -3,12 +3,15 @@ scheduler bit for bit (as a multiset, plus the longest-first order).
 
 Tile counts follow page "Mecanismo cu_seqlens en FlashAttention",
 "Lógica de cálculo de longitud": sequence b has cu[b+1] - cu[b] rows, so it
-contributes ceil(len / 128) tiles; the cost of a tile is the number of tiles
-on the other side that it must visit under the (bottom-right) causal rule.
+contributes ceil(len / 256) forward items (query blocks of 256 rows) and
+ceil(len_k / 128) backward items (key tiles); the cost of an item is the
+number of 128-row tiles on the other side that it must visit under the
+(bottom-right) causal rule.
 """
 from __future__ import annotations
 
 FWD_BM = FWD_BN = 128
+FWD_ITEM_ROWS = 256
 BWD_BN, BWD_BM = 128, 64
 HEADER = 256
 BINS = 2048
@@ -24,7 +27,7 @@ def fwd_cost(t, lq, lk, causal):
     nk = -(-lk // FWD_BN)
     if not causal:
         return nk
-    rmax = min((t + 1) * FWD_BM, lq) - 1
+    rmax = min((t + 1) * FWD_ITEM_ROWS, lq) - 1
     last = rmax + lk - lq
     if last < 0:
         return 0
@@ -47,7 +50,7 @@ def work_list(cu_q, cu_k, causal, backward=False):
     out = []
     for b in range(len(cu_q) - 1):
         lq, lk = int(cu_q[b + 1] - cu_q[b]), int(cu_k[b + 1] - cu_k[b])
-        n = -(-(lk if backward else lq) // (BWD_BN if backward else FWD_BM))
+        n = -(-(lk if backward else lq) // (BWD_BN if backward else FWD_ITEM_ROWS))
         for t in range(n):
             c = bwd_cost(t, lq, lk, causal) if backward else fwd_cost(t, lq, lk, causal)
             out.append((b, t, min(c, BINS - 1)))
@@ -57,5 +60,5 @@ def work_list(cu_q, cu_k, causal, backward=False):
 def layout(batch, total_q, total_k, backward=False):
     seq_off = HEADER
     pairs = align(seq_off + 4 * (batch + 1), 256)
-    max_pairs = (total_k // BWD_BN if backward else total_q // FWD_BM) + batch + 1
+    max_pairs = (total_k // BWD_BN if backward else total_q // FWD_ITEM_ROWS) + batch + 1
     return {"seq_off": seq_off, "pairs": pairs, "max_pairs": max_pairs}

@@ -12,10 +12,12 @@
 
 namespace fa {
 
-// Forward tiles: a work item is 128 query rows of one (sequence, head);
-// keys stream through in tiles of 128.
+// Forward tiles: a work item is 256 query rows of one (sequence, head),
+// computed as two tiles of 128 rows that share every key tile; keys stream
+// through in tiles of 128.
 constexpr int kFwdBM = 128;
 constexpr int kFwdBN = 128;
+constexpr int kFwdItemRows = 256;
 // Backward tiles: a work item is 128 key rows of one (sequence, head);
 // queries stream through in tiles of 64.
 constexpr int kBwdBN = 128;
@@ -55,7 +57,7 @@ __host__ __device__ inline WsLayout ws_layout(bool backward, int batch, int tota
   size_t off = sizeof(WsHeader);
   L.seq_off = off;
   off = align_up(off + sizeof(int32_t) * (static_cast<size_t>(batch) + 1), 256);
-  L.max_pairs = backward ? max_pairs(batch, total_k, kBwdBN) : max_pairs(batch, total_q, kFwdBM);
+  L.max_pairs = backward ? max_pairs(batch, total_k, kBwdBN) : max_pairs(batch, total_q, kFwdItemRows);
   L.pairs = off;
   off = align_up(off + 8 * static_cast<size_t>(L.max_pairs), 256);
   if (backward) {
@@ -86,14 +88,15 @@ __device__ __forceinline__ SeqInfo seq_info(const int32_t* cu_q, const int32_t* 
   return s;
 }
 
-// Number of key tiles visible from query tile t (rows t*BM ..), given the
-// bottom-right causal rule j <= i + (lk - lq). Tiles wholly above the
-// diagonal are skipped.
-__host__ __device__ inline int fwd_num_k_tiles(int t, int lq, int lk, bool causal) {
+// Number of key tiles (kFwdBN keys) visible from the query rows below
+// row_end (clamped to lq), given the bottom-right causal rule
+// j <= i + (lk - lq). Tiles wholly above the diagonal are skipped; the
+// visible tiles are always a prefix 0 .. n-1.
+__host__ __device__ inline int fwd_k_tiles(int row_end, int lq, int lk, bool causal) {
   if (lk <= 0 || lq <= 0) return 0;
   const int nk = (lk + kFwdBN - 1) / kFwdBN;
   if (!causal) return nk;
-  const int rmax = ((t + 1) * kFwdBM < lq ? (t + 1) * kFwdBM : lq) - 1;
+  const int rmax = (row_end < lq ? row_end : lq) - 1;
   const long long last = static_cast<long long>(rmax) + lk - lq;
   if (last < 0) return 0;
   const long long n = last / kFwdBN + 1;

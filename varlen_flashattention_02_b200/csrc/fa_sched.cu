@@ -3,17 +3,17 @@
 // From the device-resident cumulative offsets, one CTA
 //   1. checks them (cu[0] = 0, non-decreasing, cu[batch] = total, every
 //      length <= max_seqlen) and records FA_ERR_BAD_SEQLENS otherwise;
-//   2. counts the tiles of every sequence (forward: query tiles of 128
+//   2. counts the tiles of every sequence (forward: query blocks of 256
 //      rows; backward: key tiles of 128 rows) and prefix-sums them;
 //   3. orders all (sequence, tile) pairs by their number of visible tiles on
 //      the other side, most work first, so that the persistent kernels,
 //      which take pairs in order, start the longest items first.
-// No padding is ever enumerated: a sequence of length n yields ceil(n/128)
-// pairs. Pages: "Mecanismo cu_seqlens en FlashAttention", "Lógica de cálculo
-// de longitud" (lengths from offsets) and "Consejos de optimización" (long
-// and short sequences mixed in one batch); "Flash-Atención y
-// Flash-Atención-2", FlashAttention-2 section (parallelism over the sequence
-// dimension as well as batch and heads).
+// No padding is ever enumerated: a sequence of length n yields ceil(n/T)
+// pairs (T = 256 forward, 128 backward). Pages: "Mecanismo cu_seqlens en
+// FlashAttention", "Lógica de cálculo de longitud" (lengths from offsets)
+// and "Consejos de optimización" (long and short sequences mixed in one
+// batch); "Flash-Atención y Flash-Atención-2", FlashAttention-2 section
+// (parallelism over the sequence dimension as well as batch and heads).
 #include "fa_common.cuh"
 #include "fa_kernels.h"
 
@@ -24,7 +24,7 @@ constexpr int kThreads = 1024;
 constexpr int kBins = 2048;  // cost buckets; costs above kBins-1 share the last
 
 __device__ __forceinline__ int pair_cost(const SeqInfo& s, int tile, int mode, bool causal) {
-  if (mode == 0) return fwd_num_k_tiles(tile, s.lq, s.lk, causal);
+  if (mode == 0) return fwd_k_tiles((tile + 1) * kFwdItemRows, s.lq, s.lk, causal);
   int b, e;
   bwd_q_tiles(tile, s.lq, s.lk, causal, &b, &e);
   return e - b;
@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(kThreads) sched_prep_kernel(SchedArgs a) {
   }
 
   // Tiles per sequence, exclusive prefix sum into seq_off.
-  const int tile = a.mode == 0 ? kFwdBM : kBwdBN;
+  const int tile = a.mode == 0 ? kFwdItemRows : kBwdBN;
   for (int base = 0; base < a.batch; base += kThreads) {
     const int b = base + tid;
     int n = 0;
