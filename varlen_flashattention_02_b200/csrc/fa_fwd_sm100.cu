@@ -266,19 +266,21 @@ __device__ __forceinline__ void mma_issuer(const FwdArgs& a, uint8_t* smem, Bars
 #pragma unroll
       for (int w = 0; w < 2; ++w) {
         if (j >= it.nk[w]) continue;
-        if (!wait_bar_warp(&bars.p_full[w], np[w] & 1, ab)) goto done;
         if (j == 0 && nq[w] > 0 && !wait_bar_warp(&bars.o_empty[w], (nq[w] - 1) & 1, ab)) goto done;
         const bool more = j + 1 < it.nk[w];
         if (more && !k_ready) {
           if (!wait_bar_warp(&bars.k_full[kst], ((kvj + 1) / NK) & 1, ab)) goto done;
           k_ready = true;
         }
+        // O_w (+)= P_w V_j with P read from TMEM, then S_w,j+1. Everything
+        // that does not depend on P (the waits above, the descriptors) is
+        // done before waiting for it, so the MMAs issue as soon as P lands.
+        const uint64_t v_desc = opaque_u64(v_desc0) + static_cast<uint64_t>((vst * L::kTileBytes) >> 4);
+        const uint32_t a_p = tmem + L::kSCol + w * BN;
+        const uint32_t d_o = tmem + L::kOCol + w * D;
+        if (!wait_bar_warp(&bars.p_full[w], np[w] & 1, ab)) goto done;
         tc_fence_after();
         if (elect_one()) {
-          // O_w (+)= P_w V_j, P read from TMEM.
-          const uint64_t v_desc = opaque_u64(v_desc0) + static_cast<uint64_t>((vst * L::kTileBytes) >> 4);
-          const uint32_t a_p = tmem + L::kSCol + w * BN;
-          const uint32_t d_o = tmem + L::kOCol + w * D;
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk)
             mma_ts(d_o, a_p + kk * 8, v_desc + static_cast<uint64_t>((kk * 2048) >> 4), kIdescO,
@@ -406,16 +408,18 @@ __device__ __forceinline__ void softmax_role(const FwdArgs& a, uint8_t* smem, Ba
         }
         tmem_st16(t_s + hh * 16, pk);
       }
+      // Hand P over first; the row sum is reduced afterwards, off the path
+      // to the next MMAs.
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.p_full[W]);
       {
         float a0, a1, b0, b1;
         f2_split(f2_add(ls2[0], ls2[1]), a0, a1);
         f2_split(f2_add(ls2[2], ls2[3]), b0, b1);
         l += (a0 + a1) + (b0 + b1);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.p_full[W]);
     }
     // Hand 1/l to the epilogue warpgroup; write the LSE of valid rows.
     if (nl > 0 && !wait_bar_warp(&bars.l_empty[W], (nl - 1) & 1, ab)) return;
