@@ -49,9 +49,9 @@ class OracleLib:
         lib = ctypes.CDLL(path)
         P = ctypes.c_void_p
         I = ctypes.c_int
-        lib.fa_oracle_fwd.argtypes = [P, P, P, I, P, P, I, I, I, ctypes.c_double, I, I, P, I, P, P]
+        lib.fa_oracle_fwd.argtypes = [P, P, P, I, P, P, I, I, I, I, ctypes.c_double, I, I, P, I, P, P]
         lib.fa_oracle_fwd.restype = I
-        lib.fa_oracle_bwd.argtypes = [P, P, P, P, I, P, P, I, I, I, ctypes.c_double, I, I, P, P, P, P]
+        lib.fa_oracle_bwd.argtypes = [P, P, P, P, I, P, P, I, I, I, I, ctypes.c_double, I, I, P, P, P, P]
         lib.fa_oracle_bwd.restype = I
         lib.fa_oracle_seqlens.argtypes = [P, I, P]
         lib.fa_oracle_seqlens.restype = I
@@ -78,9 +78,11 @@ class OracleLib:
         return int(self.lib.fa_oracle_elem_offset(_ptr(cu), b, r, heads, h, d))
 
     def fwd(self, q, k, v, cu_q, cu_k, scale: float, causal: bool, units=None, row_step: int = 1):
-        """Returns (out [Tq,H,d] f64, lse [H,Tq] f64). With ``units`` (list of
-        (b, h)), only those units are computed; with ``row_step`` > 1 only
-        query rows i % row_step == 0 of each unit. Other entries are NaN."""
+        """Returns (out [Tq,H,d] f64, lse [H,Tq] f64). k and v may have fewer
+        heads than q (grouped-query attention: query head h uses key/value
+        head h // (H // Hk)). With ``units`` (list of (b, h), h a query head),
+        only those units are computed; with ``row_step`` > 1 only query rows
+        i % row_step == 0 of each unit. Other entries are NaN."""
         q, dt = _as_input(q)
         k, dtk = _as_input(k)
         v, dtv = _as_input(v)
@@ -88,18 +90,21 @@ class OracleLib:
         cu_q = np.ascontiguousarray(cu_q, dtype=np.int32)
         cu_k = np.ascontiguousarray(cu_k, dtype=np.int32)
         Tq, H, d = q.shape
+        Hk = _kv_heads(H, k, v)
         out = np.full((Tq, H, d), np.nan)
         lse = np.full((H, Tq), np.nan)
         n, _keep, up = _units_arg(units)
         rc = self.lib.fa_oracle_fwd(_ptr(q), _ptr(k), _ptr(v), dt, _ptr(cu_q), _ptr(cu_k),
-                                    len(cu_q) - 1, H, d, float(scale), int(bool(causal)), n, up,
+                                    len(cu_q) - 1, H, Hk, d, float(scale), int(bool(causal)), n, up,
                                     int(row_step), _ptr(out), _ptr(lse))
         if rc != 0:
             raise MemoryError("oracle forward failed to allocate")
         return out, lse
 
     def bwd(self, q, k, v, dout, cu_q, cu_k, scale: float, causal: bool, units=None):
-        """Returns (dq, dk, dv) as f64 arrays shaped like q, k, v."""
+        """Returns (dq, dk, dv) as f64 arrays shaped like q, k, v. With
+        ``units`` (list of (b, hk), hk a key/value head), only those units
+        are computed: dk, dv of head hk and dq of the query heads it serves."""
         q, dt = _as_input(q)
         k, _ = _as_input(k)
         v, _ = _as_input(v)
@@ -107,13 +112,14 @@ class OracleLib:
         cu_q = np.ascontiguousarray(cu_q, dtype=np.int32)
         cu_k = np.ascontiguousarray(cu_k, dtype=np.int32)
         Tq, H, d = q.shape
+        Hk = _kv_heads(H, k, v)
         Tk = k.shape[0]
         dq = np.full((Tq, H, d), np.nan)
-        dk = np.full((Tk, H, d), np.nan)
-        dv = np.full((Tk, H, d), np.nan)
+        dk = np.full((Tk, Hk, d), np.nan)
+        dv = np.full((Tk, Hk, d), np.nan)
         n, _keep, up = _units_arg(units)
         rc = self.lib.fa_oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), dt, _ptr(cu_q),
-                                    _ptr(cu_k), len(cu_q) - 1, H, d, float(scale),
+                                    _ptr(cu_k), len(cu_q) - 1, H, Hk, d, float(scale),
                                     int(bool(causal)), n, up, _ptr(dq), _ptr(dk), _ptr(dv))
         if rc != 0:
             raise MemoryError("oracle backward failed to allocate")
@@ -136,6 +142,13 @@ def _as_input(x: np.ndarray):
     if x.dtype == np.uint16:
         return np.ascontiguousarray(x), IN_BF16
     return np.ascontiguousarray(x, dtype=np.float64), IN_F64
+
+
+def _kv_heads(H: int, k: np.ndarray, v: np.ndarray) -> int:
+    Hk = k.shape[1]
+    if v.shape[1] != Hk or Hk < 1 or H % Hk != 0:
+        raise ValueError(f"query heads ({H}) must be a multiple of key/value heads ({Hk})")
+    return Hk
 
 
 def _units_arg(units):

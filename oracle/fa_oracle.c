@@ -22,17 +22,24 @@
  *  - "Flash-Atención y Flash-Atención-2" (zepes.com), sections on the
  *    backward: the backward exists and recomputes probabilities; the
  *    gradient formulas themselves are not printed, so the backward here is
- *    the chain rule of the forward definition.
+ *    the chain rule of the forward definition. Same page, FlashAttention-2
+ *    section on multi-query and grouped-query attention: several query
+ *    heads attend to one key/value head.
  *
  * Readings where the pages are silent (each also listed in the design notes):
  *  - causal alignment when lq != lk is bottom-right: key j is visible from
  *    query i iff j <= i + (lk - lq);
  *  - a row with no visible key has output 0 and logsumexp -inf, and adds
  *    nothing to any gradient;
- *  - logsumexp is the natural log of the sum of exp of the SCALED scores.
+ *  - logsumexp is the natural log of the sum of exp of the SCALED scores;
+ *  - with H query heads and Hk key/value heads (H a multiple of Hk; Hk = H
+ *    is ordinary multi-head attention, Hk = 1 multi-query), query head h
+ *    uses key/value head h / (H / Hk): consecutive query heads share one.
+ *    The key/value gradients of a shared head are the sums over its group.
  *
- * Layouts: q/dout/out/dq are [total_q, H, d]; k/v/dk/dv are [total_k, H, d];
- * lse is [H, total_q]. Element (row, h, c) sits at (row*H + h)*d + c.
+ * Layouts: q/dout/out/dq are [total_q, H, d]; k/v/dk/dv are [total_k, Hk, d];
+ * lse is [H, total_q]. Element (row, h, c) of a tensor with H heads sits at
+ * (row*H + h)*d + c.
  * Inputs are either fp64 or raw bf16 bit patterns (widened exactly).
  *
  * Each (sequence, head) unit is independent; OpenMP runs units in parallel.
@@ -136,9 +143,11 @@ static void unit_at(int64_t u, int H, const int32_t* units, int* b, int* h) {
  * row_step > 1 computes only query rows i with i % row_step == 0 (rows are
  * independent in the forward, so a sample of rows is exact). */
 int fa_oracle_fwd(const void* q, const void* k, const void* v, int dtype,
-                  const int32_t* cu_q, const int32_t* cu_k, int batch, int H, int d,
+                  const int32_t* cu_q, const int32_t* cu_k, int batch, int H, int Hk, int d,
                   double scale, int causal, int n_units, const int32_t* units, int row_step,
                   double* out, double* lse) {
+  if (Hk < 1 || H % Hk != 0) return -2;
+  const int g = H / Hk;  /* query heads per key/value head */
   const int64_t total_q = cu_q[batch];
   const int64_t nu = unit_count(batch, H, n_units, units);
   int err = 0;
@@ -155,7 +164,8 @@ int fa_oracle_fwd(const void* q, const void* k, const void* v, int dtype,
       free(koffs);
       continue;
     }
-    for (int64_t j = 0; j < lk; ++j) koffs[j] = fa_oracle_elem_offset(cu_k, b, j, H, h, d);
+    const int hk = h / g;
+    for (int64_t j = 0; j < lk; ++j) koffs[j] = fa_oracle_elem_offset(cu_k, b, j, Hk, hk, d);
     for (int64_t i = 0; i < lq; i += (row_step > 1 ? row_step : 1)) {
       const int64_t qoff = fa_oracle_elem_offset(cu_q, b, i, H, h, d);
       int64_t nvis = score_row(q, k, dtype, qoff, koffs, i, lq, lk, d, scale, causal, s);
@@ -177,17 +187,21 @@ int fa_oracle_fwd(const void* q, const void* k, const void* v, int dtype,
 /* Backward of L = sum(out * dout), recomputed from the inputs alone:
  *   P = softmax(S), dV = P^T dO, dP = dO V^T, D_i = sum_j P_ij dP_ij,
  *   dS = P * (dP - D), dQ = scale dS K, dK = scale dS^T Q.
- * Rows are visited one by one; dK and dV of the unit accumulate over rows. */
+ * A unit here is (sequence, key/value head): its query heads are visited one
+ * after the other and their rows one by one; dK and dV of the unit
+ * accumulate over all of them. */
 int fa_oracle_bwd(const void* q, const void* k, const void* v, const void* dout, int dtype,
-                  const int32_t* cu_q, const int32_t* cu_k, int batch, int H, int d,
+                  const int32_t* cu_q, const int32_t* cu_k, int batch, int H, int Hk, int d,
                   double scale, int causal, int n_units, const int32_t* units,
                   double* dq, double* dk, double* dv) {
-  const int64_t nu = unit_count(batch, H, n_units, units);
+  if (Hk < 1 || H % Hk != 0) return -2;
+  const int g = H / Hk;  /* query heads per key/value head */
+  const int64_t nu = unit_count(batch, Hk, n_units, units);
   int err = 0;
 #pragma omp parallel for schedule(dynamic, 1)
   for (int64_t u = 0; u < nu; ++u) {
-    int b, h;
-    unit_at(u, H, units, &b, &h);
+    int b, hk;
+    unit_at(u, Hk, units, &b, &hk);
     const int64_t lq = cu_q[b + 1] - cu_q[b], lk = cu_k[b + 1] - cu_k[b];
     const size_t nk = (size_t)(lk > 0 ? lk : 1);
     double* p = (double*)malloc(sizeof(double) * nk);
@@ -201,12 +215,13 @@ int fa_oracle_bwd(const void* q, const void* k, const void* v, const void* dout,
       continue;
     }
     for (int64_t j = 0; j < lk; ++j) {
-      koffs[j] = fa_oracle_elem_offset(cu_k, b, j, H, h, d);
+      koffs[j] = fa_oracle_elem_offset(cu_k, b, j, Hk, hk, d);
       for (int c = 0; c < d; ++c) {
         dk[koffs[j] + c] = 0.0;
         dv[koffs[j] + c] = 0.0;
       }
     }
+    for (int h = hk * g; h < (hk + 1) * g; ++h)
     for (int64_t i = 0; i < lq; ++i) {
       const int64_t qoff = fa_oracle_elem_offset(cu_q, b, i, H, h, d);
       int64_t nvis = score_row(q, k, dtype, qoff, koffs, i, lq, lk, d, scale, causal, p);

@@ -173,35 +173,42 @@ def pin_constant_v(orc):
 
 
 def _brute(q, k, v, do, cu_q, cu_k, scale, causal):
-    """Pure-Python definition with math.fsum, row by row (no numpy math)."""
+    """Pure-Python definition with math.fsum, row by row (no numpy math).
+    k and v may have fewer heads than q: query head h reads key/value head
+    h // (H // Hk)."""
     T, H, d = q.shape
+    g = H // k.shape[1]
     out = [[[0.0] * d for _ in range(H)] for _ in range(T)]
     lse = [[0.0] * T for _ in range(H)]
     for b in range(len(cu_q) - 1):
         lq, lk = int(cu_q[b + 1] - cu_q[b]), int(cu_k[b + 1] - cu_k[b])
         for h in range(H):
+            hk = h // g
             for i in range(lq):
                 qi = [float(x) for x in q[cu_q[b] + i, h]]
                 vis = [j for j in range(lk) if _visible(i, j, lq, lk, causal)]
                 if not vis:
                     lse[h][cu_q[b] + i] = -math.inf
                     continue
-                s = {j: scale * math.fsum(qi[c] * float(k[cu_k[b] + j, h, c]) for c in range(d))
+                s = {j: scale * math.fsum(qi[c] * float(k[cu_k[b] + j, hk, c]) for c in range(d))
                      for j in vis}
                 mx = max(s.values())
                 z = math.fsum(math.exp(s[j] - mx) for j in vis)
                 lse[h][cu_q[b] + i] = mx + math.log(z)
                 for c in range(d):
                     out[cu_q[b] + i][h][c] = math.fsum(
-                        math.exp(s[j] - mx) / z * float(v[cu_k[b] + j, h, c]) for j in vis)
+                        math.exp(s[j] - mx) / z * float(v[cu_k[b] + j, hk, c]) for j in vis)
     return np.array(out), np.array(lse)
 
 
 def pin_bruteforce(orc):
-    """Tiny inputs (lq, lk <= 4, d <= 4) against the pure-Python brute force."""
+    """Tiny inputs (lq, lk <= 4, d <= 4) against the pure-Python brute force,
+    with as many key/value heads as query heads and with 2 query heads per
+    key/value head."""
     for causal in (False, True):
-        for lq, lk in (([3, 4, 1], [4, 2, 3]),):
+        for lq, lk, Hk in (([3, 4, 1], [4, 2, 3], 2), ([3, 4, 1], [4, 2, 3], 1)):
             q, k, v, do, cu_q, cu_k = _batch(17, H=2, d=3, lq=lq, lk=lk)
+            k, v = k[:, :Hk], v[:, :Hk]
             out, lse = orc.fwd(q, k, v, cu_q, cu_k, 0.8, causal)
             bo, bl = _brute(q, k, v, do, cu_q, cu_k, 0.8, causal)
             assert np.allclose(out, bo, rtol=0, atol=1e-13)
@@ -342,9 +349,73 @@ def pin_row_and_unit_sampling(orc):
         assert np.array_equal(g[2][sk, 1], g_full[2][sk, 1])
 
 
+def _repeat_heads(x, g):
+    """[T, Hk, d] -> [T, Hk * g, d], each key/value head repeated g times in a
+    row (query heads h = hk*g .. hk*g + g - 1 read head hk)."""
+    return np.repeat(x, g, axis=1)
+
+
+def pin_gqa_is_repeated_heads(orc):
+    """Grouped-query attention is multi-head attention on key/value heads
+    repeated across their group (page "Flash-Atención y Flash-Atención-2",
+    FlashAttention-2 section: several query heads attend to one key/value
+    head): out, lse and dq equal those of the repeated-head inputs exactly,
+    and dk, dv of a shared head are the sums over its group."""
+    for H, Hk in ((6, 2), (6, 3), (4, 1)):
+        g = H // Hk
+        # d >= H keeps a planted head-stride mistake in bounds (see the mutants).
+        q, k, v, do, cu_q, cu_k = _batch(24, H=H, d=6, lq=[7, 4, 9], lk=[6, 8, 9])
+        k, v = k[:, :Hk].copy(), v[:, :Hk].copy()
+        kr, vr = _repeat_heads(k, g), _repeat_heads(v, g)
+        for causal in (False, True):
+            o, l = orc.fwd(q, k, v, cu_q, cu_k, 0.55, causal)
+            ro, rl = orc.fwd(q, kr, vr, cu_q, cu_k, 0.55, causal)
+            assert np.array_equal(o, ro) and np.array_equal(l, rl)
+            dq, dk, dv = orc.bwd(q, k, v, do, cu_q, cu_k, 0.55, causal)
+            rq, rk, rv = orc.bwd(q, kr, vr, do, cu_q, cu_k, 0.55, causal)
+            assert np.array_equal(dq, rq)
+            T = k.shape[0]
+            assert np.allclose(dk, rk.reshape(T, Hk, g, -1).sum(axis=2), rtol=0, atol=1e-12)
+            assert np.allclose(dv, rv.reshape(T, Hk, g, -1).sum(axis=2), rtol=0, atol=1e-12)
+
+
+def pin_gqa_torch_sdpa(orc):
+    """Grouped-query attention against torch's fp64 CPU
+    scaled_dot_product_attention with enable_gqa (which maps query head h to
+    key/value head h // (H // Hk)) and its autograd."""
+    import torch
+
+    H, Hk = 4, 2
+    for causal in (False, True):
+        q, k, v, do, cu_q, cu_k = _batch(25, H=H, d=6, lq=[5, 8], lk=[8, 5])
+        k, v = k[:, :Hk].copy(), v[:, :Hk].copy()
+        out, lse = orc.fwd(q, k, v, cu_q, cu_k, 0.5, causal)
+        dq, dk, dv = orc.bwd(q, k, v, do, cu_q, cu_k, 0.5, causal)
+        for b in range(2):
+            sq, sk = slice(cu_q[b], cu_q[b + 1]), slice(cu_k[b], cu_k[b + 1])
+            lq, lk = cu_q[b + 1] - cu_q[b], cu_k[b + 1] - cu_k[b]
+            mask = torch.tensor([[_visible(i, j, lq, lk, causal) for j in range(lk)] for i in range(lq)])
+            rows_ok = mask.any(dim=1)
+            tmask = mask | ~rows_ok[:, None]
+            tq = torch.tensor(q[sq]).transpose(0, 1).requires_grad_(True)
+            tk = torch.tensor(k[sk]).transpose(0, 1).requires_grad_(True)
+            tv = torch.tensor(v[sk]).transpose(0, 1).requires_grad_(True)
+            to = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=tmask, scale=0.5,
+                                                                  enable_gqa=True)
+            tdo = torch.tensor(do[sq]).transpose(0, 1) * rows_ok[None, :, None]
+            (to * tdo).sum().backward()
+            got = torch.tensor(out[sq]).transpose(0, 1)
+            assert torch.allclose(got[:, rows_ok], to.detach()[:, rows_ok], rtol=0, atol=1e-12)
+            assert torch.allclose(torch.tensor(dq[sq]).transpose(0, 1)[:, rows_ok],
+                                  tq.grad[:, rows_ok], rtol=0, atol=1e-11)
+            assert torch.allclose(torch.tensor(dk[sk]).transpose(0, 1), tk.grad, rtol=0, atol=1e-11)
+            assert torch.allclose(torch.tensor(dv[sk]).transpose(0, 1), tv.grad, rtol=0, atol=1e-11)
+
+
 ALL_PINS = [
     pin_seqlens_golden, pin_elem_offset, pin_rows_sum_to_one, pin_lse_bounds,
     pin_varlen_independence, pin_single_key, pin_causal_row0, pin_constant_v,
     pin_bruteforce, pin_torch_sdpa, pin_finite_differences, pin_grad_invariants,
-    pin_empty_rows, pin_bf16_path, pin_row_and_unit_sampling,
+    pin_empty_rows, pin_bf16_path, pin_row_and_unit_sampling, pin_gqa_is_repeated_heads,
+    pin_gqa_torch_sdpa,
 ]

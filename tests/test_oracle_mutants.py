@@ -28,6 +28,9 @@ MUTANTS = {
     "lse-row-index": ("lse[(int64_t)h * total_q + cu_q[b] + i] = l;", "lse[(int64_t)h * total_q + i] = l;"),
     "seqlen-off-by-one": ("len[b] = cu[b + 1] - cu[b];", "len[b] = cu[b + 1] - cu[b] - 1;"),
     "bf16-widen-shift": ("<< 16;", "<< 15;"),
+    "gqa-interleaved-heads": ("const int hk = h / g;", "const int hk = h % Hk;"),
+    "gqa-bwd-one-head-per-group": ("for (int h = hk * g; h < (hk + 1) * g; ++h)",
+                                   "for (int h = hk * g; h < hk * g + 1; ++h)"),
 }
 
 
