@@ -112,6 +112,33 @@ fa_status_t fa_varlen_bwd(const void* dout, const void* q, const void* k, const 
                           int head_dim, float softmax_scale, int causal, void* dq, void* dk, void* dv,
                           void* workspace, size_t workspace_bytes, fa_cuda_stream_t stream);
 
+/* Grouped-query and multi-query attention (page "Flash-Atención y
+ * Flash-Atención-2", FlashAttention-2 section: several query heads attend to
+ * one key/value head, which shrinks the key/value cache). Same as
+ * fa_varlen_fwd / fa_varlen_bwd, except that k, v, dk and dv have
+ * num_heads_k heads:
+ *   k, v, dk, dv : bf16 [total_k, num_heads_k, head_dim]
+ * num_heads must be a multiple of num_heads_k (else FA_ERR_INVALID_ARGUMENT);
+ * query head h reads key/value head h / (num_heads / num_heads_k), i.e.
+ * consecutive query heads share one (the pages do not say which heads share;
+ * this is the mapping of repeating each key/value head over its group).
+ * dk and dv of a shared head are the sums over its query heads, accumulated
+ * on chip (no atomic additions). num_heads_k == num_heads is exactly
+ * fa_varlen_fwd / fa_varlen_bwd. The workspace sizes are those of
+ * fa_varlen_fwd_workspace_size / fa_varlen_bwd_workspace_size with the query
+ * head count. */
+fa_status_t fa_varlen_fwd_gqa(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                              const int32_t* cu_seqlens_k, int batch, int total_q, int total_k, int max_seqlen_q,
+                              int max_seqlen_k, int num_heads, int num_heads_k, int head_dim, float softmax_scale,
+                              int causal, void* out, float* softmax_lse, void* workspace, size_t workspace_bytes,
+                              fa_cuda_stream_t stream);
+fa_status_t fa_varlen_bwd_gqa(const void* dout, const void* q, const void* k, const void* v, const void* out,
+                              const float* softmax_lse, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                              int batch, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
+                              int num_heads, int num_heads_k, int head_dim, float softmax_scale, int causal,
+                              void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                              fa_cuda_stream_t stream);
+
 /* Forward for callers that cannot allocate device memory. The pages have no
  * counterpart of this entry point; it exists for the library's users.
  *

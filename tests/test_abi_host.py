@@ -97,3 +97,32 @@ def test_no_cpu_fallback_in_binding():
     assert "oracle" not in src
     for forbidden in ("softmax(", "matmul", "einsum", "@ "):
         assert forbidden not in src
+
+
+def _fwd_gqa(lib, Hk, **over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, cu_q=FAKE, cu_k=FAKE, batch=2, total_q=1024, total_k=1024, max_q=824,
+             max_k=724, H=12, D=64, scale=0.125, causal=0, out=FAKE, lse=FAKE, ws=FAKE, ws_bytes=64,
+             stream=None)
+    a.update(over)
+    return lib.fa_varlen_fwd_gqa(a["q"], a["k"], a["v"], a["cu_q"], a["cu_k"], a["batch"], a["total_q"],
+                                 a["total_k"], a["max_q"], a["max_k"], a["H"], Hk, a["D"], a["scale"], a["causal"],
+                                 a["out"], a["lse"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+def _bwd_gqa(lib, Hk, **over):
+    a = dict(do=FAKE, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, cu_q=FAKE, cu_k=FAKE, batch=2, total_q=1024,
+             total_k=1024, max_q=824, max_k=724, H=12, D=64, scale=0.125, causal=1, dq=FAKE, dk=FAKE, dv=FAKE,
+             ws=FAKE, ws_bytes=1024, stream=None)
+    a.update(over)
+    return lib.fa_varlen_bwd_gqa(a["do"], a["q"], a["k"], a["v"], a["o"], a["lse"], a["cu_q"], a["cu_k"],
+                                 a["batch"], a["total_q"], a["total_k"], a["max_q"], a["max_k"], a["H"], Hk, a["D"],
+                                 a["scale"], a["causal"], a["dq"], a["dk"], a["dv"], a["ws"], a["ws_bytes"],
+                                 a["stream"])
+
+
+@pytest.mark.parametrize("Hk,code", [(0, 1), (-1, 1), (5, 1), (24, 1), (13, 1), (1, 3), (4, 3), (12, 3)])
+def test_gqa_head_counts(lib, Hk, code):
+    """num_heads must be a positive multiple of num_heads_k (invalid argument,
+    1); valid counts get as far as the too-small workspace (3)."""
+    assert _fwd_gqa(lib, Hk) == code
+    assert _bwd_gqa(lib, Hk) == code

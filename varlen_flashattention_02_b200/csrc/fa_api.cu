@@ -82,8 +82,10 @@ int sm_count() {
 }
 
 // Shared size checks of both directions.
-fa_status_t check_sizes(int batch, int total_q, int total_k, int max_sq, int max_sk, int H, int D, float scale) {
+fa_status_t check_sizes(int batch, int total_q, int total_k, int max_sq, int max_sk, int H, int Hk, int D,
+                        float scale) {
   if (batch < 1 || total_q < 0 || total_k < 0 || max_sq < 0 || max_sk < 0 || H < 1) return FA_ERR_INVALID_ARGUMENT;
+  if (Hk < 1 || Hk > H || H % Hk != 0) return FA_ERR_INVALID_ARGUMENT;
   if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARGUMENT;
   if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
   // Row indices and TMA coordinates are int32; element offsets are 64-bit.
@@ -128,10 +130,20 @@ fa_status_t fa_varlen_fwd(const void* q, const void* k, const void* v, const int
                           const int32_t* cu_seqlens_k, int batch, int total_q, int total_k, int max_seqlen_q,
                           int max_seqlen_k, int num_heads, int head_dim, float softmax_scale, int causal,
                           void* out, float* softmax_lse, void* workspace, size_t workspace_bytes,
-                          fa_cuda_stream_t stream_) {
+                          fa_cuda_stream_t stream) {
+  return fa_varlen_fwd_gqa(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
+                           max_seqlen_k, num_heads, num_heads, head_dim, softmax_scale, causal, out, softmax_lse,
+                           workspace, workspace_bytes, stream);
+}
+
+fa_status_t fa_varlen_fwd_gqa(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                              const int32_t* cu_seqlens_k, int batch, int total_q, int total_k, int max_seqlen_q,
+                              int max_seqlen_k, int num_heads, int num_heads_k, int head_dim, float softmax_scale,
+                              int causal, void* out, float* softmax_lse, void* workspace, size_t workspace_bytes,
+                              fa_cuda_stream_t stream_) {
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  fa_status_t st = check_sizes(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, num_heads, head_dim,
-                               softmax_scale);
+  fa_status_t st = check_sizes(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, num_heads, num_heads_k,
+                               head_dim, softmax_scale);
   if (st != FA_OK) return st;
   if (!cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARGUMENT;
   if (total_q > 0 && (!q || !out || !softmax_lse || !aligned16(q) || !aligned16(out))) return FA_ERR_INVALID_ARGUMENT;
@@ -147,14 +159,16 @@ fa_status_t fa_varlen_fwd(const void* q, const void* k, const void* v, const int
   if (total_q == 0) return FA_OK;
 
   const int HD = num_heads * head_dim;
+  const int HkD = num_heads_k * head_dim;
   CUtensorMap tq, tk, tv;
   // With no keys at all every row is empty and K/V are never read; the maps
   // then point at q so that they are still well formed.
   const void* kp = total_k > 0 ? k : q;
   const void* vp = total_k > 0 ? v : q;
   const int krows = total_k > 0 ? total_k : total_q;
-  if (!encode_map(&tq, q, total_q, HD, fa::kFwdBM) || !encode_map(&tk, kp, krows, HD, fa::kFwdBN) ||
-      !encode_map(&tv, vp, krows, HD, fa::kFwdBN))
+  const int kcols = total_k > 0 ? HkD : HD;
+  if (!encode_map(&tq, q, total_q, HD, fa::kFwdBM) || !encode_map(&tk, kp, krows, kcols, fa::kFwdBN) ||
+      !encode_map(&tv, vp, krows, kcols, fa::kFwdBN))
     return FA_ERR_CUDA;
 
   const int sms = sm_count();
@@ -170,6 +184,7 @@ fa_status_t fa_varlen_fwd(const void* q, const void* k, const void* v, const int
   fa_args.H = num_heads;
   fa_args.D = head_dim;
   fa_args.total_q = total_q;
+  fa_args.group = num_heads / num_heads_k;
   fa_args.causal = causal ? 1 : 0;
   fa_args.scale_log2 = softmax_scale * 1.4426950408889634f;
   fa_args.grid = static_cast<int>(items < sms ? items : sms);
@@ -182,10 +197,21 @@ fa_status_t fa_varlen_bwd(const void* dout, const void* q, const void* k, const 
                           const float* softmax_lse, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
                           int batch, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int num_heads,
                           int head_dim, float softmax_scale, int causal, void* dq, void* dk, void* dv,
-                          void* workspace, size_t workspace_bytes, fa_cuda_stream_t stream_) {
+                          void* workspace, size_t workspace_bytes, fa_cuda_stream_t stream) {
+  return fa_varlen_bwd_gqa(dout, q, k, v, out, softmax_lse, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
+                           max_seqlen_q, max_seqlen_k, num_heads, num_heads, head_dim, softmax_scale, causal, dq, dk,
+                           dv, workspace, workspace_bytes, stream);
+}
+
+fa_status_t fa_varlen_bwd_gqa(const void* dout, const void* q, const void* k, const void* v, const void* out,
+                              const float* softmax_lse, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                              int batch, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
+                              int num_heads, int num_heads_k, int head_dim, float softmax_scale, int causal,
+                              void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                              fa_cuda_stream_t stream_) {
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  fa_status_t st = check_sizes(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, num_heads, head_dim,
-                               softmax_scale);
+  fa_status_t st = check_sizes(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, num_heads, num_heads_k,
+                               head_dim, softmax_scale);
   if (st != FA_OK) return st;
   if (!cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARGUMENT;
   if (total_q > 0 && (!q || !dout || !out || !softmax_lse || !dq || !aligned16(q) || !aligned16(dout) ||
@@ -204,6 +230,7 @@ fa_status_t fa_varlen_bwd(const void* dout, const void* q, const void* k, const 
   if (total_q == 0 && total_k == 0) return FA_OK;
 
   const int HD = num_heads * head_dim;
+  const int HkD = num_heads_k * head_dim;
   CUtensorMap tq, tk, tv, tdo;
   const void* anyp = total_q > 0 ? q : k;
   const void* qp = total_q > 0 ? q : anyp;
@@ -212,13 +239,17 @@ fa_status_t fa_varlen_bwd(const void* dout, const void* q, const void* k, const 
   const void* vp = total_k > 0 ? v : anyp;
   const int qrows = total_q > 0 ? total_q : total_k;
   const int krows = total_k > 0 ? total_k : total_q;
-  if (!encode_map(&tq, qp, qrows, HD, fa::kBwdBM) || !encode_map(&tdo, dop, qrows, HD, fa::kBwdBM) ||
-      !encode_map(&tk, kp, krows, HD, fa::kBwdBN) || !encode_map(&tv, vp, krows, HD, fa::kBwdBN))
+  // With one side empty the other side's pointer stands in; the widths then
+  // follow that tensor's head count.
+  const int qcols = total_q > 0 ? HD : HkD;
+  const int kcols = total_k > 0 ? HkD : HD;
+  if (!encode_map(&tq, qp, qrows, qcols, fa::kBwdBM) || !encode_map(&tdo, dop, qrows, qcols, fa::kBwdBM) ||
+      !encode_map(&tk, kp, krows, kcols, fa::kBwdBN) || !encode_map(&tv, vp, krows, kcols, fa::kBwdBN))
     return FA_ERR_CUDA;
 
   const int sms = sm_count();
   if (sms <= 0) return FA_ERR_CUDA;
-  const long long items = static_cast<long long>(L.max_pairs) * num_heads;
+  const long long items = static_cast<long long>(L.max_pairs) * num_heads_k;
   fa::BwdArgs b{};
   b.cu_q = cu_seqlens_q;
   b.cu_k = cu_seqlens_k;
@@ -234,6 +265,8 @@ fa_status_t fa_varlen_bwd(const void* dout, const void* q, const void* k, const 
   b.dqacc_offset = L.dqacc;
   b.tq_pad = L.tq_pad;
   b.H = num_heads;
+  b.Hk = num_heads_k;
+  b.group = num_heads / num_heads_k;
   b.D = head_dim;
   b.total_q = total_q;
   b.total_k = total_k;

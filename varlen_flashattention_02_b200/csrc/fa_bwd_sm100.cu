@@ -3,9 +3,11 @@
 // Three kernels per call, after the work-list preparation (key-tile mode):
 //  1. preprocess: Dv_i = sum_c dO_ic * O_ic (fp32, [H, rows]) and zero the
 //     fp32 dQ accumulator;
-//  2. main: one persistent CTA per SM takes (sequence, head, key-tile)
-//     items, longest first, from a global counter. For 128 keys K_j, V_j of one head it loops over
-//     the 64-row query tiles that see them, recomputing the probabilities
+//  2. main: one persistent CTA per SM takes (sequence, key/value head,
+//     key-tile) items, longest first, from a global counter. For 128 keys
+//     K_j, V_j of one key/value head it loops over the query heads that read
+//     that head (one, or a group under grouped-query attention) and the
+//     64-row query tiles that see the keys, recomputing the probabilities
 //     from the saved logsumexp instead of storing them:
 //        S^T  = K_j Q_i^T,  P^T = exp2(S^T*scale*log2e - lse_i*log2e)
 //        dP^T = V_j dO_i^T, dS^T = P^T * (dP^T - Dv_i)
@@ -80,23 +82,40 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= 512, "barrier block fits its reserved space");
 
+// An item is (sequence, key/value head hk, key tile j). Its steps visit the
+// query tiles i0 .. i0+nt-1 that see the key tile, for each query head of
+// hk's group in turn: step s is query head h0 + s / nt, tile i0 + s % nt.
+// dK and dV of the tile accumulate over all of them.
 struct Item {
-  int b, h, j;
+  int b, hk, j;
   SeqInfo s;
-  int i0, n;  // first query tile and number of steps
+  int i0, nt;  // first query tile and query tiles per head
+  int h0;      // first query head of the group
+  int n;       // steps: nt * group
 };
 
 __device__ __forceinline__ Item get_item(const BwdArgs& a, const int2* pairs, int idx) {
   Item it;
-  const int2 pr = pairs[idx / a.H];
-  it.h = idx % a.H;
+  const int2 pr = pairs[idx / a.Hk];
+  it.hk = idx % a.Hk;
+  it.h0 = it.hk * a.group;
   it.b = pr.x;
   it.j = pr.y;
   it.s = seq_info(a.cu_q, a.cu_k, it.b);
   int e;
   bwd_q_tiles(it.j, it.s.lq, it.s.lk, a.causal != 0, &it.i0, &e);
-  it.n = e - it.i0;
+  it.nt = e - it.i0;
+  it.n = it.nt * a.group;
   return it;
+}
+
+// Query head and query tile of step s of an item.
+struct Step {
+  int h, t;
+};
+__device__ __forceinline__ Step item_step(const Item& it, int s) {
+  const int r = s / it.nt;
+  return Step{it.h0 + r, it.i0 + s - r * it.nt};
 }
 
 template <int D, bool CAUSAL>
@@ -154,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
   const Abort ab{&bars.abort_flag, &hdr->status};
-  const int n_items = (hdr->status == FA_OK) ? static_cast<int>(hdr->n_pairs) * a.H : 0;
+  const int n_items = (hdr->status == FA_OK) ? static_cast<int>(hdr->n_pairs) * a.Hk : 0;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -170,19 +189,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int krow = it.s.k0 + it.j * BN;
         mbar_arrive_expect_tx(&bars.kv_full, 2 * L::kKTile);
         for (int c = 0; c < L::kChunks; ++c) {
-          tma_load_2d(&tm_k, &bars.kv_full, smem + L::kK + c * L::kKChunk, it.h * D + c * 64, krow);
-          tma_load_2d(&tm_v, &bars.kv_full, smem + L::kV + c * L::kKChunk, it.h * D + c * 64, krow);
+          tma_load_2d(&tm_k, &bars.kv_full, smem + L::kK + c * L::kKChunk, it.hk * D + c * 64, krow);
+          tma_load_2d(&tm_v, &bars.kv_full, smem + L::kV + c * L::kKChunk, it.hk * D + c * 64, krow);
         }
         for (int s = 0; s < it.n; ++s, ++p) {
           const int st = p % NQ;
           if (p >= NQ && !wait_bar(&bars.qdo_empty[st], ((p / NQ) - 1) & 1, ab)) goto producer_done;
-          const int qrow = it.s.q0 + (it.i0 + s) * BM;
+          const Step sp = item_step(it, s);
+          const int qrow = it.s.q0 + sp.t * BM;
           uint8_t* sq = smem + L::kQdo + 2 * st * L::kQTile;
           uint8_t* sdo = sq + L::kQTile;
           mbar_arrive_expect_tx(&bars.qdo_full[st], 2 * L::kQTile);
           for (int c = 0; c < L::kChunks; ++c) {
-            tma_load_2d(&tm_q, &bars.qdo_full[st], sq + c * L::kQChunk, it.h * D + c * 64, qrow);
-            tma_load_2d(&tm_do, &bars.qdo_full[st], sdo + c * L::kQChunk, it.h * D + c * 64, qrow);
+            tma_load_2d(&tm_q, &bars.qdo_full[st], sq + c * L::kQChunk, sp.h * D + c * 64, qrow);
+            tma_load_2d(&tm_do, &bars.qdo_full[st], sdo + c * L::kQChunk, sp.h * D + c * 64, qrow);
           }
         }
         ++m;
@@ -301,16 +321,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < it.n; ++s, ++p) {
         const int slot = p % NQ;
         if (p >= NQ && !wait_bar_warp(&bars.ld_empty[slot], ((p / NQ) - 1) & 1, ab)) goto loader_done;
-        const int qi = (it.i0 + s) * BM + r;  // row within the sequence
+        const Step sp = item_step(it, s);
+        const int qi = sp.t * BM + r;  // row within the sequence
         // Stored negated and in base 2: -lse*log2(e); -inf for rows outside
         // the sequence or without a visible key, which makes their P exactly 0.
         float nlse2 = -INFINITY, dv = 0.f;
         if (qi < it.s.lq) {
           const size_t gq = static_cast<size_t>(it.s.q0) + qi;
-          const float l = __ldg(a.lse + static_cast<size_t>(it.h) * a.total_q + gq);
+          const float l = __ldg(a.lse + static_cast<size_t>(sp.h) * a.total_q + gq);
           if (l != -INFINITY) {
             nlse2 = -l * 1.4426950408889634f;
-            dv = __ldg(dvec + static_cast<size_t>(it.h) * a.tq_pad + gq);
+            dv = __ldg(dvec + static_cast<size_t>(sp.h) * a.tq_pad + gq);
           }
         }
         float* ld = reinterpret_cast<float*>(smem + L::kLd) + slot * 2 * BM;
@@ -344,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (p >= 2 && !wait_bar_warp(&bars.ds_empty[pb], ((p >> 1) - 1) & 1, ab)) goto compute_done;
         tc_fence_after();
         const float* ld = reinterpret_cast<const float*>(smem + L::kLd) + slot * 2 * BM;
-        const int row0 = (it.i0 + s) * BM;  // first query row of the step
+        const int row0 = item_step(it, s).t * BM;  // first query row of the step
         // Visible iff kg <= row + diag, i.e. e >= kg - diag - row0; keys past
         // the sequence see nothing.
         int e_min = CAUSAL ? kg - diag - row0 : 0;
@@ -414,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item it = get_item(a, pairs, idx);
       const int kg = it.j * BN + t;
       const bool key_ok = kg < it.s.lk;
-      const size_t krow = (static_cast<size_t>(it.s.k0) + kg) * a.H + it.h;
+      const size_t krow = (static_cast<size_t>(it.s.k0) + kg) * a.Hk + it.hk;
       if (it.n == 0) {
         if (key_ok) {
           uint4* dk = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.dk) + krow * D);
@@ -449,8 +470,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         named_bar_sync(1, 128);
         if (t == 0) {
-          const size_t q0 = static_cast<size_t>(it.s.q0) + static_cast<size_t>(it.i0 + s) * BM;
-          bulk_reduce_add_f32(dqacc + (static_cast<size_t>(it.h) * a.tq_pad + q0) * D, stage, BM * D * 4);
+          const Step sp = item_step(it, s);
+          const size_t q0 = static_cast<size_t>(it.s.q0) + static_cast<size_t>(sp.t) * BM;
+          bulk_reduce_add_f32(dqacc + (static_cast<size_t>(sp.h) * a.tq_pad + q0) * D, stage, BM * D * 4);
           bulk_commit_group();
         }
       }

@@ -43,7 +43,11 @@
 //    stale maximum stays consistent with l, so the result is exact);
 //  * masking is applied only on the last key tile of a sequence and on
 //    tiles that cross the causal diagonal; tiles wholly above it are never
-//    loaded.
+//    loaded;
+//  * grouped- and multi-query attention ("Flash-Atención y Flash-Atención-2",
+//    FlashAttention-2 section): query head h reads key/value head
+//    h / (H / Hk); items of consecutive query heads are adjacent in the work
+//    order, so a shared K/V tile is usually still in L2 for the next one.
 #include "fa_common.cuh"
 #include "fa_kernels.h"
 
@@ -102,6 +106,7 @@ static_assert(sizeof(Bars) <= 512, "barrier block fits its reserved space");
 
 struct Item {
   int b, h, t;  // t: 256-row block of the sequence
+  int hk;       // key/value head of query head h
   SeqInfo s;
   int nk[2];    // key tiles visible from query tile w (0 when the tile is empty)
 };
@@ -110,6 +115,7 @@ __device__ __forceinline__ Item get_item(const FwdArgs& a, const int2* pairs, in
   Item it;
   const int2 pr = pairs[idx / a.H];
   it.h = idx % a.H;
+  it.hk = it.h / a.group;
   it.b = pr.x;
   it.t = pr.y;
   it.s = seq_info(a.cu_q, a.cu_k, it.b);
@@ -155,8 +161,8 @@ __device__ __forceinline__ void qk_producer(const CUtensorMap* tm_q, const CUten
       if (use > 0 && !wait_bar(&bars.k_empty[st], (use - 1) & 1, ab)) goto done;
       mbar_arrive_expect_tx(&bars.k_full[st], L::kTileBytes);
       for (int c = 0; c < L::kChunks; ++c)
-        tma_load_2d(tm_k, &bars.k_full[st], smem + L::kK + st * L::kTileBytes + c * kChunkBytes, it.h * D + c * 64,
-                    it.s.k0 + j * BN);
+        tma_load_2d(tm_k, &bars.k_full[st], smem + L::kK + st * L::kTileBytes + c * kChunkBytes,
+                    it.hk * D + c * 64, it.s.k0 + j * BN);
     }
   }
 done:
@@ -186,8 +192,8 @@ __device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, const FwdArg
       if (use > 0 && !wait_bar(&bars.v_empty[st], (use - 1) & 1, ab)) goto done;
       mbar_arrive_expect_tx(&bars.v_full[st], L::kTileBytes);
       for (int c = 0; c < L::kChunks; ++c)
-        tma_load_2d(tm_v, &bars.v_full[st], smem + L::kV + st * L::kTileBytes + c * kChunkBytes, it.h * D + c * 64,
-                    it.s.k0 + j * BN);
+        tma_load_2d(tm_v, &bars.v_full[st], smem + L::kV + st * L::kTileBytes + c * kChunkBytes,
+                    it.hk * D + c * 64, it.s.k0 + j * BN);
     }
   }
 done:

@@ -32,12 +32,13 @@ struct FwdArgs {
   void* workspace;   // header + pairs
   size_t pairs_offset;
   int H, D, total_q;
+  int group;         // query heads per key/value head (H / Hk)
   int causal;
   float scale_log2;  // softmax_scale * log2(e)
   int grid;          // persistent CTAs
 };
-// tm_q / tm_k / tm_v: 2-D maps over [rows, H*D] bf16, box 128 rows x 64
-// columns, 128-byte swizzle.
+// tm_q: 2-D map over [rows, H*D] bf16; tm_k / tm_v over [rows, Hk*D]; box
+// 128 rows x 64 columns, 128-byte swizzle.
 cudaError_t launch_fwd(const FwdArgs& a, const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                        cudaStream_t stream);
 
@@ -53,15 +54,17 @@ struct BwdArgs {
   void* workspace;
   size_t pairs_offset, dvec_offset, dqacc_offset;
   int tq_pad;
-  int H, D, total_q, total_k;
+  int H, D, total_q, total_k;  // H: query heads
+  int Hk, group;               // key/value heads, query heads per key/value head
   int causal;
   float scale;        // softmax_scale
   float scale_log2;   // softmax_scale * log2(e)
   int grid;
 };
 // Backward in three launches: preprocess (rowsum(dO*O) and zero the dQ
-// accumulator), main, dQ conversion. tm_q / tm_do: box 64 rows x 64 columns;
-// tm_k / tm_v: box 128 rows x 64 columns; all 128-byte swizzle.
+// accumulator), main, dQ conversion. tm_q / tm_do: [rows, H*D], box 64 rows x
+// 64 columns; tm_k / tm_v: [rows, Hk*D], box 128 rows x 64 columns; all
+// 128-byte swizzle.
 cudaError_t launch_bwd_preprocess(const BwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_main(const BwdArgs& a, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                             const CUtensorMap& tm_v, const CUtensorMap& tm_do, cudaStream_t stream);

@@ -49,6 +49,11 @@ def _load():
     lib.fa_varlen_bwd.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, ctypes.c_float, I,
                                   P, P, P, P, S, P]
     lib.fa_varlen_bwd.restype = I
+    lib.fa_varlen_fwd_gqa.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, I, ctypes.c_float, I, P, P, P, S, P]
+    lib.fa_varlen_fwd_gqa.restype = I
+    lib.fa_varlen_bwd_gqa.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, ctypes.c_float, I,
+                                      P, P, P, P, S, P]
+    lib.fa_varlen_bwd_gqa.restype = I
     lib.fa_get_device_status.argtypes = [P, P]
     lib.fa_get_device_status.restype = I
     lib.fa_varlen_fwd_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, ctypes.c_float, I, P, P, P]
@@ -63,8 +68,8 @@ def _load():
 lib = _load()
 
 EXPORTED = ("fa_varlen_fwd_workspace_size", "fa_varlen_bwd_workspace_size", "fa_varlen_fwd",
-            "fa_varlen_bwd", "fa_varlen_fwd_noalloc", "fa_get_device_status", "fa_set_kernel_events",
-            "fa_status_string")
+            "fa_varlen_bwd", "fa_varlen_fwd_gqa", "fa_varlen_bwd_gqa", "fa_varlen_fwd_noalloc",
+            "fa_get_device_status", "fa_set_kernel_events", "fa_status_string")
 
 
 def _p(t):
@@ -151,6 +156,76 @@ def fa_varlen_bwd(dout, q, k, v, out, softmax_lse, cu_seqlens_q, cu_seqlens_k, m
                            _p(workspace), workspace.numel(), _stream(stream))
     if rc != FA_OK:
         raise FaError(rc, "fa_varlen_bwd")
+    return dq, dk, dv
+
+
+def _kv_heads(H, k):
+    Hk = k.shape[1]
+    if Hk < 1 or H % Hk != 0:
+        raise ValueError(f"query heads ({H}) must be a multiple of key/value heads ({Hk})")
+    return Hk
+
+
+def fa_varlen_fwd_gqa(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                      softmax_scale: float, causal: bool, out=None, softmax_lse=None, workspace=None,
+                      stream=None):
+    """Grouped-/multi-query forward: k and v have Hk heads, H a multiple of
+    Hk; query head h reads key/value head h // (H // Hk). Returns (out,
+    softmax_lse) as fa_varlen_fwd does."""
+    _check_qkv("q", q)
+    Tq, H, D = q.shape
+    _check_qkv("k", k)
+    Hk = _kv_heads(H, k)
+    _check_qkv("k", k, Hk, D)
+    _check_qkv("v", v, Hk, D)
+    _check_cu("cu_seqlens_q", cu_seqlens_q)
+    _check_cu("cu_seqlens_k", cu_seqlens_k)
+    batch = cu_seqlens_q.numel() - 1
+    if out is None:
+        out = torch.empty_like(q)
+    if softmax_lse is None:
+        softmax_lse = torch.empty((H, Tq), dtype=torch.float32, device=q.device)
+    need = fwd_workspace_size(batch, Tq, H, D)
+    if workspace is None:
+        workspace = new_workspace(need, q.device)
+    rc = lib.fa_varlen_fwd_gqa(_p(q), _p(k), _p(v), _p(cu_seqlens_q), _p(cu_seqlens_k), batch, Tq,
+                               k.shape[0], int(max_seqlen_q), int(max_seqlen_k), H, Hk, D,
+                               float(softmax_scale), int(bool(causal)), _p(out), _p(softmax_lse),
+                               _p(workspace), workspace.numel(), _stream(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_varlen_fwd_gqa")
+    return out, softmax_lse
+
+
+def fa_varlen_bwd_gqa(dout, q, k, v, out, softmax_lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
+                      max_seqlen_k: int, softmax_scale: float, causal: bool, dq=None, dk=None, dv=None,
+                      workspace=None, stream=None):
+    """Grouped-/multi-query backward: dk, dv have Hk heads and hold the sums
+    over each key/value head's query heads. Returns (dq, dk, dv)."""
+    _check_qkv("q", q)
+    Tq, H, D = q.shape
+    _check_qkv("k", k)
+    Hk = _kv_heads(H, k)
+    for name, t in (("k", k), ("v", v)):
+        _check_qkv(name, t, Hk, D)
+    for name, t in (("dout", dout), ("out", out)):
+        _check_qkv(name, t, H, D)
+    _check_cu("cu_seqlens_q", cu_seqlens_q)
+    _check_cu("cu_seqlens_k", cu_seqlens_k)
+    batch = cu_seqlens_q.numel() - 1
+    Tk = k.shape[0]
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = bwd_workspace_size(batch, Tq, Tk, H, D)
+    if workspace is None:
+        workspace = new_workspace(need, q.device)
+    rc = lib.fa_varlen_bwd_gqa(_p(dout), _p(q), _p(k), _p(v), _p(out), _p(softmax_lse), _p(cu_seqlens_q),
+                               _p(cu_seqlens_k), batch, Tq, Tk, int(max_seqlen_q), int(max_seqlen_k), H, Hk, D,
+                               float(softmax_scale), int(bool(causal)), _p(dq), _p(dk), _p(dv),
+                               _p(workspace), workspace.numel(), _stream(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_varlen_bwd_gqa")
     return dq, dk, dv
 
 

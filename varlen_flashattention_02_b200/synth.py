@@ -79,7 +79,12 @@ class Workload:
     causal: bool
     seed: int
     with_grad: bool = False
+    heads_k: int | None = None  # key/value heads (grouped-query attention); None: = heads
     _tensors: dict = field(default_factory=dict, repr=False)
+
+    @property
+    def kv_heads(self) -> int:
+        return self.heads if self.heads_k is None else self.heads_k
 
     @property
     def batch(self) -> int:
@@ -102,24 +107,25 @@ class Workload:
         return int(np.max(np.diff(self.cu_k))) if self.batch else 0
 
     def tensors(self) -> dict:
-        """q, k, v (and dout) as bf16 bits, [tokens, heads, head_dim]."""
+        """q, dout as bf16 bits [tokens, heads, head_dim]; k, v as
+        [tokens, kv_heads, head_dim]. Drawn in the order q, k, v, dout."""
         if not self._tensors:
             rng = np.random.default_rng(self.seed)
-            H, d = self.heads, self.head_dim
+            H, Hk, d = self.heads, self.kv_heads, self.head_dim
             self._tensors["q"] = bf16_normal(rng, (self.total_q, H, d))
-            self._tensors["k"] = bf16_normal(rng, (self.total_k, H, d))
-            self._tensors["v"] = bf16_normal(rng, (self.total_k, H, d))
+            self._tensors["k"] = bf16_normal(rng, (self.total_k, Hk, d))
+            self._tensors["v"] = bf16_normal(rng, (self.total_k, Hk, d))
             self._tensors["dout"] = bf16_normal(rng, (self.total_q, H, d))
         return self._tensors
 
 
 def make_workload(name: str, lengths_q, lengths_k=None, heads=1, head_dim=64,
-                  causal=False, seed=0, scale=None, with_grad=False) -> Workload:
+                  causal=False, seed=0, scale=None, with_grad=False, heads_k=None) -> Workload:
     lengths_k = lengths_q if lengths_k is None else lengths_k
     if scale is None:
         scale = 1.0 / math.sqrt(head_dim)
     return Workload(name, cu_from_lengths(lengths_q), cu_from_lengths(lengths_k), heads,
-                    head_dim, float(scale), bool(causal), int(seed), with_grad)
+                    head_dim, float(scale), bool(causal), int(seed), with_grad, heads_k)
 
 
 def standard_workload(n: int, causal: bool | None = None, head_dim: int | None = None) -> Workload:
