@@ -361,14 +361,18 @@ def fwd_only_workloads(dev, stream, flush, peak, iters=10):
     from varlen_flashattention_02_b200 import fa_varlen
 
     res = {}
+    gqa = lambda: synth.make_workload("gqa", synth.lengths_uniform(5, synth.TOTAL_TOKENS, 512, 8192), heads=32,
+                                      head_dim=128, causal=True, seed=5, heads_k=8)
     specs = [("varlen-2seq-h12-d64 (cu_q=[0,200,1024], cu_k=[0,300,1024])", 1, {}),
              ("fixed-8x2048-h16-d128 non-causal", 2, {"causal": False}),
              ("fixed-8x2048-h16-d128 causal", 2, {"causal": True}),
              ("packed-16k-U128..4096-h32-d128 causal", 3, {}),
              ("long-1x16384-h16-d64 causal", 4, {"head_dim": 64}),
-             ("long-1x16384-h16-d128 causal", 4, {"head_dim": 128})]
+             ("long-1x16384-h16-d128 causal", 4, {"head_dim": 128}),
+             ("grouped-query varlen-16k-U512..8192 (seed 5) h32 kv8 d128 causal", gqa, {})]
     for name, n, kw in specs:
-        w = synth.standard_workload(n, **kw)
+        w = n() if callable(n) else synth.standard_workload(n, **kw)
+        fwd_fn = fa_varlen.fa_varlen_fwd_gqa if w.kv_heads != w.heads else fa_varlen.fa_varlen_fwd
         t = w.tensors()
         mk = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)
         q, k, v = mk(t["q"]), mk(t["k"]), mk(t["v"])
@@ -376,8 +380,8 @@ def fwd_only_workloads(dev, stream, flush, peak, iters=10):
         out = torch.empty_like(q)
         lse = torch.empty((w.heads, w.total_q), dtype=torch.float32, device=dev)
         ws = fa_varlen.new_workspace(fa_varlen.fwd_workspace_size(w.batch, w.total_q, w.heads, w.head_dim), dev)
-        call = lambda: fa_varlen.fa_varlen_fwd(q, k, v, cq, ck, w.max_seqlen_q, w.max_seqlen_k, w.scale,
-                                               w.causal, out=out, softmax_lse=lse, workspace=ws, stream=stream)
+        call = lambda: fwd_fn(q, k, v, cq, ck, w.max_seqlen_q, w.max_seqlen_k, w.scale, w.causal, out=out,
+                              softmax_lse=lse, workspace=ws, stream=stream)
         for _ in range(3):
             call()
         evs = []

@@ -139,6 +139,34 @@ fa_status_t fa_varlen_bwd_gqa(const void* dout, const void* q, const void* k, co
                               void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
                               fa_cuda_stream_t stream);
 
+/* Forward over a key/value cache: the keys of each sequence are given by a
+ * per-sequence length instead of cumulative offsets, optionally after some
+ * left padding (page "Mecanismo cu_seqlens en FlashAttention", "Lógica de
+ * cálculo de longitud": the key array may be non-cumulative, and the cache
+ * length of a sequence is its key count minus its left padding).
+ *   k_cache, v_cache : bf16 [batch, cache_rows, num_heads_k, head_dim]; slot b
+ *                      holds sequence b's keys at rows leftpad_k[b] ..
+ *                      seqlens_k[b]-1, so it has lk = seqlens_k[b] - leftpad_k[b]
+ *                      keys (rows outside that range are never read).
+ *   seqlens_k        : int32 [batch], device memory.
+ *   leftpad_k        : int32 [batch], device memory, or NULL (no padding).
+ * Queries, out and softmax_lse are packed with cu_seqlens_q exactly as in
+ * fa_varlen_fwd; the causal rule uses lq and lk as defined here (key j of
+ * the valid range is visible from query i iff j <= i + lk - lq). Grouped
+ * heads as in fa_varlen_fwd_gqa. The workspace size is
+ * fa_varlen_fwd_workspace_size(batch, total_q, num_heads, head_dim).
+ * Errors: FA_ERR_INVALID_ARGUMENT for a null seqlens_k; on the device,
+ * FA_ERR_BAD_SEQLENS unless 0 <= leftpad_k[b] <= seqlens_k[b] <= cache_rows
+ * for every b (besides the checks of cu_seqlens_q); batch * cache_rows must
+ * stay below 2^31 - 256 rows (FA_ERR_UNSUPPORTED). There is no backward for
+ * this layout. */
+fa_status_t fa_varlen_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache,
+                                  const int32_t* cu_seqlens_q, const int32_t* seqlens_k, const int32_t* leftpad_k,
+                                  int batch, int total_q, int cache_rows, int max_seqlen_q, int num_heads,
+                                  int num_heads_k, int head_dim, float softmax_scale, int causal, void* out,
+                                  float* softmax_lse, void* workspace, size_t workspace_bytes,
+                                  fa_cuda_stream_t stream);
+
 /* Forward for callers that cannot allocate device memory. The pages have no
  * counterpart of this entry point; it exists for the library's users.
  *

@@ -126,6 +126,32 @@ class OracleLib:
         return dq, dk, dv
 
 
+def kvcache_to_packed(k_cache, v_cache, seqlens_k, leftpad_k=None):
+    """Key/value cache layout -> packed layout (page "Mecanismo cu_seqlens en
+    FlashAttention", "Lógica de cálculo de longitud": with non-cumulative key
+    lengths, sequence b has seqlens_k[b] - leftpad_k[b] keys). Slot b of the
+    [batch, rows, Hk, d] cache holds them at rows leftpad_k[b] ..
+    seqlens_k[b]-1. Returns (k, v, cu_k) packed back to back."""
+    seqlens_k = np.asarray(seqlens_k, dtype=np.int64)
+    batch, rows = k_cache.shape[:2]
+    leftpad_k = np.zeros(batch, dtype=np.int64) if leftpad_k is None else np.asarray(leftpad_k, dtype=np.int64)
+    if np.any(leftpad_k < 0) or np.any(seqlens_k < leftpad_k) or np.any(seqlens_k > rows):
+        raise ValueError("need 0 <= leftpad_k <= seqlens_k <= cache rows")
+    lk = seqlens_k - leftpad_k
+    cu_k = np.concatenate([[0], np.cumsum(lk)]).astype(np.int32)
+    k = np.concatenate([k_cache[b, leftpad_k[b]:seqlens_k[b]] for b in range(batch)], axis=0)
+    v = np.concatenate([v_cache[b, leftpad_k[b]:seqlens_k[b]] for b in range(batch)], axis=0)
+    return np.ascontiguousarray(k), np.ascontiguousarray(v), cu_k
+
+
+def fwd_kvcache(q, k_cache, v_cache, cu_q, seqlens_k, leftpad_k, scale: float, causal: bool, units=None,
+                row_step: int = 1):
+    """The forward over a key/value cache: the plain varlen forward on the
+    keys the cache holds for each sequence."""
+    k, v, cu_k = kvcache_to_packed(k_cache, v_cache, seqlens_k, leftpad_k)
+    return fwd(q, k, v, cu_q, cu_k, scale, causal, units, row_step)
+
+
 def _load() -> OracleLib:
     global _lib
     with _lock:

@@ -48,3 +48,38 @@ def test_seqlens_rejects_bad_offsets(orc):
         orc.seqlens([1, 4, 6])
     with pytest.raises(ValueError):
         orc.seqlens([0, 4, 3])
+
+
+def test_kvcache_layout_is_the_packed_definition():
+    """Key/value cache layout (page 1, "Lógica de cálculo de longitud":
+    non-cumulative key lengths with left padding): sequence b has
+    seqlens_k[b] - leftpad_k[b] keys at slot rows leftpad_k[b] ..
+    seqlens_k[b]-1. A cache built here by scattering packed keys into slots
+    (garbage everywhere else) must give exactly the packed forward."""
+    rng = np.random.default_rng(31)
+    H, Hk, d, rows = 4, 2, 6, 40
+    lk = np.array([12, 0, 25, 1])
+    pad = np.array([3, 7, 15, 0])
+    lq = [5, 3, 9, 1]
+    cu_q = np.concatenate([[0], np.cumsum(lq)]).astype(np.int32)
+    cu_k = np.concatenate([[0], np.cumsum(lk)]).astype(np.int32)
+    q = rng.standard_normal((cu_q[-1], H, d))
+    k = rng.standard_normal((cu_k[-1], Hk, d))
+    v = rng.standard_normal((cu_k[-1], Hk, d))
+    kc = rng.standard_normal((4, rows, Hk, d)) * 50.0
+    vc = rng.standard_normal((4, rows, Hk, d)) * 50.0
+    for b in range(4):
+        kc[b, pad[b]:pad[b] + lk[b]] = k[cu_k[b]:cu_k[b + 1]]
+        vc[b, pad[b]:pad[b] + lk[b]] = v[cu_k[b]:cu_k[b + 1]]
+    seqlens_k = pad + lk
+    kp, vp, ck = oracle.kvcache_to_packed(kc, vc, seqlens_k, pad)
+    assert list(np.diff(ck)) == list(seqlens_k - pad)
+    assert np.array_equal(kp, k) and np.array_equal(vp, v)
+    for causal in (False, True):
+        a = oracle.fwd_kvcache(q, kc, vc, cu_q, seqlens_k, pad, 0.4, causal)
+        b_ = oracle.fwd(q, k, v, cu_q, cu_k, 0.4, causal)
+        assert np.array_equal(a[0], b_[0]) and np.array_equal(a[1], b_[1])
+    with pytest.raises(ValueError):
+        oracle.kvcache_to_packed(kc, vc, np.array([5, 5, 5, 5]), np.array([6, 0, 0, 0]))
+    with pytest.raises(ValueError):
+        oracle.kvcache_to_packed(kc, vc, np.array([5, 5, rows + 1, 5]), None)

@@ -99,6 +99,63 @@ fa_status_t check_sizes(int batch, int total_q, int total_k, int max_sq, int max
   return FA_OK;
 }
 
+// The forward for either key layout. total_k: rows of the key/value tensors.
+fa_status_t run_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q, const fa::KeyRows& keys,
+                    int batch, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int num_heads,
+                    int num_heads_k, int head_dim, float softmax_scale, int causal, void* out, float* softmax_lse,
+                    void* workspace, size_t workspace_bytes, fa_cuda_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  fa_status_t st = check_sizes(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, num_heads, num_heads_k,
+                               head_dim, softmax_scale);
+  if (st != FA_OK) return st;
+  if (!cu_seqlens_q) return FA_ERR_INVALID_ARGUMENT;
+  if (total_q > 0 && (!q || !out || !softmax_lse || !aligned16(q) || !aligned16(out))) return FA_ERR_INVALID_ARGUMENT;
+  if (total_k > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return FA_ERR_INVALID_ARGUMENT;
+  const WsLayout L = fa::ws_layout(false, batch, total_q, total_k, num_heads, head_dim);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < L.total)
+    return FA_ERR_WORKSPACE;
+
+  t_events.next = 0;
+  fa::SchedArgs sa{cu_seqlens_q, keys, batch, total_q, total_k, max_seqlen_q, max_seqlen_k,
+                   causal ? 1 : 0, 0, workspace, L.seq_off, L.pairs, L.max_pairs};
+  if (timed_launch(stream, [&] { return fa::launch_sched_prep(sa, stream); }) != cudaSuccess) return FA_ERR_CUDA;
+  if (total_q == 0) return FA_OK;
+
+  const int HD = num_heads * head_dim;
+  const int HkD = num_heads_k * head_dim;
+  CUtensorMap tq, tk, tv;
+  // With no keys at all every row is empty and K/V are never read; the maps
+  // then point at q so that they are still well formed.
+  const void* kp = total_k > 0 ? k : q;
+  const void* vp = total_k > 0 ? v : q;
+  const int krows = total_k > 0 ? total_k : total_q;
+  const int kcols = total_k > 0 ? HkD : HD;
+  if (!encode_map(&tq, q, total_q, HD, fa::kFwdBM) || !encode_map(&tk, kp, krows, kcols, fa::kFwdBN) ||
+      !encode_map(&tv, vp, krows, kcols, fa::kFwdBN))
+    return FA_ERR_CUDA;
+
+  const int sms = sm_count();
+  if (sms <= 0) return FA_ERR_CUDA;
+  const long long items = static_cast<long long>(L.max_pairs) * num_heads;
+  fa::FwdArgs fa_args{};
+  fa_args.cu_q = cu_seqlens_q;
+  fa_args.keys = keys;
+  fa_args.out = out;
+  fa_args.lse = softmax_lse;
+  fa_args.workspace = workspace;
+  fa_args.pairs_offset = L.pairs;
+  fa_args.H = num_heads;
+  fa_args.D = head_dim;
+  fa_args.total_q = total_q;
+  fa_args.group = num_heads / num_heads_k;
+  fa_args.causal = causal ? 1 : 0;
+  fa_args.scale_log2 = softmax_scale * 1.4426950408889634f;
+  fa_args.grid = static_cast<int>(items < sms ? items : sms);
+  if (timed_launch(stream, [&] { return fa::launch_fwd(fa_args, tq, tk, tv, stream); }) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -140,57 +197,25 @@ fa_status_t fa_varlen_fwd_gqa(const void* q, const void* k, const void* v, const
                               const int32_t* cu_seqlens_k, int batch, int total_q, int total_k, int max_seqlen_q,
                               int max_seqlen_k, int num_heads, int num_heads_k, int head_dim, float softmax_scale,
                               int causal, void* out, float* softmax_lse, void* workspace, size_t workspace_bytes,
-                              fa_cuda_stream_t stream_) {
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  fa_status_t st = check_sizes(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, num_heads, num_heads_k,
-                               head_dim, softmax_scale);
-  if (st != FA_OK) return st;
-  if (!cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARGUMENT;
-  if (total_q > 0 && (!q || !out || !softmax_lse || !aligned16(q) || !aligned16(out))) return FA_ERR_INVALID_ARGUMENT;
-  if (total_k > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return FA_ERR_INVALID_ARGUMENT;
-  const WsLayout L = fa::ws_layout(false, batch, total_q, total_k, num_heads, head_dim);
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < L.total)
-    return FA_ERR_WORKSPACE;
+                              fa_cuda_stream_t stream) {
+  if (!cu_seqlens_k) return FA_ERR_INVALID_ARGUMENT;
+  return run_fwd(q, k, v, cu_seqlens_q, fa::KeyRows{cu_seqlens_k, nullptr, nullptr, 0}, batch, total_q, total_k,
+                 max_seqlen_q, max_seqlen_k, num_heads, num_heads_k, head_dim, softmax_scale, causal, out,
+                 softmax_lse, workspace, workspace_bytes, stream);
+}
 
-  t_events.next = 0;
-  fa::SchedArgs sa{cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q, max_seqlen_k,
-                   causal ? 1 : 0, 0, workspace, L.seq_off, L.pairs, L.max_pairs};
-  if (timed_launch(stream, [&] { return fa::launch_sched_prep(sa, stream); }) != cudaSuccess) return FA_ERR_CUDA;
-  if (total_q == 0) return FA_OK;
-
-  const int HD = num_heads * head_dim;
-  const int HkD = num_heads_k * head_dim;
-  CUtensorMap tq, tk, tv;
-  // With no keys at all every row is empty and K/V are never read; the maps
-  // then point at q so that they are still well formed.
-  const void* kp = total_k > 0 ? k : q;
-  const void* vp = total_k > 0 ? v : q;
-  const int krows = total_k > 0 ? total_k : total_q;
-  const int kcols = total_k > 0 ? HkD : HD;
-  if (!encode_map(&tq, q, total_q, HD, fa::kFwdBM) || !encode_map(&tk, kp, krows, kcols, fa::kFwdBN) ||
-      !encode_map(&tv, vp, krows, kcols, fa::kFwdBN))
-    return FA_ERR_CUDA;
-
-  const int sms = sm_count();
-  if (sms <= 0) return FA_ERR_CUDA;
-  const long long items = static_cast<long long>(L.max_pairs) * num_heads;
-  fa::FwdArgs fa_args{};
-  fa_args.cu_q = cu_seqlens_q;
-  fa_args.cu_k = cu_seqlens_k;
-  fa_args.out = out;
-  fa_args.lse = softmax_lse;
-  fa_args.workspace = workspace;
-  fa_args.pairs_offset = L.pairs;
-  fa_args.H = num_heads;
-  fa_args.D = head_dim;
-  fa_args.total_q = total_q;
-  fa_args.group = num_heads / num_heads_k;
-  fa_args.causal = causal ? 1 : 0;
-  fa_args.scale_log2 = softmax_scale * 1.4426950408889634f;
-  fa_args.grid = static_cast<int>(items < sms ? items : sms);
-  if (timed_launch(stream, [&] { return fa::launch_fwd(fa_args, tq, tk, tv, stream); }) != cudaSuccess)
-    return FA_ERR_CUDA;
-  return FA_OK;
+fa_status_t fa_varlen_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache,
+                                  const int32_t* cu_seqlens_q, const int32_t* seqlens_k, const int32_t* leftpad_k,
+                                  int batch, int total_q, int cache_rows, int max_seqlen_q, int num_heads,
+                                  int num_heads_k, int head_dim, float softmax_scale, int causal, void* out,
+                                  float* softmax_lse, void* workspace, size_t workspace_bytes,
+                                  fa_cuda_stream_t stream) {
+  if (!seqlens_k || batch < 1 || cache_rows < 0) return FA_ERR_INVALID_ARGUMENT;
+  const long long rows = static_cast<long long>(batch) * cache_rows;
+  if (rows > (1ll << 31) - 1 - 2 * fa::kFwdBN) return FA_ERR_UNSUPPORTED;
+  return run_fwd(q, k_cache, v_cache, cu_seqlens_q, fa::KeyRows{nullptr, seqlens_k, leftpad_k, cache_rows}, batch,
+                 total_q, static_cast<int>(rows), max_seqlen_q, cache_rows, num_heads, num_heads_k, head_dim,
+                 softmax_scale, causal, out, softmax_lse, workspace, workspace_bytes, stream);
 }
 
 fa_status_t fa_varlen_bwd(const void* dout, const void* q, const void* k, const void* v, const void* out,
@@ -224,8 +249,8 @@ fa_status_t fa_varlen_bwd_gqa(const void* dout, const void* q, const void* k, co
     return FA_ERR_WORKSPACE;
 
   t_events.next = 0;
-  fa::SchedArgs sa{cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q, max_seqlen_k,
-                   causal ? 1 : 0, 1, workspace, L.seq_off, L.pairs, L.max_pairs};
+  fa::SchedArgs sa{cu_seqlens_q, fa::KeyRows{cu_seqlens_k, nullptr, nullptr, 0}, batch, total_q, total_k,
+                   max_seqlen_q, max_seqlen_k, causal ? 1 : 0, 1, workspace, L.seq_off, L.pairs, L.max_pairs};
   if (timed_launch(stream, [&] { return fa::launch_sched_prep(sa, stream); }) != cudaSuccess) return FA_ERR_CUDA;
   if (total_q == 0 && total_k == 0) return FA_OK;
 
@@ -252,7 +277,7 @@ fa_status_t fa_varlen_bwd_gqa(const void* dout, const void* q, const void* k, co
   const long long items = static_cast<long long>(L.max_pairs) * num_heads_k;
   fa::BwdArgs b{};
   b.cu_q = cu_seqlens_q;
-  b.cu_k = cu_seqlens_k;
+  b.keys = fa::KeyRows{cu_seqlens_k, nullptr, nullptr, 0};
   b.dout = dout;
   b.out = out;
   b.lse = softmax_lse;

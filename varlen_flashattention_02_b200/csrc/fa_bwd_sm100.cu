@@ -101,7 +101,7 @@ __device__ __forceinline__ Item get_item(const BwdArgs& a, const int2* pairs, in
   it.h0 = it.hk * a.group;
   it.b = pr.x;
   it.j = pr.y;
-  it.s = seq_info(a.cu_q, a.cu_k, it.b);
+  it.s = seq_info(a.cu_q, a.keys, it.b);
   int e;
   bwd_q_tiles(it.j, it.s.lq, it.s.lk, a.causal != 0, &it.i0, &e);
   it.nt = e - it.i0;

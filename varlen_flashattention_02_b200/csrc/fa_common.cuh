@@ -73,18 +73,36 @@ __host__ __device__ inline WsLayout ws_layout(bool backward, int batch, int tota
 
 // ---------------------------------------------------------------- sequences
 // Page "Mecanismo cu_seqlens en FlashAttention", "Lógica de cálculo de
-// longitud": sequence b starts at packed row cu[b] and has cu[b+1] - cu[b]
-// rows (the cumulative branch; lengths-only and left-padded keys are not
-// supported).
+// longitud": query sequence b starts at packed row cu_q[b] and has
+// cu_q[b+1] - cu_q[b] rows. Its keys are found one of two ways:
+//  * packed (cumulative offsets): rows cu_k[b] .. cu_k[b+1]-1 of the key
+//    tensor;
+//  * key/value cache (per-sequence lengths, not cumulative, with left
+//    padding): sequence b owns a slot of cache_rows rows starting at row
+//    b*cache_rows, and its keys are slot rows leftpad_k[b] .. seqlens_k[b]-1,
+//    so it has seqlens_k[b] - leftpad_k[b] of them.
+struct KeyRows {
+  const int32_t* cu_k;       // packed layout: [batch + 1] cumulative offsets
+  const int32_t* seqlens_k;  // cache layout: [batch] key counts incl. padding (null: packed)
+  const int32_t* leftpad_k;  // cache layout: [batch] left padding, or null (none)
+  int cache_rows;            // cache layout: rows per sequence slot
+};
+
 struct SeqInfo {
   int q0, lq, k0, lk;
 };
-__device__ __forceinline__ SeqInfo seq_info(const int32_t* cu_q, const int32_t* cu_k, int b) {
+__device__ __forceinline__ SeqInfo seq_info(const int32_t* cu_q, const KeyRows& kr, int b) {
   SeqInfo s;
   s.q0 = __ldg(cu_q + b);
   s.lq = __ldg(cu_q + b + 1) - s.q0;
-  s.k0 = __ldg(cu_k + b);
-  s.lk = __ldg(cu_k + b + 1) - s.k0;
+  if (kr.seqlens_k) {
+    const int lp = kr.leftpad_k ? __ldg(kr.leftpad_k + b) : 0;
+    s.k0 = b * kr.cache_rows + lp;
+    s.lk = __ldg(kr.seqlens_k + b) - lp;
+  } else {
+    s.k0 = __ldg(kr.cu_k + b);
+    s.lk = __ldg(kr.cu_k + b + 1) - s.k0;
+  }
   return s;
 }
 

@@ -118,7 +118,7 @@ __device__ __forceinline__ Item get_item(const FwdArgs& a, const int2* pairs, in
   it.hk = it.h / a.group;
   it.b = pr.x;
   it.t = pr.y;
-  it.s = seq_info(a.cu_q, a.cu_k, it.b);
+  it.s = seq_info(a.cu_q, a.keys, it.b);
 #pragma unroll
   for (int w = 0; w < 2; ++w) {
     const int row0 = (it.t * kQTiles + w) * BM;

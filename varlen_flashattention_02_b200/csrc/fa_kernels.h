@@ -7,6 +7,8 @@
 
 #include <cstdint>
 
+#include "fa_common.cuh"
+
 namespace fa {
 
 // Work-list preparation (one CTA): validates the cumulative offsets, counts
@@ -14,7 +16,7 @@ namespace fa {
 // workspace. mode 0: forward query tiles; mode 1: backward key tiles.
 struct SchedArgs {
   const int32_t* cu_q;
-  const int32_t* cu_k;
+  KeyRows keys;
   int batch, total_q, total_k, max_seqlen_q, max_seqlen_k;
   int causal;
   int mode;
@@ -26,7 +28,7 @@ cudaError_t launch_sched_prep(const SchedArgs& a, cudaStream_t stream);
 
 struct FwdArgs {
   const int32_t* cu_q;
-  const int32_t* cu_k;
+  KeyRows keys;
   void* out;         // bf16 [total_q, H, D]
   float* lse;        // fp32 [H, total_q]
   void* workspace;   // header + pairs
@@ -44,7 +46,7 @@ cudaError_t launch_fwd(const FwdArgs& a, const CUtensorMap& tm_q, const CUtensor
 
 struct BwdArgs {
   const int32_t* cu_q;
-  const int32_t* cu_k;
+  KeyRows keys;      // packed layout only
   const void* dout;   // bf16 [total_q, H, D]
   const void* out;    // bf16 [total_q, H, D]
   const float* lse;   // fp32 [H, total_q]

@@ -2,7 +2,8 @@
 //
 // From the device-resident cumulative offsets, one CTA
 //   1. checks them (cu[0] = 0, non-decreasing, cu[batch] = total, every
-//      length <= max_seqlen) and records FA_ERR_BAD_SEQLENS otherwise;
+//      length <= max_seqlen; for a key/value cache 0 <= leftpad_k[b] <=
+//      seqlens_k[b] <= cache_rows) and records FA_ERR_BAD_SEQLENS otherwise;
 //   2. counts the tiles of every sequence (forward: query blocks of 256
 //      rows; backward: key tiles of 128 rows) and prefix-sums them;
 //   3. orders all (sequence, tile) pairs by their number of visible tiles on
@@ -79,18 +80,28 @@ __global__ void __launch_bounds__(kThreads) sched_prep_kernel(SchedArgs a) {
   const int tid = threadIdx.x;
   const bool causal = a.causal != 0;
 
+  const bool cache = a.keys.seqlens_k != nullptr;
   if (tid == 0) {
     s_err = 0;
     s_total = 0;
     hdr->work_counter = 0;
-    if (a.cu_q[0] != 0 || a.cu_k[0] != 0 || a.cu_q[a.batch] != a.total_q || a.cu_k[a.batch] != a.total_k)
-      s_err = 1;
+    if (a.cu_q[0] != 0 || a.cu_q[a.batch] != a.total_q) s_err = 1;
+    if (!cache && (a.keys.cu_k[0] != 0 || a.keys.cu_k[a.batch] != a.total_k)) s_err = 1;
   }
   for (int i = tid; i < kBins; i += kThreads) s_hist[i] = 0;
   __syncthreads();
   for (int b = tid; b < a.batch; b += kThreads) {
     const int lq = a.cu_q[b + 1] - a.cu_q[b];
-    const int lk = a.cu_k[b + 1] - a.cu_k[b];
+    int lk;
+    if (cache) {
+      // 0 <= leftpad <= seqlens_k <= cache_rows.
+      const int lp = a.keys.leftpad_k ? a.keys.leftpad_k[b] : 0;
+      const int sl = a.keys.seqlens_k[b];
+      if (lp < 0 || sl < lp || sl > a.keys.cache_rows) s_err = 1;
+      lk = sl - lp;
+    } else {
+      lk = a.keys.cu_k[b + 1] - a.keys.cu_k[b];
+    }
     if (lq < 0 || lk < 0 || lq > a.max_seqlen_q || lk > a.max_seqlen_k) s_err = 1;
   }
   __syncthreads();
@@ -108,7 +119,7 @@ __global__ void __launch_bounds__(kThreads) sched_prep_kernel(SchedArgs a) {
     const int b = base + tid;
     int n = 0;
     if (b < a.batch) {
-      const int len = a.mode == 0 ? a.cu_q[b + 1] - a.cu_q[b] : a.cu_k[b + 1] - a.cu_k[b];
+      const int len = a.mode == 0 ? a.cu_q[b + 1] - a.cu_q[b] : a.keys.cu_k[b + 1] - a.keys.cu_k[b];
       n = (len + tile - 1) / tile;
     }
     const int incl = block_inclusive_scan(n, s_warp);
@@ -131,7 +142,7 @@ __global__ void __launch_bounds__(kThreads) sched_prep_kernel(SchedArgs a) {
   // Histogram of costs.
   for (int p = tid; p < n_pairs; p += kThreads) {
     const int b = find_seq(seq_off, a.batch, p);
-    const SeqInfo s = seq_info(a.cu_q, a.cu_k, b);
+    const SeqInfo s = seq_info(a.cu_q, a.keys, b);
     const int c = min(pair_cost(s, p - seq_off[b], a.mode, causal), kBins - 1);
     atomicAdd(&s_hist[c], 1);
   }
@@ -160,7 +171,7 @@ __global__ void __launch_bounds__(kThreads) sched_prep_kernel(SchedArgs a) {
   // Scatter.
   for (int p = tid; p < n_pairs; p += kThreads) {
     const int b = find_seq(seq_off, a.batch, p);
-    const SeqInfo s = seq_info(a.cu_q, a.cu_k, b);
+    const SeqInfo s = seq_info(a.cu_q, a.keys, b);
     const int t = p - seq_off[b];
     const int c = min(pair_cost(s, t, a.mode, causal), kBins - 1);
     const int pos = atomicAdd(&s_hist[c], 1);

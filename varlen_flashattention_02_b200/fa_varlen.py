@@ -54,6 +54,8 @@ def _load():
     lib.fa_varlen_bwd_gqa.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, ctypes.c_float, I,
                                       P, P, P, P, S, P]
     lib.fa_varlen_bwd_gqa.restype = I
+    lib.fa_varlen_fwd_kvcache.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, ctypes.c_float, I, P, P, P, S, P]
+    lib.fa_varlen_fwd_kvcache.restype = I
     lib.fa_get_device_status.argtypes = [P, P]
     lib.fa_get_device_status.restype = I
     lib.fa_varlen_fwd_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, ctypes.c_float, I, P, P, P]
@@ -68,7 +70,8 @@ def _load():
 lib = _load()
 
 EXPORTED = ("fa_varlen_fwd_workspace_size", "fa_varlen_bwd_workspace_size", "fa_varlen_fwd",
-            "fa_varlen_bwd", "fa_varlen_fwd_gqa", "fa_varlen_bwd_gqa", "fa_varlen_fwd_noalloc",
+            "fa_varlen_bwd", "fa_varlen_fwd_gqa", "fa_varlen_bwd_gqa", "fa_varlen_fwd_kvcache",
+            "fa_varlen_fwd_noalloc",
             "fa_get_device_status", "fa_set_kernel_events", "fa_status_string")
 
 
@@ -227,6 +230,43 @@ def fa_varlen_bwd_gqa(dout, q, k, v, out, softmax_lse, cu_seqlens_q, cu_seqlens_
     if rc != FA_OK:
         raise FaError(rc, "fa_varlen_bwd_gqa")
     return dq, dk, dv
+
+
+def fa_varlen_fwd_kvcache(q, k_cache, v_cache, cu_seqlens_q, seqlens_k, leftpad_k, max_seqlen_q: int,
+                          softmax_scale: float, causal: bool, out=None, softmax_lse=None, workspace=None,
+                          stream=None):
+    """Forward over a key/value cache [batch, cache_rows, Hk, D]: sequence b's
+    keys are rows leftpad_k[b] .. seqlens_k[b]-1 of slot b (leftpad_k may be
+    None). Returns (out, softmax_lse) as fa_varlen_fwd does."""
+    _check_qkv("q", q)
+    Tq, H, D = q.shape
+    for name, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+        if t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor [batch, cache_rows, heads_k, head_dim]")
+    batch, rows, Hk, Dk = k_cache.shape
+    if tuple(v_cache.shape) != (batch, rows, Hk, Dk) or Dk != D:
+        raise ValueError("k_cache and v_cache must both be [batch, cache_rows, heads_k, head_dim]")
+    _kv_heads(H, k_cache[0])
+    _check_cu("cu_seqlens_q", cu_seqlens_q)
+    for name, t in (("seqlens_k", seqlens_k), ("leftpad_k", leftpad_k)):
+        if t is not None and (t.dtype != torch.int32 or t.dim() != 1 or t.numel() != batch or not t.is_cuda):
+            raise ValueError(f"{name} must be an int32 CUDA tensor [batch]")
+    if cu_seqlens_q.numel() - 1 != batch:
+        raise ValueError("cu_seqlens_q must have batch + 1 entries")
+    if out is None:
+        out = torch.empty_like(q)
+    if softmax_lse is None:
+        softmax_lse = torch.empty((H, Tq), dtype=torch.float32, device=q.device)
+    need = fwd_workspace_size(batch, Tq, H, D)
+    if workspace is None:
+        workspace = new_workspace(need, q.device)
+    rc = lib.fa_varlen_fwd_kvcache(_p(q), _p(k_cache), _p(v_cache), _p(cu_seqlens_q), _p(seqlens_k),
+                                   _p(leftpad_k), batch, Tq, rows, int(max_seqlen_q), H, Hk, D,
+                                   float(softmax_scale), int(bool(causal)), _p(out), _p(softmax_lse),
+                                   _p(workspace), workspace.numel(), _stream(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_varlen_fwd_kvcache")
+    return out, softmax_lse
 
 
 def fa_varlen_fwd_noalloc(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
