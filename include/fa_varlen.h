@@ -167,6 +167,31 @@ fa_status_t fa_varlen_fwd_kvcache(const void* q, const void* k_cache, const void
                                   float* softmax_lse, void* workspace, size_t workspace_bytes,
                                   fa_cuda_stream_t stream);
 
+/* Forward over a paged key/value cache (the pages' "caché KV paginada", on
+ * the cu_seqlens page, section "Integración con máscaras causales y caché
+ * paginada"): keys and values sit in a pool of fixed-size pages and each
+ * sequence lists its pages in a block table.
+ *   k_pages, v_pages : bf16 [num_pages, page_size, num_heads_k, head_dim]
+ *   seqlens_k        : int32 [batch], device: sequence b has seqlens_k[b]
+ *                      keys, key position p in page block_table[b][p /
+ *                      page_size] at row p % page_size.
+ *   block_table      : int32 [batch, max_pages_per_seq], device, row-major;
+ *                      entries past a sequence's last page are not read.
+ * page_size must be a multiple of 128 (FA_ERR_UNSUPPORTED otherwise: a key
+ * tile of 128 rows is then always inside one page). max_seqlen_k bounds
+ * seqlens_k. Queries, outputs, causal rule and grouped heads as in
+ * fa_varlen_fwd_gqa; workspace as fa_varlen_fwd_workspace_size(batch,
+ * total_q, num_heads, head_dim). On the device, FA_ERR_BAD_SEQLENS unless
+ * 0 <= seqlens_k[b] <= min(max_seqlen_k, max_pages_per_seq * page_size)
+ * and every page a sequence uses is in [0, num_pages). There is no backward
+ * for this layout. */
+fa_status_t fa_varlen_fwd_paged(const void* q, const void* k_pages, const void* v_pages,
+                                const int32_t* cu_seqlens_q, const int32_t* seqlens_k, const int32_t* block_table,
+                                int batch, int total_q, int num_pages, int page_size, int max_pages_per_seq,
+                                int max_seqlen_q, int max_seqlen_k, int num_heads, int num_heads_k, int head_dim,
+                                float softmax_scale, int causal, void* out, float* softmax_lse, void* workspace,
+                                size_t workspace_bytes, fa_cuda_stream_t stream);
+
 /* Forward for callers that cannot allocate device memory. The pages have no
  * counterpart of this entry point; it exists for the library's users.
  *

@@ -144,6 +144,36 @@ def kvcache_to_packed(k_cache, v_cache, seqlens_k, leftpad_k=None):
     return np.ascontiguousarray(k), np.ascontiguousarray(v), cu_k
 
 
+def paged_to_packed(k_pages, v_pages, seqlens_k, block_table):
+    """Paged key/value cache -> packed layout: sequence b has seqlens_k[b]
+    keys; key position p lives in page block_table[b][p // page_size] at row
+    p % page_size of the [num_pages, page_size, Hk, d] pools. Returns
+    (k, v, cu_k) packed back to back."""
+    seqlens_k = np.asarray(seqlens_k, dtype=np.int64)
+    block_table = np.asarray(block_table, dtype=np.int64)
+    num_pages, page_size = k_pages.shape[:2]
+    ks, vs = [], []
+    for b, lk in enumerate(seqlens_k):
+        pos = np.arange(lk)
+        if lk > block_table.shape[1] * page_size:
+            raise ValueError("sequence longer than its block table")
+        pages = block_table[b, pos // page_size]
+        if np.any(pages < 0) or np.any(pages >= num_pages):
+            raise ValueError("page index outside the pool")
+        ks.append(k_pages[pages, pos % page_size])
+        vs.append(v_pages[pages, pos % page_size])
+    cu_k = np.concatenate([[0], np.cumsum(seqlens_k)]).astype(np.int32)
+    return np.ascontiguousarray(np.concatenate(ks)), np.ascontiguousarray(np.concatenate(vs)), cu_k
+
+
+def fwd_paged(q, k_pages, v_pages, cu_q, seqlens_k, block_table, scale: float, causal: bool, units=None,
+              row_step: int = 1):
+    """The forward over a paged key/value cache: the plain varlen forward on
+    each sequence's keys gathered from its pages."""
+    k, v, cu_k = paged_to_packed(k_pages, v_pages, seqlens_k, block_table)
+    return fwd(q, k, v, cu_q, cu_k, scale, causal, units, row_step)
+
+
 def fwd_kvcache(q, k_cache, v_cache, cu_q, seqlens_k, leftpad_k, scale: float, causal: bool, units=None,
                 row_step: int = 1):
     """The forward over a key/value cache: the plain varlen forward on the

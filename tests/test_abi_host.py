@@ -126,3 +126,14 @@ def test_gqa_head_counts(lib, Hk, code):
     1); valid counts get as far as the too-small workspace (3)."""
     assert _fwd_gqa(lib, Hk) == code
     assert _bwd_gqa(lib, Hk) == code
+
+
+def test_paged_rejects_page_size_not_multiple_of_tile(lib):
+    """Pages must hold whole 128-key tiles (FA_ERR_UNSUPPORTED), checked before
+    anything touches the GPU."""
+    rc = lib.fa_varlen_fwd_paged(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 64, 8, 64, 4, 32, 256, 4, 4, 128,
+                                 0.1, 1, FAKE, FAKE, FAKE, 1 << 20, None)
+    assert rc == 2
+    rc = lib.fa_varlen_fwd_paged(FAKE, FAKE, FAKE, FAKE, None, FAKE, 2, 64, 8, 128, 4, 32, 256, 4, 4, 128,
+                                 0.1, 1, FAKE, FAKE, FAKE, 1 << 20, None)
+    assert rc == 1

@@ -83,3 +83,43 @@ def test_kvcache_layout_is_the_packed_definition():
         oracle.kvcache_to_packed(kc, vc, np.array([5, 5, 5, 5]), np.array([6, 0, 0, 0]))
     with pytest.raises(ValueError):
         oracle.kvcache_to_packed(kc, vc, np.array([5, 5, rows + 1, 5]), None)
+
+
+def test_paged_layout_is_the_packed_definition():
+    """Paged key/value cache (the cu_seqlens page, "Integración con máscaras
+    causales y caché paginada"): key position p of sequence b lives in page
+    block_table[b][p // page_size], row p % page_size. Packed keys scattered
+    into a shuffled page pool (garbage in unused pages and rows) must give
+    exactly the packed forward."""
+    rng = np.random.default_rng(32)
+    H, Hk, d, ps = 2, 1, 5, 4
+    lk = np.array([9, 0, 4, 13])
+    lq = [3, 2, 4, 6]
+    cu_q = np.concatenate([[0], np.cumsum(lq)]).astype(np.int32)
+    cu_k = np.concatenate([[0], np.cumsum(lk)]).astype(np.int32)
+    q = rng.standard_normal((cu_q[-1], H, d))
+    k = rng.standard_normal((cu_k[-1], Hk, d))
+    v = rng.standard_normal((cu_k[-1], Hk, d))
+    n_pages, max_pages = 12, 5
+    kp = rng.standard_normal((n_pages, ps, Hk, d)) * 40.0
+    vp = rng.standard_normal((n_pages, ps, Hk, d)) * 40.0
+    perm = rng.permutation(n_pages)
+    bt = np.full((4, max_pages), -7, dtype=np.int32)  # unused entries are never read
+    nxt = 0
+    for b in range(4):
+        for i in range(-(-lk[b] // ps)):
+            bt[b, i] = perm[nxt]
+            nxt += 1
+        for pos in range(lk[b]):
+            kp[bt[b, pos // ps], pos % ps] = k[cu_k[b] + pos]
+            vp[bt[b, pos // ps], pos % ps] = v[cu_k[b] + pos]
+    k2, v2, ck = oracle.paged_to_packed(kp, vp, lk, bt)
+    assert np.array_equal(ck, cu_k) and np.array_equal(k2, k) and np.array_equal(v2, v)
+    for causal in (False, True):
+        a = oracle.fwd_paged(q, kp, vp, cu_q, lk, bt, 0.45, causal)
+        b_ = oracle.fwd(q, k, v, cu_q, cu_k, 0.45, causal)
+        assert np.array_equal(a[0], b_[0]) and np.array_equal(a[1], b_[1])
+    bad = bt.copy()
+    bad[0, 1] = n_pages
+    with pytest.raises(ValueError):
+        oracle.paged_to_packed(kp, vp, lk, bad)

@@ -199,9 +199,28 @@ fa_status_t fa_varlen_fwd_gqa(const void* q, const void* k, const void* v, const
                               int causal, void* out, float* softmax_lse, void* workspace, size_t workspace_bytes,
                               fa_cuda_stream_t stream) {
   if (!cu_seqlens_k) return FA_ERR_INVALID_ARGUMENT;
-  return run_fwd(q, k, v, cu_seqlens_q, fa::KeyRows{cu_seqlens_k, nullptr, nullptr, 0}, batch, total_q, total_k,
+  return run_fwd(q, k, v, cu_seqlens_q, fa::KeyRows{cu_seqlens_k, nullptr, nullptr, 0, nullptr, 0, 0}, batch, total_q, total_k,
                  max_seqlen_q, max_seqlen_k, num_heads, num_heads_k, head_dim, softmax_scale, causal, out,
                  softmax_lse, workspace, workspace_bytes, stream);
+}
+
+fa_status_t fa_varlen_fwd_paged(const void* q, const void* k_pages, const void* v_pages,
+                                const int32_t* cu_seqlens_q, const int32_t* seqlens_k, const int32_t* block_table,
+                                int batch, int total_q, int num_pages, int page_size, int max_pages_per_seq,
+                                int max_seqlen_q, int max_seqlen_k, int num_heads, int num_heads_k, int head_dim,
+                                float softmax_scale, int causal, void* out, float* softmax_lse, void* workspace,
+                                size_t workspace_bytes, fa_cuda_stream_t stream) {
+  if (!seqlens_k || !block_table || batch < 1 || num_pages < 1 || max_pages_per_seq < 1 || page_size < 1)
+    return FA_ERR_INVALID_ARGUMENT;
+  if (page_size % fa::kFwdBN != 0) return FA_ERR_UNSUPPORTED;
+  const long long rows = static_cast<long long>(num_pages) * page_size;
+  if (rows > (1ll << 31) - 1 - 2 * fa::kFwdBN ||
+      static_cast<long long>(max_pages_per_seq) * page_size > (1ll << 31) - 1)
+    return FA_ERR_UNSUPPORTED;
+  return run_fwd(q, k_pages, v_pages, cu_seqlens_q,
+                 fa::KeyRows{nullptr, seqlens_k, nullptr, 0, block_table, max_pages_per_seq, page_size}, batch,
+                 total_q, static_cast<int>(rows), max_seqlen_q, max_seqlen_k, num_heads, num_heads_k, head_dim,
+                 softmax_scale, causal, out, softmax_lse, workspace, workspace_bytes, stream);
 }
 
 fa_status_t fa_varlen_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache,
@@ -213,7 +232,7 @@ fa_status_t fa_varlen_fwd_kvcache(const void* q, const void* k_cache, const void
   if (!seqlens_k || batch < 1 || cache_rows < 0) return FA_ERR_INVALID_ARGUMENT;
   const long long rows = static_cast<long long>(batch) * cache_rows;
   if (rows > (1ll << 31) - 1 - 2 * fa::kFwdBN) return FA_ERR_UNSUPPORTED;
-  return run_fwd(q, k_cache, v_cache, cu_seqlens_q, fa::KeyRows{nullptr, seqlens_k, leftpad_k, cache_rows}, batch,
+  return run_fwd(q, k_cache, v_cache, cu_seqlens_q, fa::KeyRows{nullptr, seqlens_k, leftpad_k, cache_rows, nullptr, 0, 0}, batch,
                  total_q, static_cast<int>(rows), max_seqlen_q, cache_rows, num_heads, num_heads_k, head_dim,
                  softmax_scale, causal, out, softmax_lse, workspace, workspace_bytes, stream);
 }
@@ -249,7 +268,7 @@ fa_status_t fa_varlen_bwd_gqa(const void* dout, const void* q, const void* k, co
     return FA_ERR_WORKSPACE;
 
   t_events.next = 0;
-  fa::SchedArgs sa{cu_seqlens_q, fa::KeyRows{cu_seqlens_k, nullptr, nullptr, 0}, batch, total_q, total_k,
+  fa::SchedArgs sa{cu_seqlens_q, fa::KeyRows{cu_seqlens_k, nullptr, nullptr, 0, nullptr, 0, 0}, batch, total_q, total_k,
                    max_seqlen_q, max_seqlen_k, causal ? 1 : 0, 1, workspace, L.seq_off, L.pairs, L.max_pairs};
   if (timed_launch(stream, [&] { return fa::launch_sched_prep(sa, stream); }) != cudaSuccess) return FA_ERR_CUDA;
   if (total_q == 0 && total_k == 0) return FA_OK;
@@ -277,7 +296,7 @@ fa_status_t fa_varlen_bwd_gqa(const void* dout, const void* q, const void* k, co
   const long long items = static_cast<long long>(L.max_pairs) * num_heads_k;
   fa::BwdArgs b{};
   b.cu_q = cu_seqlens_q;
-  b.keys = fa::KeyRows{cu_seqlens_k, nullptr, nullptr, 0};
+  b.keys = fa::KeyRows{cu_seqlens_k, nullptr, nullptr, 0, nullptr, 0, 0};
   b.dout = dout;
   b.out = out;
   b.lse = softmax_lse;

@@ -80,12 +80,18 @@ __host__ __device__ inline WsLayout ws_layout(bool backward, int batch, int tota
 //  * key/value cache (per-sequence lengths, not cumulative, with left
 //    padding): sequence b owns a slot of cache_rows rows starting at row
 //    b*cache_rows, and its keys are slot rows leftpad_k[b] .. seqlens_k[b]-1,
-//    so it has seqlens_k[b] - leftpad_k[b] of them.
+//    so it has seqlens_k[b] - leftpad_k[b] of them;
+//  * paged key/value cache (the pages' "caché KV paginada"): seqlens_k[b]
+//    keys whose position p lives in page block_table[b][p / page_size] at
+//    row p % page_size; the pool is pages of page_size rows, back to back.
 struct KeyRows {
-  const int32_t* cu_k;       // packed layout: [batch + 1] cumulative offsets
-  const int32_t* seqlens_k;  // cache layout: [batch] key counts incl. padding (null: packed)
-  const int32_t* leftpad_k;  // cache layout: [batch] left padding, or null (none)
-  int cache_rows;            // cache layout: rows per sequence slot
+  const int32_t* cu_k;         // packed layout: [batch + 1] cumulative offsets
+  const int32_t* seqlens_k;    // cache layouts: [batch] key counts (incl. padding) (null: packed)
+  const int32_t* leftpad_k;    // cache layout: [batch] left padding, or null (none)
+  int cache_rows;              // cache layout: rows per sequence slot
+  const int32_t* block_table;  // paged layout: [batch, max_pages] page indices (null: not paged)
+  int max_pages;               // paged layout: block-table entries per sequence
+  int page_size;               // paged layout: rows per page (a multiple of kFwdBN)
 };
 
 struct SeqInfo {
@@ -95,7 +101,10 @@ __device__ __forceinline__ SeqInfo seq_info(const int32_t* cu_q, const KeyRows& 
   SeqInfo s;
   s.q0 = __ldg(cu_q + b);
   s.lq = __ldg(cu_q + b + 1) - s.q0;
-  if (kr.seqlens_k) {
+  if (kr.block_table) {
+    s.k0 = 0;  // rows come from the block table (key_tile_row)
+    s.lk = __ldg(kr.seqlens_k + b);
+  } else if (kr.seqlens_k) {
     const int lp = kr.leftpad_k ? __ldg(kr.leftpad_k + b) : 0;
     s.k0 = b * kr.cache_rows + lp;
     s.lk = __ldg(kr.seqlens_k + b) - lp;
@@ -104,6 +113,18 @@ __device__ __forceinline__ SeqInfo seq_info(const int32_t* cu_q, const KeyRows& 
     s.lk = __ldg(kr.cu_k + b + 1) - s.k0;
   }
   return s;
+}
+
+// Row, in the key/value tensor, of the first key of key tile j of sequence
+// b. A tile never straddles two pages: the page size is a multiple of the
+// tile.
+__device__ __forceinline__ int key_tile_row(const KeyRows& kr, int b, const SeqInfo& s, int j) {
+  if (kr.block_table) {
+    const int pos = j * kFwdBN;
+    const int page = __ldg(kr.block_table + static_cast<size_t>(b) * kr.max_pages + pos / kr.page_size);
+    return page * kr.page_size + pos % kr.page_size;
+  }
+  return s.k0 + j * kFwdBN;
 }
 
 // Number of key tiles (kFwdBN keys) visible from the query rows below

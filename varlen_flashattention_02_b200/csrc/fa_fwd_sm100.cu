@@ -158,11 +158,12 @@ __device__ __forceinline__ void qk_producer(const CUtensorMap* tm_q, const CUten
     for (int j = 0; j < nkb; ++j, ++kc) {
       const int st = kc % NK;
       const uint32_t use = kc / NK;
+      const int krow = key_tile_row(a.keys, it.b, it.s, j);  // (a block-table read when paged)
       if (use > 0 && !wait_bar(&bars.k_empty[st], (use - 1) & 1, ab)) goto done;
       mbar_arrive_expect_tx(&bars.k_full[st], L::kTileBytes);
       for (int c = 0; c < L::kChunks; ++c)
         tma_load_2d(tm_k, &bars.k_full[st], smem + L::kK + st * L::kTileBytes + c * kChunkBytes,
-                    it.hk * D + c * 64, it.s.k0 + j * BN);
+                    it.hk * D + c * 64, krow);
     }
   }
 done:
@@ -189,11 +190,12 @@ __device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, const FwdArg
     for (int j = 0; j < nkb; ++j, ++vc) {
       const int st = vc % NV;
       const uint32_t use = vc / NV;
+      const int vrow = key_tile_row(a.keys, it.b, it.s, j);
       if (use > 0 && !wait_bar(&bars.v_empty[st], (use - 1) & 1, ab)) goto done;
       mbar_arrive_expect_tx(&bars.v_full[st], L::kTileBytes);
       for (int c = 0; c < L::kChunks; ++c)
         tma_load_2d(tm_v, &bars.v_full[st], smem + L::kV + st * L::kTileBytes + c * kChunkBytes,
-                    it.hk * D + c * 64, it.s.k0 + j * BN);
+                    it.hk * D + c * 64, vrow);
     }
   }
 done:

@@ -3,7 +3,8 @@
 // From the device-resident cumulative offsets, one CTA
 //   1. checks them (cu[0] = 0, non-decreasing, cu[batch] = total, every
 //      length <= max_seqlen; for a key/value cache 0 <= leftpad_k[b] <=
-//      seqlens_k[b] <= cache_rows) and records FA_ERR_BAD_SEQLENS otherwise;
+//      seqlens_k[b] <= cache_rows; for a paged cache every page a sequence
+//      uses inside the pool) and records FA_ERR_BAD_SEQLENS otherwise;
 //   2. counts the tiles of every sequence (forward: query blocks of 256
 //      rows; backward: key tiles of 128 rows) and prefix-sums them;
 //   3. orders all (sequence, tile) pairs by their number of visible tiles on
@@ -93,7 +94,21 @@ __global__ void __launch_bounds__(kThreads) sched_prep_kernel(SchedArgs a) {
   for (int b = tid; b < a.batch; b += kThreads) {
     const int lq = a.cu_q[b + 1] - a.cu_q[b];
     int lk;
-    if (cache) {
+    if (a.keys.block_table) {
+      // 0 <= seqlens_k <= max_pages * page_size, and every page it uses
+      // inside the pool.
+      lk = a.keys.seqlens_k[b];
+      if (lk < 0 || lk > a.keys.max_pages * a.keys.page_size) {
+        s_err = 1;
+      } else {
+        const int n_pages = (lk + a.keys.page_size - 1) / a.keys.page_size;
+        const int pool_pages = a.total_k / a.keys.page_size;
+        for (int i = 0; i < n_pages; ++i) {
+          const int pg = a.keys.block_table[static_cast<size_t>(b) * a.keys.max_pages + i];
+          if (pg < 0 || pg >= pool_pages) s_err = 1;
+        }
+      }
+    } else if (cache) {
       // 0 <= leftpad <= seqlens_k <= cache_rows.
       const int lp = a.keys.leftpad_k ? a.keys.leftpad_k[b] : 0;
       const int sl = a.keys.seqlens_k[b];

@@ -56,6 +56,9 @@ def _load():
     lib.fa_varlen_bwd_gqa.restype = I
     lib.fa_varlen_fwd_kvcache.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, ctypes.c_float, I, P, P, P, S, P]
     lib.fa_varlen_fwd_kvcache.restype = I
+    lib.fa_varlen_fwd_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, ctypes.c_float, I, P, P,
+                                        P, S, P]
+    lib.fa_varlen_fwd_paged.restype = I
     lib.fa_get_device_status.argtypes = [P, P]
     lib.fa_get_device_status.restype = I
     lib.fa_varlen_fwd_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, ctypes.c_float, I, P, P, P]
@@ -71,7 +74,7 @@ lib = _load()
 
 EXPORTED = ("fa_varlen_fwd_workspace_size", "fa_varlen_bwd_workspace_size", "fa_varlen_fwd",
             "fa_varlen_bwd", "fa_varlen_fwd_gqa", "fa_varlen_bwd_gqa", "fa_varlen_fwd_kvcache",
-            "fa_varlen_fwd_noalloc",
+            "fa_varlen_fwd_paged", "fa_varlen_fwd_noalloc",
             "fa_get_device_status", "fa_set_kernel_events", "fa_status_string")
 
 
@@ -266,6 +269,45 @@ def fa_varlen_fwd_kvcache(q, k_cache, v_cache, cu_seqlens_q, seqlens_k, leftpad_
                                    _p(workspace), workspace.numel(), _stream(stream))
     if rc != FA_OK:
         raise FaError(rc, "fa_varlen_fwd_kvcache")
+    return out, softmax_lse
+
+
+def fa_varlen_fwd_paged(q, k_pages, v_pages, cu_seqlens_q, seqlens_k, block_table, max_seqlen_q: int,
+                        max_seqlen_k: int, softmax_scale: float, causal: bool, out=None, softmax_lse=None,
+                        workspace=None, stream=None):
+    """Forward over a paged key/value cache: pools [num_pages, page_size, Hk,
+    D] (page_size a multiple of 128), block_table int32 [batch, max_pages],
+    seqlens_k int32 [batch]. Returns (out, softmax_lse) as fa_varlen_fwd."""
+    _check_qkv("q", q)
+    Tq, H, D = q.shape
+    for name, t in (("k_pages", k_pages), ("v_pages", v_pages)):
+        if t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor [num_pages, page_size, heads_k, head_dim]")
+    num_pages, page_size, Hk, Dk = k_pages.shape
+    if tuple(v_pages.shape) != tuple(k_pages.shape) or Dk != D:
+        raise ValueError("k_pages and v_pages must both be [num_pages, page_size, heads_k, head_dim]")
+    _kv_heads(H, k_pages[0])
+    _check_cu("cu_seqlens_q", cu_seqlens_q)
+    batch = cu_seqlens_q.numel() - 1
+    if seqlens_k.dtype != torch.int32 or seqlens_k.numel() != batch or not seqlens_k.is_cuda:
+        raise ValueError("seqlens_k must be an int32 CUDA tensor [batch]")
+    if (block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != batch
+            or not block_table.is_contiguous() or not block_table.is_cuda):
+        raise ValueError("block_table must be a contiguous int32 CUDA tensor [batch, max_pages]")
+    if out is None:
+        out = torch.empty_like(q)
+    if softmax_lse is None:
+        softmax_lse = torch.empty((H, Tq), dtype=torch.float32, device=q.device)
+    need = fwd_workspace_size(batch, Tq, H, D)
+    if workspace is None:
+        workspace = new_workspace(need, q.device)
+    rc = lib.fa_varlen_fwd_paged(_p(q), _p(k_pages), _p(v_pages), _p(cu_seqlens_q), _p(seqlens_k),
+                                 _p(block_table), batch, Tq, num_pages, page_size, block_table.shape[1],
+                                 int(max_seqlen_q), int(max_seqlen_k), H, Hk, D, float(softmax_scale),
+                                 int(bool(causal)), _p(out), _p(softmax_lse), _p(workspace), workspace.numel(),
+                                 _stream(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_varlen_fwd_paged")
     return out, softmax_lse
 
 
