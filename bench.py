@@ -363,13 +363,16 @@ def fwd_only_workloads(dev, stream, flush, peak, iters=10):
     res = {}
     gqa = lambda: synth.make_workload("gqa", synth.lengths_uniform(5, synth.TOTAL_TOKENS, 512, 8192), heads=32,
                                       head_dim=128, causal=True, seed=5, heads_k=8)
+    d256 = lambda: synth.make_workload("d256", synth.lengths_uniform(5, synth.TOTAL_TOKENS, 512, 8192), heads=16,
+                                       head_dim=256, causal=True, seed=5)
     specs = [("varlen-2seq-h12-d64 (cu_q=[0,200,1024], cu_k=[0,300,1024])", 1, {}),
              ("fixed-8x2048-h16-d128 non-causal", 2, {"causal": False}),
              ("fixed-8x2048-h16-d128 causal", 2, {"causal": True}),
              ("packed-16k-U128..4096-h32-d128 causal", 3, {}),
              ("long-1x16384-h16-d64 causal", 4, {"head_dim": 64}),
              ("long-1x16384-h16-d128 causal", 4, {"head_dim": 128}),
-             ("grouped-query varlen-16k-U512..8192 (seed 5) h32 kv8 d128 causal", gqa, {})]
+             ("grouped-query varlen-16k-U512..8192 (seed 5) h32 kv8 d128 causal", gqa, {}),
+             ("varlen-16k-U512..8192 (seed 5) h16 d256 causal", d256, {})]
     for name, n, kw in specs:
         w = n() if callable(n) else synth.standard_workload(n, **kw)
         fwd_fn = fa_varlen.fa_varlen_fwd_gqa if w.kv_heads != w.heads else fa_varlen.fa_varlen_fwd

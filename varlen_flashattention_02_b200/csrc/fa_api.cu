@@ -87,7 +87,7 @@ fa_status_t check_sizes(int batch, int total_q, int total_k, int max_sq, int max
   if (batch < 1 || total_q < 0 || total_k < 0 || max_sq < 0 || max_sk < 0 || H < 1) return FA_ERR_INVALID_ARGUMENT;
   if (Hk < 1 || Hk > H || H % Hk != 0) return FA_ERR_INVALID_ARGUMENT;
   if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARGUMENT;
-  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128 && D != 256) return FA_ERR_UNSUPPORTED;  // 256: forward only
   // Row indices and TMA coordinates are int32; element offsets are 64-bit.
   const long long hd = static_cast<long long>(H) * D;
   if (hd > (1ll << 31) - 1 || static_cast<long long>(total_q) + 2 * fa::kFwdBM > (1ll << 31) - 1 ||
@@ -117,7 +117,7 @@ fa_status_t run_fwd(const void* q, const void* k, const void* v, const int32_t* 
 
   t_events.next = 0;
   fa::SchedArgs sa{cu_seqlens_q, keys, batch, total_q, total_k, max_seqlen_q, max_seqlen_k,
-                   causal ? 1 : 0, 0, workspace, L.seq_off, L.pairs, L.max_pairs};
+                   causal ? 1 : 0, 0, fa::fwd_item_rows(head_dim), workspace, L.seq_off, L.pairs, L.max_pairs};
   if (timed_launch(stream, [&] { return fa::launch_sched_prep(sa, stream); }) != cudaSuccess) return FA_ERR_CUDA;
   if (total_q == 0) return FA_OK;
 
@@ -130,8 +130,9 @@ fa_status_t run_fwd(const void* q, const void* k, const void* v, const int32_t* 
   const void* vp = total_k > 0 ? v : q;
   const int krows = total_k > 0 ? total_k : total_q;
   const int kcols = total_k > 0 ? HkD : HD;
-  if (!encode_map(&tq, q, total_q, HD, fa::kFwdBM) || !encode_map(&tk, kp, krows, kcols, fa::kFwdBN) ||
-      !encode_map(&tv, vp, krows, kcols, fa::kFwdBN))
+  const int kbox = head_dim == 256 ? 64 : fa::kFwdBN;  // rows per K/V tile
+  if (!encode_map(&tq, q, total_q, HD, fa::kFwdBM) || !encode_map(&tk, kp, krows, kcols, kbox) ||
+      !encode_map(&tv, vp, krows, kcols, kbox))
     return FA_ERR_CUDA;
 
   const int sms = sm_count();
@@ -151,8 +152,8 @@ fa_status_t run_fwd(const void* q, const void* k, const void* v, const int32_t* 
   fa_args.causal = causal ? 1 : 0;
   fa_args.scale_log2 = softmax_scale * 1.4426950408889634f;
   fa_args.grid = static_cast<int>(items < sms ? items : sms);
-  if (timed_launch(stream, [&] { return fa::launch_fwd(fa_args, tq, tk, tv, stream); }) != cudaSuccess)
-    return FA_ERR_CUDA;
+  auto launch = head_dim == 256 ? fa::launch_fwd_d256 : fa::launch_fwd;
+  if (timed_launch(stream, [&] { return launch(fa_args, tq, tk, tv, stream); }) != cudaSuccess) return FA_ERR_CUDA;
   return FA_OK;
 }
 
@@ -257,6 +258,7 @@ fa_status_t fa_varlen_bwd_gqa(const void* dout, const void* q, const void* k, co
   fa_status_t st = check_sizes(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, num_heads, num_heads_k,
                                head_dim, softmax_scale);
   if (st != FA_OK) return st;
+  if (head_dim == 256) return FA_ERR_UNSUPPORTED;  // the backward supports head_dim 64 and 128
   if (!cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARGUMENT;
   if (total_q > 0 && (!q || !dout || !out || !softmax_lse || !dq || !aligned16(q) || !aligned16(dout) ||
                       !aligned16(out) || !aligned16(dq)))
@@ -269,7 +271,7 @@ fa_status_t fa_varlen_bwd_gqa(const void* dout, const void* q, const void* k, co
 
   t_events.next = 0;
   fa::SchedArgs sa{cu_seqlens_q, fa::KeyRows{cu_seqlens_k, nullptr, nullptr, 0, nullptr, 0, 0}, batch, total_q, total_k,
-                   max_seqlen_q, max_seqlen_k, causal ? 1 : 0, 1, workspace, L.seq_off, L.pairs, L.max_pairs};
+                   max_seqlen_q, max_seqlen_k, causal ? 1 : 0, 1, 0, workspace, L.seq_off, L.pairs, L.max_pairs};
   if (timed_launch(stream, [&] { return fa::launch_sched_prep(sa, stream); }) != cudaSuccess) return FA_ERR_CUDA;
   if (total_q == 0 && total_k == 0) return FA_OK;
 

@@ -18,6 +18,9 @@ namespace fa {
 constexpr int kFwdBM = 128;
 constexpr int kFwdBN = 128;
 constexpr int kFwdItemRows = 256;
+// Query rows per forward work item: head_dim 256 leaves TMEM room for one
+// 128-row query tile per CTA only.
+__host__ __device__ inline int fwd_item_rows(int D) { return D > 128 ? kFwdBM : kFwdItemRows; }
 // Backward tiles: a work item is 128 key rows of one (sequence, head);
 // queries stream through in tiles of 64.
 constexpr int kBwdBN = 128;
@@ -57,7 +60,7 @@ __host__ __device__ inline WsLayout ws_layout(bool backward, int batch, int tota
   size_t off = sizeof(WsHeader);
   L.seq_off = off;
   off = align_up(off + sizeof(int32_t) * (static_cast<size_t>(batch) + 1), 256);
-  L.max_pairs = backward ? max_pairs(batch, total_k, kBwdBN) : max_pairs(batch, total_q, kFwdItemRows);
+  L.max_pairs = backward ? max_pairs(batch, total_k, kBwdBN) : max_pairs(batch, total_q, fwd_item_rows(D));
   L.pairs = off;
   off = align_up(off + 8 * static_cast<size_t>(L.max_pairs), 256);
   if (backward) {
@@ -115,30 +118,30 @@ __device__ __forceinline__ SeqInfo seq_info(const int32_t* cu_q, const KeyRows& 
   return s;
 }
 
-// Row, in the key/value tensor, of the first key of key tile j of sequence
-// b. A tile never straddles two pages: the page size is a multiple of the
-// tile.
-__device__ __forceinline__ int key_tile_row(const KeyRows& kr, int b, const SeqInfo& s, int j) {
+// Row, in the key/value tensor, of the first key of key tile j (tiles of bn
+// keys) of sequence b. A tile never straddles two pages: the page size is a
+// multiple of 128, hence of bn.
+__device__ __forceinline__ int key_tile_row(const KeyRows& kr, int b, const SeqInfo& s, int j, int bn = kFwdBN) {
   if (kr.block_table) {
-    const int pos = j * kFwdBN;
+    const int pos = j * bn;
     const int page = __ldg(kr.block_table + static_cast<size_t>(b) * kr.max_pages + pos / kr.page_size);
     return page * kr.page_size + pos % kr.page_size;
   }
-  return s.k0 + j * kFwdBN;
+  return s.k0 + j * bn;
 }
 
 // Number of key tiles (kFwdBN keys) visible from the query rows below
 // row_end (clamped to lq), given the bottom-right causal rule
 // j <= i + (lk - lq). Tiles wholly above the diagonal are skipped; the
 // visible tiles are always a prefix 0 .. n-1.
-__host__ __device__ inline int fwd_k_tiles(int row_end, int lq, int lk, bool causal) {
+__host__ __device__ inline int fwd_k_tiles(int row_end, int lq, int lk, bool causal, int bn = kFwdBN) {
   if (lk <= 0 || lq <= 0) return 0;
-  const int nk = (lk + kFwdBN - 1) / kFwdBN;
+  const int nk = (lk + bn - 1) / bn;
   if (!causal) return nk;
   const int rmax = (row_end < lq ? row_end : lq) - 1;
   const long long last = static_cast<long long>(rmax) + lk - lq;
   if (last < 0) return 0;
-  const long long n = last / kFwdBN + 1;
+  const long long n = last / bn + 1;
   return n < nk ? static_cast<int>(n) : nk;
 }
 

@@ -20,6 +20,7 @@ struct SchedArgs {
   int batch, total_q, total_k, max_seqlen_q, max_seqlen_k;
   int causal;
   int mode;
+  int item_rows;  // forward: query rows per work item (fwd_item_rows)
   void* workspace;
   size_t seq_off_offset, pairs_offset;
   int max_pairs;
@@ -43,6 +44,10 @@ struct FwdArgs {
 // 128 rows x 64 columns, 128-byte swizzle.
 cudaError_t launch_fwd(const FwdArgs& a, const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                        cudaStream_t stream);
+// head_dim 256: 128-row query items, 64-key tiles; tm_k / tm_v with boxes of
+// 64 rows x 64 columns.
+cudaError_t launch_fwd_d256(const FwdArgs& a, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                            const CUtensorMap& tm_v, cudaStream_t stream);
 
 struct BwdArgs {
   const int32_t* cu_q;

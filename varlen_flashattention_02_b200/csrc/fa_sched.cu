@@ -25,8 +25,8 @@ namespace {
 constexpr int kThreads = 1024;
 constexpr int kBins = 2048;  // cost buckets; costs above kBins-1 share the last
 
-__device__ __forceinline__ int pair_cost(const SeqInfo& s, int tile, int mode, bool causal) {
-  if (mode == 0) return fwd_k_tiles((tile + 1) * kFwdItemRows, s.lq, s.lk, causal);
+__device__ __forceinline__ int pair_cost(const SeqInfo& s, int tile, int mode, int rows, bool causal) {
+  if (mode == 0) return fwd_k_tiles((tile + 1) * rows, s.lq, s.lk, causal);
   int b, e;
   bwd_q_tiles(tile, s.lq, s.lk, causal, &b, &e);
   return e - b;
@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(kThreads) sched_prep_kernel(SchedArgs a) {
   }
 
   // Tiles per sequence, exclusive prefix sum into seq_off.
-  const int tile = a.mode == 0 ? kFwdItemRows : kBwdBN;
+  const int tile = a.mode == 0 ? a.item_rows : kBwdBN;
   for (int base = 0; base < a.batch; base += kThreads) {
     const int b = base + tid;
     int n = 0;
@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(kThreads) sched_prep_kernel(SchedArgs a) {
   for (int p = tid; p < n_pairs; p += kThreads) {
     const int b = find_seq(seq_off, a.batch, p);
     const SeqInfo s = seq_info(a.cu_q, a.keys, b);
-    const int c = min(pair_cost(s, p - seq_off[b], a.mode, causal), kBins - 1);
+    const int c = min(pair_cost(s, p - seq_off[b], a.mode, a.item_rows, causal), kBins - 1);
     atomicAdd(&s_hist[c], 1);
   }
   __syncthreads();
@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(kThreads) sched_prep_kernel(SchedArgs a) {
     const int b = find_seq(seq_off, a.batch, p);
     const SeqInfo s = seq_info(a.cu_q, a.keys, b);
     const int t = p - seq_off[b];
-    const int c = min(pair_cost(s, t, a.mode, causal), kBins - 1);
+    const int c = min(pair_cost(s, t, a.mode, a.item_rows, causal), kBins - 1);
     const int pos = atomicAdd(&s_hist[c], 1);
     pairs[pos] = make_int2(b, t);
   }
