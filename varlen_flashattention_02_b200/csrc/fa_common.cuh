@@ -100,6 +100,31 @@ struct KeyRows {
 struct SeqInfo {
   int q0, lq, k0, lk;
 };
+
+// The three key layouts, for kernels specialised on one of them.
+enum KeyLayout : int { kKeysPacked = 0, kKeysSlots = 1, kKeysPaged = 2 };
+__host__ __device__ inline int key_layout(const KeyRows& kr) {
+  return kr.block_table ? kKeysPaged : (kr.seqlens_k ? kKeysSlots : kKeysPacked);
+}
+template <int KL>
+__device__ __forceinline__ SeqInfo seq_info_l(const int32_t* cu_q, const KeyRows& kr, int b) {
+  SeqInfo s;
+  s.q0 = __ldg(cu_q + b);
+  s.lq = __ldg(cu_q + b + 1) - s.q0;
+  if (KL == kKeysPaged) {
+    s.k0 = 0;  // rows come from the block table (key_tile_row)
+    s.lk = __ldg(kr.seqlens_k + b);
+  } else if (KL == kKeysSlots) {
+    const int lp = kr.leftpad_k ? __ldg(kr.leftpad_k + b) : 0;
+    s.k0 = b * kr.cache_rows + lp;
+    s.lk = __ldg(kr.seqlens_k + b) - lp;
+  } else {
+    s.k0 = __ldg(kr.cu_k + b);
+    s.lk = __ldg(kr.cu_k + b + 1) - s.k0;
+  }
+  return s;
+}
+
 __device__ __forceinline__ SeqInfo seq_info(const int32_t* cu_q, const KeyRows& kr, int b) {
   SeqInfo s;
   s.q0 = __ldg(cu_q + b);

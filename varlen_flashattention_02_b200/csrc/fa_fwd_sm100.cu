@@ -111,6 +111,7 @@ struct Item {
   int nk[2];    // key tiles visible from query tile w (0 when the tile is empty)
 };
 
+template <int KL>
 __device__ __forceinline__ Item get_item(const FwdArgs& a, const int2* pairs, int idx) {
   Item it;
   const int2 pr = pairs[idx / a.H];
@@ -118,7 +119,7 @@ __device__ __forceinline__ Item get_item(const FwdArgs& a, const int2* pairs, in
   it.hk = it.h / a.group;
   it.b = pr.x;
   it.t = pr.y;
-  it.s = seq_info(a.cu_q, a.keys, it.b);
+  it.s = seq_info_l<KL>(a.cu_q, a.keys, it.b);
 #pragma unroll
   for (int w = 0; w < 2; ++w) {
     const int row0 = (it.t * kQTiles + w) * BM;
@@ -131,7 +132,9 @@ __device__ __forceinline__ Item get_item(const FwdArgs& a, const int2* pairs, in
 // Each role is inlined into the kernel: code after a register reallocation
 // may not call out-of-line functions.
 
-template <int D>
+// KL: the key layout (packed, cache slots, pages), a compile-time choice:
+// code for the other layouts in these loops slows them measurably.
+template <int D, int KL>
 __device__ __forceinline__ void qk_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const FwdArgs& a,
                                             uint8_t* smem, Bars& bars, WsHeader* hdr, const int2* pairs,
                                             int n_items, const Abort& ab) {
@@ -142,7 +145,7 @@ __device__ __forceinline__ void qk_producer(const CUtensorMap* tm_q, const CUten
     int idx;
     if (!publish_item(bars.items, ni, &hdr->work_counter, n_items, idx, ab)) goto done;
     if (idx < 0) break;
-    const Item it = get_item(a, pairs, idx);
+    const Item it = get_item<KL>(a, pairs, idx);
     const int nkb = max(it.nk[0], it.nk[1]);
     if (nkb == 0) continue;
 #pragma unroll
@@ -158,7 +161,8 @@ __device__ __forceinline__ void qk_producer(const CUtensorMap* tm_q, const CUten
     for (int j = 0; j < nkb; ++j, ++kc) {
       const int st = kc % NK;
       const uint32_t use = kc / NK;
-      const int krow = key_tile_row(a.keys, it.b, it.s, j);  // (a block-table read when paged)
+      // A block-table read for a paged cache, issued before the stage wait.
+      const int krow = KL == kKeysPaged ? key_tile_row(a.keys, it.b, it.s, j) : it.s.k0 + j * BN;
       if (use > 0 && !wait_bar(&bars.k_empty[st], (use - 1) & 1, ab)) goto done;
       mbar_arrive_expect_tx(&bars.k_full[st], L::kTileBytes);
       for (int c = 0; c < L::kChunks; ++c)
@@ -174,7 +178,7 @@ done:
   for (uint32_t i = (kc > NK ? kc - NK : 0); i < kc; ++i) wait_bar_final(&bars.k_full[i % NK], (i / NK) & 1, ab);
 }
 
-template <int D>
+template <int D, int KL>
 __device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, const FwdArgs& a, uint8_t* smem, Bars& bars,
                                            const int2* pairs, const Abort& ab) {
   using L = FwdSmem<D>;
@@ -185,12 +189,12 @@ __device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, const FwdArg
     const int idx = consume_item<false>(bars.items, ni, slot, ab);
     if (idx < 0) break;
     mbar_arrive(&bars.items.empty[slot]);
-    const Item it = get_item(a, pairs, idx);
+    const Item it = get_item<KL>(a, pairs, idx);
     const int nkb = max(it.nk[0], it.nk[1]);
     for (int j = 0; j < nkb; ++j, ++vc) {
       const int st = vc % NV;
       const uint32_t use = vc / NV;
-      const int vrow = key_tile_row(a.keys, it.b, it.s, j);
+      const int vrow = KL == kKeysPaged ? key_tile_row(a.keys, it.b, it.s, j) : it.s.k0 + j * BN;
       if (use > 0 && !wait_bar(&bars.v_empty[st], (use - 1) & 1, ab)) goto done;
       mbar_arrive_expect_tx(&bars.v_full[st], L::kTileBytes);
       for (int c = 0; c < L::kChunks; ++c)
@@ -210,7 +214,7 @@ done:
 // tile j): wait for P_w,j; O_w (+)= P_w,j V_j; S_w,j+1 = Q_w K_{j+1}^T.
 // The two tiles' softmax phases are thereby offset: while warpgroup w works
 // on S_w,j+1, the tensor pipe runs the other tile's PV and Q K^T.
-template <int D>
+template <int D, int KL>
 __device__ __forceinline__ void mma_issuer(const FwdArgs& a, uint8_t* smem, Bars& bars, const int2* pairs,
                                            uint32_t tmem, const Abort& ab) {
   using L = FwdSmem<D>;
@@ -242,7 +246,7 @@ __device__ __forceinline__ void mma_issuer(const FwdArgs& a, uint8_t* smem, Bars
     if (idx < 0) break;
     if (elect_one()) mbar_arrive(&bars.items.empty[slot]);
     __syncwarp();
-    const Item it = get_item(a, pairs, idx);
+    const Item it = get_item<KL>(a, pairs, idx);
     const int nkb = max(it.nk[0], it.nk[1]);
     if (nkb == 0) continue;
 #pragma unroll
@@ -322,7 +326,7 @@ done:
 }
 
 // Softmax of query tile W (warps 4+4W .. 7+4W, one thread per row).
-template <int D, bool CAUSAL, int W>
+template <int D, bool CAUSAL, int W, int KL>
 __device__ __forceinline__ void softmax_role(const FwdArgs& a, uint8_t* smem, Bars& bars, const int2* pairs,
                                              uint32_t tmem, const Abort& ab, int warp, int lane) {
   using L = FwdSmem<D>;
@@ -338,7 +342,7 @@ __device__ __forceinline__ void softmax_role(const FwdArgs& a, uint8_t* smem, Ba
     if (idx < 0) break;
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars.items.empty[slot]);
-    const Item it = get_item(a, pairs, idx);
+    const Item it = get_item<KL>(a, pairs, idx);
     const int nk = it.nk[W];
     if (nk == 0) continue;  // the epilogue warpgroup writes empty rows
     const int tq = it.t * kQTiles + W;  // 128-row tile of the sequence
@@ -442,7 +446,7 @@ __device__ __forceinline__ void softmax_role(const FwdArgs& a, uint8_t* smem, Ba
 
 // Epilogue (warps 12-15, one thread per row): out = O / l for both query
 // tiles of every item, zero rows for tiles that see no key.
-template <int D>
+template <int D, int KL>
 __device__ __forceinline__ void epilogue_role(const FwdArgs& a, uint8_t* smem, Bars& bars, const int2* pairs,
                                               uint32_t tmem, const Abort& ab, int warp, int lane) {
   using L = FwdSmem<D>;
@@ -456,7 +460,7 @@ __device__ __forceinline__ void epilogue_role(const FwdArgs& a, uint8_t* smem, B
     if (idx < 0) break;
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars.items.empty[slot]);
-    const Item it = get_item(a, pairs, idx);
+    const Item it = get_item<KL>(a, pairs, idx);
 #pragma unroll
     for (int w = 0; w < 2; ++w) {
       const int r = (it.t * kQTiles + w) * BM + row;
@@ -518,7 +522,7 @@ __device__ __forceinline__ void teardown(uint32_t tmem, int warp) {
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, int KL>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
@@ -585,37 +589,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (wgroup == 0) {
     warpgroup_reg_dealloc<kRegsLoad>();
     if (warp == 0) {
-      if (lane == 0) qk_producer<D>(&tm_q, &tm_k, a, smem, bars, hdr, pairs, n_items, ab);
+      if (lane == 0) qk_producer<D, KL>(&tm_q, &tm_k, a, smem, bars, hdr, pairs, n_items, ab);
     } else if (warp == 1) {
-      mma_issuer<D>(a, smem, bars, pairs, tmem, ab);
+      mma_issuer<D, KL>(a, smem, bars, pairs, tmem, ab);
     } else if (warp == 2) {
-      if (lane == 0) v_producer<D>(&tm_v, a, smem, bars, pairs, ab);
+      if (lane == 0) v_producer<D, KL>(&tm_v, a, smem, bars, pairs, ab);
     }
     __syncwarp();
     teardown(tmem, warp);
   } else if (wgroup == 1) {
     warpgroup_reg_alloc<kRegsSoftmax>();
-    softmax_role<D, CAUSAL, 0>(a, smem, bars, pairs, tmem, ab, warp, lane);
+    softmax_role<D, CAUSAL, 0, KL>(a, smem, bars, pairs, tmem, ab, warp, lane);
     __syncwarp();
     teardown(tmem, warp);
   } else if (wgroup == 2) {
     warpgroup_reg_alloc<kRegsSoftmax>();
-    softmax_role<D, CAUSAL, 1>(a, smem, bars, pairs, tmem, ab, warp, lane);
+    softmax_role<D, CAUSAL, 1, KL>(a, smem, bars, pairs, tmem, ab, warp, lane);
     __syncwarp();
     teardown(tmem, warp);
   } else {
     warpgroup_reg_dealloc<kRegsEpilogue>();
-    epilogue_role<D>(a, smem, bars, pairs, tmem, ab, warp, lane);
+    epilogue_role<D, KL>(a, smem, bars, pairs, tmem, ab, warp, lane);
     __syncwarp();
     teardown(tmem, warp);
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, int KL>
 cudaError_t launch_one(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        cudaStream_t stream) {
   using L = FwdSmem<D>;
-  auto kern = fwd_kernel<D, CAUSAL>;
+  auto kern = fwd_kernel<D, CAUSAL, KL>;
   // The warpgroups' register shares add up to exactly the launch's 128 per
   // thread; with any other count an increase could wait forever.
   static const int launch_regs = [&] {
@@ -629,12 +633,25 @@ cudaError_t launch_one(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMa
   return cudaGetLastError();
 }
 
+template <int KL>
+cudaError_t launch_layout(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          cudaStream_t stream) {
+  if (a.D == 64)
+    return a.causal ? launch_one<64, true, KL>(a, tq, tk, tv, stream)
+                    : launch_one<64, false, KL>(a, tq, tk, tv, stream);
+  return a.causal ? launch_one<128, true, KL>(a, tq, tk, tv, stream)
+                  : launch_one<128, false, KL>(a, tq, tk, tv, stream);
+}
+
 }  // namespace
 
 cudaError_t launch_fwd(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        cudaStream_t stream) {
-  if (a.D == 64) return a.causal ? launch_one<64, true>(a, tq, tk, tv, stream) : launch_one<64, false>(a, tq, tk, tv, stream);
-  return a.causal ? launch_one<128, true>(a, tq, tk, tv, stream) : launch_one<128, false>(a, tq, tk, tv, stream);
+  switch (key_layout(a.keys)) {
+    case kKeysPaged: return launch_layout<kKeysPaged>(a, tq, tk, tv, stream);
+    case kKeysSlots: return launch_layout<kKeysSlots>(a, tq, tk, tv, stream);
+    default: return launch_layout<kKeysPacked>(a, tq, tk, tv, stream);
+  }
 }
 
 }  // namespace fa
