@@ -105,7 +105,8 @@ fa_status_t fa_varlen_fwd(const void* q, const void* k, const void* v, const int
 /* Backward of L = sum(out * dout) given the forward's out and softmax_lse.
  * Recomputes the probabilities from softmax_lse; writes dq, dk, dv.
  * The query gradient is accumulated with fp32 atomic reductions, so dq may
- * differ in the last bits between runs. */
+ * differ in the last bits between runs (fa_varlen_bwd_deterministic does
+ * not). */
 fa_status_t fa_varlen_bwd(const void* dout, const void* q, const void* k, const void* v, const void* out,
                           const float* softmax_lse, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
                           int batch, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int num_heads,
@@ -138,6 +139,25 @@ fa_status_t fa_varlen_bwd_gqa(const void* dout, const void* q, const void* k, co
                               int num_heads, int num_heads_k, int head_dim, float softmax_scale, int causal,
                               void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
                               fa_cuda_stream_t stream);
+
+/* Deterministic backward (same arguments and results as fa_varlen_bwd_gqa).
+ * The page "Flash-Atención y Flash-Atención-2" (backward paragraph) has the
+ * column workers aggregate the query gradient with atomic additions, whose
+ * order, and so whose rounding, changes from run to run. Here every 64-row
+ * query tile receives its dQ contributions in key-tile order: key tile j
+ * waits (on a per-tile counter in the workspace) until key tiles 0 .. j-1
+ * have added theirs. dq, dk and dv are then bitwise identical from run to
+ * run for the same inputs, sizes and GPU model. The work list is taken in
+ * (sequence, key tile) order rather than longest first, so the call is
+ * somewhat slower than fa_varlen_bwd_gqa. A wait that does not end within
+ * its time limit is reported as FA_ERR_DEVICE_TIMEOUT in the workspace
+ * status. Workspace: fa_varlen_bwd_workspace_size. */
+fa_status_t fa_varlen_bwd_deterministic(const void* dout, const void* q, const void* k, const void* v,
+                                        const void* out, const float* softmax_lse, const int32_t* cu_seqlens_q,
+                                        const int32_t* cu_seqlens_k, int batch, int total_q, int total_k,
+                                        int max_seqlen_q, int max_seqlen_k, int num_heads, int num_heads_k,
+                                        int head_dim, float softmax_scale, int causal, void* dq, void* dk, void* dv,
+                                        void* workspace, size_t workspace_bytes, fa_cuda_stream_t stream);
 
 /* Forward over a key/value cache: the keys of each sequence are given by a
  * per-sequence length instead of cumulative offsets, optionally after some

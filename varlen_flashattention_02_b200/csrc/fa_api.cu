@@ -117,7 +117,7 @@ fa_status_t run_fwd(const void* q, const void* k, const void* v, const int32_t* 
 
   t_events.next = 0;
   fa::SchedArgs sa{cu_seqlens_q, keys, batch, total_q, total_k, max_seqlen_q, max_seqlen_k,
-                   causal ? 1 : 0, 0, fa::fwd_item_rows(head_dim), workspace, L.seq_off, L.pairs, L.max_pairs};
+                   causal ? 1 : 0, 0, fa::fwd_item_rows(head_dim), 0, workspace, L.seq_off, L.pairs, L.max_pairs};
   if (timed_launch(stream, [&] { return fa::launch_sched_prep(sa, stream); }) != cudaSuccess) return FA_ERR_CUDA;
   if (total_q == 0) return FA_OK;
 
@@ -154,6 +154,88 @@ fa_status_t run_fwd(const void* q, const void* k, const void* v, const int32_t* 
   fa_args.grid = static_cast<int>(items < sms ? items : sms);
   auto launch = head_dim == 256 ? fa::launch_fwd_d256 : fa::launch_fwd;
   if (timed_launch(stream, [&] { return launch(fa_args, tq, tk, tv, stream); }) != cudaSuccess) return FA_ERR_CUDA;
+  return FA_OK;
+}
+
+// The backward; deterministic: dQ contributions added in key-tile order.
+fa_status_t run_bwd(const void* dout, const void* q, const void* k, const void* v, const void* out,
+                    const float* softmax_lse, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int batch,
+                    int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int num_heads, int num_heads_k,
+                    int head_dim, float softmax_scale, int causal, void* dq, void* dk, void* dv, void* workspace,
+                    size_t workspace_bytes, fa_cuda_stream_t stream_, bool deterministic) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  fa_status_t st = check_sizes(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, num_heads, num_heads_k,
+                               head_dim, softmax_scale);
+  if (st != FA_OK) return st;
+  if (head_dim == 256) return FA_ERR_UNSUPPORTED;  // the backward supports head_dim 64 and 128
+  if (!cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARGUMENT;
+  if (total_q > 0 && (!q || !dout || !out || !softmax_lse || !dq || !aligned16(q) || !aligned16(dout) ||
+                      !aligned16(out) || !aligned16(dq)))
+    return FA_ERR_INVALID_ARGUMENT;
+  if (total_k > 0 && (!k || !v || !dk || !dv || !aligned16(k) || !aligned16(v) || !aligned16(dk) || !aligned16(dv)))
+    return FA_ERR_INVALID_ARGUMENT;
+  const WsLayout L = fa::ws_layout(true, batch, total_q, total_k, num_heads, head_dim);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < L.total)
+    return FA_ERR_WORKSPACE;
+
+  t_events.next = 0;
+  fa::SchedArgs sa{cu_seqlens_q, fa::KeyRows{cu_seqlens_k, nullptr, nullptr, 0, nullptr, 0, 0}, batch, total_q, total_k,
+                   max_seqlen_q, max_seqlen_k, causal ? 1 : 0, 1, 0, deterministic ? 1 : 0, workspace, L.seq_off,
+                   L.pairs, L.max_pairs};
+  if (timed_launch(stream, [&] { return fa::launch_sched_prep(sa, stream); }) != cudaSuccess) return FA_ERR_CUDA;
+  if (total_q == 0 && total_k == 0) return FA_OK;
+
+  const int HD = num_heads * head_dim;
+  const int HkD = num_heads_k * head_dim;
+  CUtensorMap tq, tk, tv, tdo;
+  const void* anyp = total_q > 0 ? q : k;
+  const void* qp = total_q > 0 ? q : anyp;
+  const void* dop = total_q > 0 ? dout : anyp;
+  const void* kp = total_k > 0 ? k : anyp;
+  const void* vp = total_k > 0 ? v : anyp;
+  const int qrows = total_q > 0 ? total_q : total_k;
+  const int krows = total_k > 0 ? total_k : total_q;
+  // With one side empty the other side's pointer stands in; the widths then
+  // follow that tensor's head count.
+  const int qcols = total_q > 0 ? HD : HkD;
+  const int kcols = total_k > 0 ? HkD : HD;
+  if (!encode_map(&tq, qp, qrows, qcols, fa::kBwdBM) || !encode_map(&tdo, dop, qrows, qcols, fa::kBwdBM) ||
+      !encode_map(&tk, kp, krows, kcols, fa::kBwdBN) || !encode_map(&tv, vp, krows, kcols, fa::kBwdBN))
+    return FA_ERR_CUDA;
+
+  const int sms = sm_count();
+  if (sms <= 0) return FA_ERR_CUDA;
+  const long long items = static_cast<long long>(L.max_pairs) * num_heads_k;
+  fa::BwdArgs b{};
+  b.cu_q = cu_seqlens_q;
+  b.keys = fa::KeyRows{cu_seqlens_k, nullptr, nullptr, 0, nullptr, 0, 0};
+  b.dout = dout;
+  b.out = out;
+  b.lse = softmax_lse;
+  b.dq = dq;
+  b.dk = dk;
+  b.dv = dv;
+  b.workspace = workspace;
+  b.pairs_offset = L.pairs;
+  b.dvec_offset = L.dvec;
+  b.qcount_offset = L.qcount;
+  b.deterministic = deterministic ? 1 : 0;
+  b.dqacc_offset = L.dqacc;
+  b.tq_pad = L.tq_pad;
+  b.H = num_heads;
+  b.Hk = num_heads_k;
+  b.group = num_heads / num_heads_k;
+  b.D = head_dim;
+  b.total_q = total_q;
+  b.total_k = total_k;
+  b.causal = causal ? 1 : 0;
+  b.scale = softmax_scale;
+  b.scale_log2 = softmax_scale * 1.4426950408889634f;
+  b.grid = static_cast<int>(items < sms ? items : sms);
+  if (timed_launch(stream, [&] { return fa::launch_bwd_preprocess(b, stream); }) != cudaSuccess ||
+      timed_launch(stream, [&] { return fa::launch_bwd_main(b, tq, tk, tv, tdo, stream); }) != cudaSuccess ||
+      timed_launch(stream, [&] { return fa::launch_bwd_convert(b, stream); }) != cudaSuccess)
+    return FA_ERR_CUDA;
   return FA_OK;
 }
 
@@ -253,78 +335,21 @@ fa_status_t fa_varlen_bwd_gqa(const void* dout, const void* q, const void* k, co
                               int batch, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
                               int num_heads, int num_heads_k, int head_dim, float softmax_scale, int causal,
                               void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
-                              fa_cuda_stream_t stream_) {
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  fa_status_t st = check_sizes(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, num_heads, num_heads_k,
-                               head_dim, softmax_scale);
-  if (st != FA_OK) return st;
-  if (head_dim == 256) return FA_ERR_UNSUPPORTED;  // the backward supports head_dim 64 and 128
-  if (!cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARGUMENT;
-  if (total_q > 0 && (!q || !dout || !out || !softmax_lse || !dq || !aligned16(q) || !aligned16(dout) ||
-                      !aligned16(out) || !aligned16(dq)))
-    return FA_ERR_INVALID_ARGUMENT;
-  if (total_k > 0 && (!k || !v || !dk || !dv || !aligned16(k) || !aligned16(v) || !aligned16(dk) || !aligned16(dv)))
-    return FA_ERR_INVALID_ARGUMENT;
-  const WsLayout L = fa::ws_layout(true, batch, total_q, total_k, num_heads, head_dim);
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < L.total)
-    return FA_ERR_WORKSPACE;
+                              fa_cuda_stream_t stream) {
+  return run_bwd(dout, q, k, v, out, softmax_lse, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
+                 max_seqlen_k, num_heads, num_heads_k, head_dim, softmax_scale, causal, dq, dk, dv, workspace,
+                 workspace_bytes, stream, false);
+}
 
-  t_events.next = 0;
-  fa::SchedArgs sa{cu_seqlens_q, fa::KeyRows{cu_seqlens_k, nullptr, nullptr, 0, nullptr, 0, 0}, batch, total_q, total_k,
-                   max_seqlen_q, max_seqlen_k, causal ? 1 : 0, 1, 0, workspace, L.seq_off, L.pairs, L.max_pairs};
-  if (timed_launch(stream, [&] { return fa::launch_sched_prep(sa, stream); }) != cudaSuccess) return FA_ERR_CUDA;
-  if (total_q == 0 && total_k == 0) return FA_OK;
-
-  const int HD = num_heads * head_dim;
-  const int HkD = num_heads_k * head_dim;
-  CUtensorMap tq, tk, tv, tdo;
-  const void* anyp = total_q > 0 ? q : k;
-  const void* qp = total_q > 0 ? q : anyp;
-  const void* dop = total_q > 0 ? dout : anyp;
-  const void* kp = total_k > 0 ? k : anyp;
-  const void* vp = total_k > 0 ? v : anyp;
-  const int qrows = total_q > 0 ? total_q : total_k;
-  const int krows = total_k > 0 ? total_k : total_q;
-  // With one side empty the other side's pointer stands in; the widths then
-  // follow that tensor's head count.
-  const int qcols = total_q > 0 ? HD : HkD;
-  const int kcols = total_k > 0 ? HkD : HD;
-  if (!encode_map(&tq, qp, qrows, qcols, fa::kBwdBM) || !encode_map(&tdo, dop, qrows, qcols, fa::kBwdBM) ||
-      !encode_map(&tk, kp, krows, kcols, fa::kBwdBN) || !encode_map(&tv, vp, krows, kcols, fa::kBwdBN))
-    return FA_ERR_CUDA;
-
-  const int sms = sm_count();
-  if (sms <= 0) return FA_ERR_CUDA;
-  const long long items = static_cast<long long>(L.max_pairs) * num_heads_k;
-  fa::BwdArgs b{};
-  b.cu_q = cu_seqlens_q;
-  b.keys = fa::KeyRows{cu_seqlens_k, nullptr, nullptr, 0, nullptr, 0, 0};
-  b.dout = dout;
-  b.out = out;
-  b.lse = softmax_lse;
-  b.dq = dq;
-  b.dk = dk;
-  b.dv = dv;
-  b.workspace = workspace;
-  b.pairs_offset = L.pairs;
-  b.dvec_offset = L.dvec;
-  b.dqacc_offset = L.dqacc;
-  b.tq_pad = L.tq_pad;
-  b.H = num_heads;
-  b.Hk = num_heads_k;
-  b.group = num_heads / num_heads_k;
-  b.D = head_dim;
-  b.total_q = total_q;
-  b.total_k = total_k;
-  b.causal = causal ? 1 : 0;
-  b.scale = softmax_scale;
-  b.scale_log2 = softmax_scale * 1.4426950408889634f;
-  b.grid = static_cast<int>(items < sms ? items : sms);
-  if (timed_launch(stream, [&] { return fa::launch_bwd_preprocess(b, stream); }) != cudaSuccess ||
-      timed_launch(stream, [&] { return fa::launch_bwd_main(b, tq, tk, tv, tdo, stream); }) != cudaSuccess ||
-      timed_launch(stream, [&] { return fa::launch_bwd_convert(b, stream); }) != cudaSuccess)
-    return FA_ERR_CUDA;
-  return FA_OK;
+fa_status_t fa_varlen_bwd_deterministic(const void* dout, const void* q, const void* k, const void* v,
+                                        const void* out, const float* softmax_lse, const int32_t* cu_seqlens_q,
+                                        const int32_t* cu_seqlens_k, int batch, int total_q, int total_k,
+                                        int max_seqlen_q, int max_seqlen_k, int num_heads, int num_heads_k,
+                                        int head_dim, float softmax_scale, int causal, void* dq, void* dk, void* dv,
+                                        void* workspace, size_t workspace_bytes, fa_cuda_stream_t stream) {
+  return run_bwd(dout, q, k, v, out, softmax_lse, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
+                 max_seqlen_k, num_heads, num_heads_k, head_dim, softmax_scale, causal, dq, dk, dv, workspace,
+                 workspace_bytes, stream, true);
 }
 
 void fa_set_kernel_events(void* const* events, int n_pairs) {

@@ -118,7 +118,29 @@ __device__ __forceinline__ Step item_step(const Item& it, int s) {
   return Step{it.h0 + r, it.i0 + s - r * it.nt};
 }
 
-template <int D, bool CAUSAL>
+// Deterministic mode: wait until the dQ additions of key tiles 0 .. j-1 to
+// the query tile whose counter is `cnt` are done (bounded, like every wait).
+__device__ __forceinline__ bool wait_dq_turn(const uint32_t* cnt, uint32_t j, const Abort& ab) {
+  if (ld_acquire_gpu(cnt) >= j) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (ld_acquire_gpu(cnt) >= j) return true;
+    if (*ab.flag) return false;
+    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      raise_abort(ab);
+      return false;
+    }
+  }
+}
+
+// DET: deterministic dQ. Every query tile receives its dQ contributions in
+// key-tile order j = 0, 1, ...: key tile j waits on the tile's counter for
+// its turn, adds, waits for the addition to land and advances the counter.
+// The work list is then in (sequence, key tile) order, so a key tile only
+// ever waits for items claimed before it: no cycle of waits can form.
+template <int D, bool CAUSAL, bool DET>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -132,6 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int2* pairs = reinterpret_cast<const int2*>(static_cast<const char*>(a.workspace) + a.pairs_offset);
   const float* dvec = reinterpret_cast<const float*>(static_cast<const char*>(a.workspace) + a.dvec_offset);
   float* dqacc = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + a.dqacc_offset);
+  uint32_t* qcount = reinterpret_cast<uint32_t*>(static_cast<char*>(a.workspace) + a.qcount_offset);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -425,6 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     float* stage = reinterpret_cast<float*>(smem + L::kStage);
     uint32_t p = 0, m = 0, ni = 0;
+    uint32_t* det_prev = nullptr;  // deterministic mode: counter whose turn is still to be passed on
     for (;;) {
       int islot;
       const int idx = consume_item<true>(bars.items, ni, islot, ab);
@@ -472,9 +496,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (t == 0) {
           const Step sp = item_step(it, s);
           const size_t q0 = static_cast<size_t>(it.s.q0) + static_cast<size_t>(sp.t) * BM;
-          bulk_reduce_add_f32(dqacc + (static_cast<size_t>(sp.h) * a.tq_pad + q0) * D, stage, BM * D * 4);
-          bulk_commit_group();
+          uint32_t* cnt = qcount + static_cast<size_t>(sp.h) * a.tq_pad + q0;
+          const bool turn = !DET || wait_dq_turn(cnt, static_cast<uint32_t>(it.j), ab);
+          if (turn) {
+            if (DET) fence_proxy_async_global();
+            bulk_reduce_add_f32(dqacc + (static_cast<size_t>(sp.h) * a.tq_pad + q0) * D, stage, BM * D * 4);
+            bulk_commit_group();
+            if (DET) {
+              // Pass the previous step's turn on once its addition has been
+              // performed (it was issued a step ago, so this rarely waits);
+              // this step's turn passes on at the next step or item end.
+              if (det_prev) {
+                bulk_wait_group1();
+                fence_proxy_async_global();
+                st_release_gpu(det_prev, static_cast<uint32_t>(it.j) + 1u);
+              }
+              det_prev = cnt;
+            }
+          }
         }
+      }
+      if (DET && t == 0 && det_prev) {
+        bulk_wait_group0();
+        fence_proxy_async_global();
+        st_release_gpu(det_prev, static_cast<uint32_t>(it.j) + 1u);
+        det_prev = nullptr;
       }
       // dK, dV of this key tile.
       if (!named_bar_and(1, 128, wait_bar(&bars.dkv_full, m & 1, ab))) goto drain_done;
@@ -559,7 +605,11 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdArgs a) {
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   float* dvec = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + a.dvec_offset);
   float* dqacc = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + a.dqacc_offset);
-  if (lane == 0) dvec[static_cast<size_t>(h) * a.tq_pad + row] = acc;
+  if (lane == 0) {
+    dvec[static_cast<size_t>(h) * a.tq_pad + row] = acc;
+    reinterpret_cast<uint32_t*>(static_cast<char*>(a.workspace) + a.qcount_offset)[static_cast<size_t>(h) * a.tq_pad +
+                                                                                  row] = 0u;
+  }
   float4* z = reinterpret_cast<float4*>(dqacc + (static_cast<size_t>(h) * a.tq_pad + row) * D);
   for (int i = lane; i < D / 4; i += 32) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
@@ -587,11 +637,11 @@ __global__ void __launch_bounds__(256) bwd_convert_kernel(const BwdArgs a) {
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool DET>
 cudaError_t launch_main(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const CUtensorMap& tdo, cudaStream_t stream) {
   using L = BwdSmem<D>;
-  auto kern = bwd_kernel<D, CAUSAL>;
+  auto kern = bwd_kernel<D, CAUSAL, DET>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
   kern<<<a.grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, tdo, a);
@@ -611,13 +661,20 @@ cudaError_t launch_bwd_preprocess(const BwdArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_main(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+template <bool DET>
+cudaError_t launch_main_det(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, cudaStream_t stream) {
   if (a.D == 64)
-    return a.causal ? launch_main<64, true>(a, tq, tk, tv, tdo, stream)
-                    : launch_main<64, false>(a, tq, tk, tv, tdo, stream);
-  return a.causal ? launch_main<128, true>(a, tq, tk, tv, tdo, stream)
-                  : launch_main<128, false>(a, tq, tk, tv, tdo, stream);
+    return a.causal ? launch_main<64, true, DET>(a, tq, tk, tv, tdo, stream)
+                    : launch_main<64, false, DET>(a, tq, tk, tv, tdo, stream);
+  return a.causal ? launch_main<128, true, DET>(a, tq, tk, tv, tdo, stream)
+                  : launch_main<128, false, DET>(a, tq, tk, tv, tdo, stream);
+}
+
+cudaError_t launch_bwd_main(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, cudaStream_t stream) {
+  return a.deterministic ? launch_main_det<true>(a, tq, tk, tv, tdo, stream)
+                         : launch_main_det<false>(a, tq, tk, tv, tdo, stream);
 }
 
 cudaError_t launch_bwd_convert(const BwdArgs& a, cudaStream_t stream) {

@@ -49,6 +49,7 @@ struct WsLayout {
   size_t seq_off;  // int32 [batch + 1]: first pair index of each sequence
   size_t pairs;    // int2  [max_pairs]: (sequence, tile), longest first
   size_t dvec;     // fp32  [H, tq_pad] (backward only): rowsum(dO * O)
+  size_t qcount;   // u32   [H, tq_pad] (backward only): dQ additions done per query tile (deterministic mode)
   size_t dqacc;    // fp32  [H, tq_pad, D] (backward only)
   size_t total;
   int max_pairs;
@@ -67,6 +68,8 @@ __host__ __device__ inline WsLayout ws_layout(bool backward, int batch, int tota
     L.tq_pad = dq_rows_padded(total_q);
     L.dvec = off;
     off = align_up(off + sizeof(float) * static_cast<size_t>(H) * L.tq_pad, 256);
+    L.qcount = off;
+    off = align_up(off + sizeof(uint32_t) * static_cast<size_t>(H) * L.tq_pad, 256);
     L.dqacc = off;
     off = align_up(off + sizeof(float) * static_cast<size_t>(H) * L.tq_pad * D, 256);
   }

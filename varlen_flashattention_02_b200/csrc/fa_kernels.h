@@ -20,7 +20,8 @@ struct SchedArgs {
   int batch, total_q, total_k, max_seqlen_q, max_seqlen_k;
   int causal;
   int mode;
-  int item_rows;  // forward: query rows per work item (fwd_item_rows)
+  int item_rows;      // forward: query rows per work item (fwd_item_rows)
+  int natural_order;  // 1: tiles of each sequence in increasing order (tile-major), not longest first
   void* workspace;
   size_t seq_off_offset, pairs_offset;
   int max_pairs;
@@ -59,7 +60,8 @@ struct BwdArgs {
   void* dk;           // bf16 [total_k, H, D]
   void* dv;           // bf16 [total_k, H, D]
   void* workspace;
-  size_t pairs_offset, dvec_offset, dqacc_offset;
+  size_t pairs_offset, dvec_offset, qcount_offset, dqacc_offset;
+  int deterministic;  // add dQ contributions in key-tile order (bitwise reproducible)
   int tq_pad;
   int H, D, total_q, total_k;  // H: query heads
   int Hk, group;               // key/value heads, query heads per key/value head

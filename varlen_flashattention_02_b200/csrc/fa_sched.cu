@@ -9,7 +9,8 @@
 //      rows; backward: key tiles of 128 rows) and prefix-sums them;
 //   3. orders all (sequence, tile) pairs by their number of visible tiles on
 //      the other side, most work first, so that the persistent kernels,
-//      which take pairs in order, start the longest items first.
+//      which take pairs in order, start the longest items first (or, for
+//      the deterministic backward, keeps (sequence, tile) order).
 // No padding is ever enumerated: a sequence of length n yields ceil(n/T)
 // pairs (T = 256 forward, 128 backward). Pages: "Mecanismo cu_seqlens en
 // FlashAttention", "Lógica de cálculo de longitud" (lengths from offsets)
@@ -75,6 +76,7 @@ __global__ void __launch_bounds__(kThreads) sched_prep_kernel(SchedArgs a) {
   __shared__ int s_warp[32];
   __shared__ int s_err;
   __shared__ int s_total;
+  __shared__ int s_max_tiles;
   auto* hdr = reinterpret_cast<WsHeader*>(a.workspace);
   auto* seq_off = reinterpret_cast<int32_t*>(static_cast<char*>(a.workspace) + a.seq_off_offset);
   auto* pairs = reinterpret_cast<int2*>(static_cast<char*>(a.workspace) + a.pairs_offset);
@@ -85,6 +87,7 @@ __global__ void __launch_bounds__(kThreads) sched_prep_kernel(SchedArgs a) {
   if (tid == 0) {
     s_err = 0;
     s_total = 0;
+    s_max_tiles = 0;
     hdr->work_counter = 0;
     if (a.cu_q[0] != 0 || a.cu_q[a.batch] != a.total_q) s_err = 1;
     if (!cache && (a.keys.cu_k[0] != 0 || a.keys.cu_k[a.batch] != a.total_k)) s_err = 1;
@@ -136,6 +139,7 @@ __global__ void __launch_bounds__(kThreads) sched_prep_kernel(SchedArgs a) {
     if (b < a.batch) {
       const int len = a.mode == 0 ? a.cu_q[b + 1] - a.cu_q[b] : a.keys.cu_k[b + 1] - a.keys.cu_k[b];
       n = (len + tile - 1) / tile;
+      atomicMax(&s_max_tiles, n);
     }
     const int incl = block_inclusive_scan(n, s_warp);
     if (b < a.batch) seq_off[b] = s_total + incl - n;
@@ -154,11 +158,32 @@ __global__ void __launch_bounds__(kThreads) sched_prep_kernel(SchedArgs a) {
   }
   __syncthreads();
 
+  // Tile-major order (deterministic backward): every sequence's tile 0, then
+  // every tile 1, ...; the tiles of one sequence are then claimed in
+  // increasing order, which is what the deterministic dQ turn-taking needs
+  // (the order among sequences does not matter to the result). Tile 0 sees
+  // the most queries under the causal mask, so this is also longest first.
+  // Sequences with more tiles than histogram buckets fall back to plain
+  // (sequence, tile) order.
+  const bool tile_major = a.natural_order && s_max_tiles <= kBins;
+  if (a.natural_order && !tile_major) {
+    for (int p = tid; p < n_pairs; p += kThreads) {
+      const int b = find_seq(seq_off, a.batch, p);
+      pairs[p] = make_int2(b, p - seq_off[b]);
+    }
+    if (tid == 0) {
+      hdr->status = FA_OK;
+      hdr->n_pairs = static_cast<uint32_t>(n_pairs);
+    }
+    return;
+  }
+
   // Histogram of costs.
   for (int p = tid; p < n_pairs; p += kThreads) {
     const int b = find_seq(seq_off, a.batch, p);
     const SeqInfo s = seq_info(a.cu_q, a.keys, b);
-    const int c = min(pair_cost(s, p - seq_off[b], a.mode, a.item_rows, causal), kBins - 1);
+    const int t = p - seq_off[b];
+    const int c = tile_major ? kBins - 1 - t : min(pair_cost(s, t, a.mode, a.item_rows, causal), kBins - 1);
     atomicAdd(&s_hist[c], 1);
   }
   __syncthreads();
@@ -188,7 +213,7 @@ __global__ void __launch_bounds__(kThreads) sched_prep_kernel(SchedArgs a) {
     const int b = find_seq(seq_off, a.batch, p);
     const SeqInfo s = seq_info(a.cu_q, a.keys, b);
     const int t = p - seq_off[b];
-    const int c = min(pair_cost(s, t, a.mode, a.item_rows, causal), kBins - 1);
+    const int c = tile_major ? kBins - 1 - t : min(pair_cost(s, t, a.mode, a.item_rows, causal), kBins - 1);
     const int pos = atomicAdd(&s_hist[c], 1);
     pairs[pos] = make_int2(b, t);
   }

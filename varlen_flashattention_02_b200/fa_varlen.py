@@ -54,6 +54,9 @@ def _load():
     lib.fa_varlen_bwd_gqa.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, ctypes.c_float, I,
                                       P, P, P, P, S, P]
     lib.fa_varlen_bwd_gqa.restype = I
+    lib.fa_varlen_bwd_deterministic.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, ctypes.c_float, I,
+                                                P, P, P, P, S, P]
+    lib.fa_varlen_bwd_deterministic.restype = I
     lib.fa_varlen_fwd_kvcache.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, ctypes.c_float, I, P, P, P, S, P]
     lib.fa_varlen_fwd_kvcache.restype = I
     lib.fa_varlen_fwd_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, ctypes.c_float, I, P, P,
@@ -74,7 +77,7 @@ lib = _load()
 
 EXPORTED = ("fa_varlen_fwd_workspace_size", "fa_varlen_bwd_workspace_size", "fa_varlen_fwd",
             "fa_varlen_bwd", "fa_varlen_fwd_gqa", "fa_varlen_bwd_gqa", "fa_varlen_fwd_kvcache",
-            "fa_varlen_fwd_paged", "fa_varlen_fwd_noalloc",
+            "fa_varlen_fwd_paged", "fa_varlen_bwd_deterministic", "fa_varlen_fwd_noalloc",
             "fa_get_device_status", "fa_set_kernel_events", "fa_status_string")
 
 
@@ -203,9 +206,19 @@ def fa_varlen_fwd_gqa(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, ma
     return out, softmax_lse
 
 
+def fa_varlen_bwd_deterministic(dout, q, k, v, out, softmax_lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
+                                max_seqlen_k: int, softmax_scale: float, causal: bool, dq=None, dk=None, dv=None,
+                                workspace=None, stream=None):
+    """Backward whose results are bitwise identical from run to run (dQ
+    contributions added in key-tile order). k, v may have fewer heads than q
+    as in fa_varlen_bwd_gqa. Returns (dq, dk, dv)."""
+    return fa_varlen_bwd_gqa(dout, q, k, v, out, softmax_lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                             max_seqlen_k, softmax_scale, causal, dq, dk, dv, workspace, stream, _deterministic=True)
+
+
 def fa_varlen_bwd_gqa(dout, q, k, v, out, softmax_lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
                       max_seqlen_k: int, softmax_scale: float, causal: bool, dq=None, dk=None, dv=None,
-                      workspace=None, stream=None):
+                      workspace=None, stream=None, _deterministic=False):
     """Grouped-/multi-query backward: dk, dv have Hk heads and hold the sums
     over each key/value head's query heads. Returns (dq, dk, dv)."""
     _check_qkv("q", q)
@@ -226,12 +239,12 @@ def fa_varlen_bwd_gqa(dout, q, k, v, out, softmax_lse, cu_seqlens_q, cu_seqlens_
     need = bwd_workspace_size(batch, Tq, Tk, H, D)
     if workspace is None:
         workspace = new_workspace(need, q.device)
-    rc = lib.fa_varlen_bwd_gqa(_p(dout), _p(q), _p(k), _p(v), _p(out), _p(softmax_lse), _p(cu_seqlens_q),
-                               _p(cu_seqlens_k), batch, Tq, Tk, int(max_seqlen_q), int(max_seqlen_k), H, Hk, D,
-                               float(softmax_scale), int(bool(causal)), _p(dq), _p(dk), _p(dv),
-                               _p(workspace), workspace.numel(), _stream(stream))
+    fn = lib.fa_varlen_bwd_deterministic if _deterministic else lib.fa_varlen_bwd_gqa
+    rc = fn(_p(dout), _p(q), _p(k), _p(v), _p(out), _p(softmax_lse), _p(cu_seqlens_q), _p(cu_seqlens_k), batch,
+            Tq, Tk, int(max_seqlen_q), int(max_seqlen_k), H, Hk, D, float(softmax_scale), int(bool(causal)),
+            _p(dq), _p(dk), _p(dv), _p(workspace), workspace.numel(), _stream(stream))
     if rc != FA_OK:
-        raise FaError(rc, "fa_varlen_bwd_gqa")
+        raise FaError(rc, "fa_varlen_bwd_deterministic" if _deterministic else "fa_varlen_bwd_gqa")
     return dq, dk, dv
 
 
