@@ -212,6 +212,50 @@ fa_status_t fa_varlen_fwd_paged(const void* q, const void* k_pages, const void* 
                                 float softmax_scale, int causal, void* out, float* softmax_lse, void* workspace,
                                 size_t workspace_bytes, fa_cuda_stream_t stream);
 
+/* Where the keys and values of each sequence live, for
+ * fa_varlen_fwd_splitkv (exactly one of the three layouts):
+ *  - packed: cu_seqlens_k [batch+1] cumulative offsets (as fa_varlen_fwd);
+ *  - key/value cache slots: seqlens_k, leftpad_k (or NULL), cache_rows (as
+ *    fa_varlen_fwd_kvcache; k and v are [batch * cache_rows, Hk, d]);
+ *  - paged cache: seqlens_k, block_table, page_size (a multiple of 128),
+ *    max_pages_per_seq (as fa_varlen_fwd_paged; k and v are
+ *    [num_pages * page_size, Hk, d]).
+ * total_rows is the number of rows of k and v. All pointers are device
+ * memory; unused fields are NULL / 0. */
+typedef struct {
+  const int32_t* cu_seqlens_k;
+  const int32_t* seqlens_k;
+  const int32_t* leftpad_k;
+  const int32_t* block_table;
+  int cache_rows;
+  int page_size;
+  int max_pages_per_seq;
+  int total_rows;
+} fa_kv_layout_t;
+
+/* Split-KV forward for decoding and other short-query calls (the page
+ * "FlashAttention-2 GPU work partitioning", section "Cómo documentar una
+ * diferencia técnica", separates prefill from token-by-token decoding, whose
+ * bottleneck differs). Same results as fa_varlen_fwd_gqa (and the cache
+ * forwards) for any num_splits; the work decomposition differs:
+ *  - the g = num_heads / num_heads_k query heads that share a key/value head
+ *    (g <= 128) and 128 / g consecutive query tokens of a sequence form one
+ *    128-row tile, so each key/value tile is read once per group;
+ *  - each tile's key tiles are divided into num_splits ranges processed in
+ *    parallel; each writes a normalised partial output and its logsumexp
+ *    into the workspace (fp32) and a combine kernel merges them
+ *    (num_splits = 1 writes out directly).
+ * head_dim 64 or 128 (FA_ERR_UNSUPPORTED otherwise). The workspace must
+ * hold fa_varlen_fwd_splitkv_workspace_size(...) bytes (0 = invalid sizes).
+ * Layout-specific checks are those of the matching entry point. */
+size_t fa_varlen_fwd_splitkv_workspace_size(int batch, int total_q, int num_heads, int num_heads_k, int head_dim,
+                                            int num_splits);
+fa_status_t fa_varlen_fwd_splitkv(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                                  const fa_kv_layout_t* kv, int batch, int total_q, int max_seqlen_q,
+                                  int max_seqlen_k, int num_heads, int num_heads_k, int head_dim, float softmax_scale,
+                                  int causal, int num_splits, void* out, float* softmax_lse, void* workspace,
+                                  size_t workspace_bytes, fa_cuda_stream_t stream);
+
 /* Forward for callers that cannot allocate device memory. The pages have no
  * counterpart of this entry point; it exists for the library's users.
  *

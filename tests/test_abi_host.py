@@ -137,3 +137,20 @@ def test_paged_rejects_page_size_not_multiple_of_tile(lib):
     rc = lib.fa_varlen_fwd_paged(FAKE, FAKE, FAKE, FAKE, None, FAKE, 2, 64, 8, 128, 4, 32, 256, 4, 4, 128,
                                  0.1, 1, FAKE, FAKE, FAKE, 1 << 20, None)
     assert rc == 1
+
+
+def test_splitkv_rejects(lib):
+    """Split-KV forward: a null layout or a split count below 1 is an invalid
+    argument; more than 128 query heads per key/value head is unsupported."""
+    from varlen_flashattention_02_b200 import fa_varlen
+
+    lay = fa_varlen.KvLayout()
+    lay.cu_seqlens_k = FAKE
+    lay.total_rows = 64
+    args = lambda lay_ptr, splits, H, Hk: lib.fa_varlen_fwd_splitkv(
+        FAKE, FAKE, FAKE, FAKE, lay_ptr, 2, 64, 32, 32, H, Hk, 128, 0.1, 1, splits, FAKE, FAKE, FAKE, 1 << 20, None)
+    assert args(None, 2, 8, 1) == 1
+    assert args(ctypes.byref(lay), 0, 8, 1) == 1
+    assert args(ctypes.byref(lay), 2, 256, 1) == 2
+    assert lib.fa_varlen_fwd_splitkv_workspace_size(2, 64, 8, 3, 128, 2) == 0
+    assert lib.fa_varlen_fwd_splitkv_workspace_size(2, 64, 8, 2, 128, 4) > 4 * 64 * 8 * 128 * 4

@@ -48,6 +48,22 @@ bool encode_map(CUtensorMap* map, const void* base, int rows, int cols, int box_
   return r == CUDA_SUCCESS;
 }
 
+// 3-D bf16 map over q viewed as [tokens, H, D]: box = 64 channels x g heads x
+// tq tokens, 128-byte swizzle; it lands the (token, head) rows of a group
+// as consecutive 128-byte rows.
+bool encode_map_q3(CUtensorMap* map, const void* base, int tokens, int H, int D, int g, int tq) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(tokens)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(g), static_cast<cuuint32_t>(tq)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Measurement hook state (per host thread): events recorded around each
 // kernel launch of the next calls.
 struct KernelEvents {
@@ -239,9 +255,118 @@ fa_status_t run_bwd(const void* dout, const void* q, const void* k, const void* 
   return FA_OK;
 }
 
+// Workspace of the split-KV forward: header, per-sequence offsets and the
+// (sequence, token tile) list, then the split partials.
+struct DecodeLayout {
+  size_t seq_off, pairs, opart, lpart, total;
+  int max_pairs, tq;
+};
+DecodeLayout decode_layout(int batch, int total_q, int H, int Hk, int D, int splits) {
+  DecodeLayout L{};
+  L.tq = 128 / (H / Hk);
+  size_t off = sizeof(fa::WsHeader);
+  L.seq_off = off;
+  off = fa::align_up(off + sizeof(int32_t) * (static_cast<size_t>(batch) + 1), 256);
+  L.max_pairs = fa::max_pairs(batch, total_q, L.tq);
+  L.pairs = off;
+  off = fa::align_up(off + 8 * static_cast<size_t>(L.max_pairs), 256);
+  const size_t rows = static_cast<size_t>(total_q) * H;
+  if (splits > 1) {
+    L.opart = off;
+    off = fa::align_up(off + sizeof(float) * splits * rows * D, 256);
+    L.lpart = off;
+    off = fa::align_up(off + sizeof(float) * splits * rows, 256);
+  }
+  L.total = off;
+  return L;
+}
+
+bool kv_layout_ok(const fa_kv_layout_t* kv) {
+  if (!kv || kv->total_rows < 0) return false;
+  if (kv->block_table) return kv->seqlens_k && kv->page_size > 0 && kv->max_pages_per_seq > 0 && !kv->leftpad_k;
+  if (kv->seqlens_k) return kv->cache_rows >= 0;
+  return kv->cu_seqlens_k != nullptr;
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t fa_varlen_fwd_splitkv_workspace_size(int batch, int total_q, int num_heads, int num_heads_k, int head_dim,
+                                            int num_splits) {
+  if (batch < 1 || total_q < 0 || num_heads < 1 || num_heads_k < 1 || num_heads % num_heads_k != 0 ||
+      num_heads / num_heads_k > 128 || num_splits < 1)
+    return 0;
+  return decode_layout(batch, total_q, num_heads, num_heads_k, head_dim, num_splits).total;
+}
+
+fa_status_t fa_varlen_fwd_splitkv(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                                  const fa_kv_layout_t* kv, int batch, int total_q, int max_seqlen_q,
+                                  int max_seqlen_k, int num_heads, int num_heads_k, int head_dim, float softmax_scale,
+                                  int causal, int num_splits, void* out, float* softmax_lse, void* workspace,
+                                  size_t workspace_bytes, fa_cuda_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (!kv_layout_ok(kv) || !cu_seqlens_q || num_splits < 1 || num_splits > 1024) return FA_ERR_INVALID_ARGUMENT;
+  const int total_k = kv->total_rows;
+  fa_status_t st = check_sizes(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, num_heads, num_heads_k,
+                               head_dim, softmax_scale);
+  if (st != FA_OK) return st;
+  if (head_dim == 256 || num_heads / num_heads_k > 128) return FA_ERR_UNSUPPORTED;
+  if (kv->block_table && kv->page_size % fa::kFwdBN != 0) return FA_ERR_UNSUPPORTED;
+  if (total_q > 0 && (!q || !out || !softmax_lse || !aligned16(q) || !aligned16(out))) return FA_ERR_INVALID_ARGUMENT;
+  if (total_k > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return FA_ERR_INVALID_ARGUMENT;
+  const DecodeLayout L = decode_layout(batch, total_q, num_heads, num_heads_k, head_dim, num_splits);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < L.total)
+    return FA_ERR_WORKSPACE;
+  const fa::KeyRows keys{kv->block_table || kv->seqlens_k ? nullptr : kv->cu_seqlens_k, kv->seqlens_k, kv->leftpad_k,
+                         kv->cache_rows, kv->block_table, kv->max_pages_per_seq, kv->page_size};
+
+  t_events.next = 0;
+  fa::SchedArgs sa{cu_seqlens_q, keys, batch, total_q, total_k, max_seqlen_q, max_seqlen_k,
+                   causal ? 1 : 0, 0, L.tq, 0, workspace, L.seq_off, L.pairs, L.max_pairs};
+  if (timed_launch(stream, [&] { return fa::launch_sched_prep(sa, stream); }) != cudaSuccess) return FA_ERR_CUDA;
+  if (total_q == 0) return FA_OK;
+
+  const int g = num_heads / num_heads_k;
+  const int HkD = num_heads_k * head_dim;
+  CUtensorMap tq3, tk, tv;
+  const void* kp = total_k > 0 ? k : q;
+  const void* vp = total_k > 0 ? v : q;
+  const int krows = total_k > 0 ? total_k : total_q;
+  const int kcols = total_k > 0 ? HkD : num_heads * head_dim;
+  if (!encode_map_q3(&tq3, q, total_q, num_heads, head_dim, g, L.tq) ||
+      !encode_map(&tk, kp, krows, kcols, fa::kFwdBN) || !encode_map(&tv, vp, krows, kcols, fa::kFwdBN))
+    return FA_ERR_CUDA;
+
+  const int sms = sm_count();
+  if (sms <= 0) return FA_ERR_CUDA;
+  const long long items = static_cast<long long>(L.max_pairs) * num_heads_k * num_splits;
+  fa::DecodeArgs d{};
+  d.cu_q = cu_seqlens_q;
+  d.keys = keys;
+  d.out = out;
+  d.lse = softmax_lse;
+  char* ws = static_cast<char*>(workspace);
+  d.opart = num_splits > 1 ? reinterpret_cast<float*>(ws + L.opart) : nullptr;
+  d.lpart = num_splits > 1 ? reinterpret_cast<float*>(ws + L.lpart) : nullptr;
+  d.workspace = workspace;
+  d.pairs_offset = L.pairs;
+  d.H = num_heads;
+  d.Hk = num_heads_k;
+  d.group = g;
+  d.D = head_dim;
+  d.total_q = total_q;
+  d.tq = L.tq;
+  d.splits = num_splits;
+  d.causal = causal ? 1 : 0;
+  d.scale_log2 = softmax_scale * 1.4426950408889634f;
+  d.grid = static_cast<int>(items < sms ? items : sms);
+  if (timed_launch(stream, [&] { return fa::launch_decode(d, tq3, tk, tv, stream); }) != cudaSuccess ||
+      timed_launch(stream, [&] { return fa::launch_decode_combine(d, stream); }) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return FA_OK;
+}
+
 
 size_t fa_varlen_fwd_workspace_size(int batch, int total_q, int num_heads, int head_dim) {
   if (batch < 1 || total_q < 0 || num_heads < 1) return 0;

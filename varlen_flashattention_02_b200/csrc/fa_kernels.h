@@ -50,6 +50,33 @@ cudaError_t launch_fwd(const FwdArgs& a, const CUtensorMap& tm_q, const CUtensor
 cudaError_t launch_fwd_d256(const FwdArgs& a, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                             const CUtensorMap& tm_v, cudaStream_t stream);
 
+// Split-KV forward with the query heads of a key/value group packed into
+// the rows of one tile (the decode path): an item is (sequence, key/value
+// head, tile of tq = 128 / group query tokens, key split); its 128 rows are
+// (token, head-in-group) pairs. With splits > 1 every split writes a
+// normalised partial output and its logsumexp (fp32) and the combine kernel
+// merges them. tm_q3: 3-D map over q as [tokens, H, D] with box (64, group,
+// tq); tm_k / tm_v as for launch_fwd.
+struct DecodeArgs {
+  const int32_t* cu_q;
+  KeyRows keys;
+  void* out;        // bf16 [total_q, H, D]
+  float* lse;       // fp32 [H, total_q]
+  float* opart;     // fp32 [splits, total_q * H, D] (splits > 1)
+  float* lpart;     // fp32 [splits, total_q * H]    (splits > 1)
+  void* workspace;  // header + pairs
+  size_t pairs_offset;
+  int H, Hk, group, D, total_q;
+  int tq;           // query tokens per item
+  int splits;
+  int causal;
+  float scale_log2;
+  int grid;
+};
+cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tm_q3, const CUtensorMap& tm_k,
+                          const CUtensorMap& tm_v, cudaStream_t stream);
+cudaError_t launch_decode_combine(const DecodeArgs& a, cudaStream_t stream);
+
 struct BwdArgs {
   const int32_t* cu_q;
   KeyRows keys;      // packed layout only

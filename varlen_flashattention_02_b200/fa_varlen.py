@@ -34,6 +34,13 @@ class FaError(RuntimeError):
         super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
 
 
+class KvLayout(ctypes.Structure):
+    """fa_kv_layout_t: where the keys and values of each sequence live."""
+    _fields_ = [("cu_seqlens_k", ctypes.c_void_p), ("seqlens_k", ctypes.c_void_p), ("leftpad_k", ctypes.c_void_p),
+                ("block_table", ctypes.c_void_p), ("cache_rows", ctypes.c_int), ("page_size", ctypes.c_int),
+                ("max_pages_per_seq", ctypes.c_int), ("total_rows", ctypes.c_int)]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
@@ -57,6 +64,11 @@ def _load():
     lib.fa_varlen_bwd_deterministic.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, ctypes.c_float, I,
                                                 P, P, P, P, S, P]
     lib.fa_varlen_bwd_deterministic.restype = I
+    lib.fa_varlen_fwd_splitkv_workspace_size.argtypes = [I, I, I, I, I, I]
+    lib.fa_varlen_fwd_splitkv_workspace_size.restype = S
+    lib.fa_varlen_fwd_splitkv.argtypes = [P, P, P, P, ctypes.POINTER(KvLayout), I, I, I, I, I, I, I,
+                                          ctypes.c_float, I, I, P, P, P, S, P]
+    lib.fa_varlen_fwd_splitkv.restype = I
     lib.fa_varlen_fwd_kvcache.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, ctypes.c_float, I, P, P, P, S, P]
     lib.fa_varlen_fwd_kvcache.restype = I
     lib.fa_varlen_fwd_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, ctypes.c_float, I, P, P,
@@ -77,7 +89,8 @@ lib = _load()
 
 EXPORTED = ("fa_varlen_fwd_workspace_size", "fa_varlen_bwd_workspace_size", "fa_varlen_fwd",
             "fa_varlen_bwd", "fa_varlen_fwd_gqa", "fa_varlen_bwd_gqa", "fa_varlen_fwd_kvcache",
-            "fa_varlen_fwd_paged", "fa_varlen_bwd_deterministic", "fa_varlen_fwd_noalloc",
+            "fa_varlen_fwd_paged", "fa_varlen_bwd_deterministic", "fa_varlen_fwd_splitkv",
+            "fa_varlen_fwd_splitkv_workspace_size", "fa_varlen_fwd_noalloc",
             "fa_get_device_status", "fa_set_kernel_events", "fa_status_string")
 
 
@@ -321,6 +334,53 @@ def fa_varlen_fwd_paged(q, k_pages, v_pages, cu_seqlens_q, seqlens_k, block_tabl
                                  _stream(stream))
     if rc != FA_OK:
         raise FaError(rc, "fa_varlen_fwd_paged")
+    return out, softmax_lse
+
+
+def fa_varlen_fwd_splitkv(q, k, v, cu_seqlens_q, max_seqlen_q: int, max_seqlen_k: int, softmax_scale: float,
+                          causal: bool, num_splits: int, cu_seqlens_k=None, seqlens_k=None, leftpad_k=None,
+                          block_table=None, out=None, softmax_lse=None, workspace=None, stream=None):
+    """Split-KV forward with the query heads of a key/value group packed into
+    one tile (decoding). Keys are packed (cu_seqlens_k; k, v [Tk, Hk, D]),
+    in cache slots (seqlens_k, optional leftpad_k; k, v [batch, rows, Hk,
+    D]) or paged (seqlens_k, block_table; k, v [pages, page_size, Hk, D]).
+    Returns (out, softmax_lse) as fa_varlen_fwd does."""
+    _check_qkv("q", q)
+    Tq, H, D = q.shape
+    _check_cu("cu_seqlens_q", cu_seqlens_q)
+    batch = cu_seqlens_q.numel() - 1
+    lay = KvLayout()
+    if block_table is not None:
+        num_pages, page_size, Hk = k.shape[0], k.shape[1], k.shape[2]
+        lay.seqlens_k, lay.block_table = seqlens_k.data_ptr(), block_table.data_ptr()
+        lay.page_size, lay.max_pages_per_seq, lay.total_rows = page_size, block_table.shape[1], num_pages * page_size
+    elif seqlens_k is not None:
+        rows, Hk = k.shape[1], k.shape[2]
+        lay.seqlens_k = seqlens_k.data_ptr()
+        lay.leftpad_k = leftpad_k.data_ptr() if leftpad_k is not None else None
+        lay.cache_rows, lay.total_rows = rows, batch * rows
+    else:
+        _check_cu("cu_seqlens_k", cu_seqlens_k)
+        Hk = k.shape[1]
+        lay.cu_seqlens_k, lay.total_rows = cu_seqlens_k.data_ptr(), k.shape[0]
+    for name, t in (("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or not t.is_cuda or t.shape[-1] != D:
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor with head_dim {D}")
+    if H % Hk != 0:
+        raise ValueError(f"query heads ({H}) must be a multiple of key/value heads ({Hk})")
+    if out is None:
+        out = torch.empty_like(q)
+    if softmax_lse is None:
+        softmax_lse = torch.empty((H, Tq), dtype=torch.float32, device=q.device)
+    need = int(lib.fa_varlen_fwd_splitkv_workspace_size(batch, Tq, H, Hk, D, int(num_splits)))
+    if workspace is None:
+        workspace = new_workspace(need, q.device)
+    rc = lib.fa_varlen_fwd_splitkv(_p(q), _p(k), _p(v), _p(cu_seqlens_q), ctypes.byref(lay), batch, Tq,
+                                   int(max_seqlen_q), int(max_seqlen_k), H, Hk, D, float(softmax_scale),
+                                   int(bool(causal)), int(num_splits), _p(out), _p(softmax_lse), _p(workspace),
+                                   workspace.numel(), _stream(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_varlen_fwd_splitkv")
     return out, softmax_lse
 
 
