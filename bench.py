@@ -388,6 +388,7 @@ def run_ours(args, rank, world, local_rank):
     }
     if rank == 0 and not args.no_aux:
         result["fwd_by_workload"] = fwd_only_workloads(dev, stream, flush, peak)
+        result["decode_by_workload"] = decode_workloads(dev, stream, flush, float(peaks["hbm_gbs"]))
     return result, w
 
 
@@ -436,6 +437,52 @@ def fwd_only_workloads(dev, stream, flush, peak, iters=10):
         ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
         F = fwd_flops(w.cu_q, w.cu_k, w.heads, w.head_dim, w.causal)
         res[name] = {"ms": ms, "tflops": F / (ms * 1e-3) / 1e12, "pct_of_peak": 100 * F / (ms * 1e-3) / 1e12 / peak}
+        del q, k, v, out, lse, ws
+    return res
+
+
+def decode_workloads(dev, stream, flush, hbm_peak_gbs, iters=10):
+    """Split-KV decoding: one query token per sequence against a long key/value
+    cache, 32 query heads over 8 key/value heads, d=128. The bound is HBM: the
+    figure is the K/V bytes the call must read over its time, against the
+    measured copy bandwidth."""
+    import torch
+
+    from varlen_flashattention_02_b200 import fa_varlen
+
+    res = {}
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    for batch, lk in ((64, 8192), (4, 32768)):
+        H, Hk, D = 32, 8, 128
+        rng = np.random.default_rng(9)
+        q = torch.from_numpy(synth.bf16_normal(rng, (batch, H, D)).view(np.int16)).view(torch.bfloat16).to(dev)
+        k = torch.randn(batch * lk, Hk, D, device=dev, dtype=torch.bfloat16)
+        v = torch.randn(batch * lk, Hk, D, device=dev, dtype=torch.bfloat16)
+        cu_q = torch.arange(batch + 1, dtype=torch.int32, device=dev)
+        cu_k = torch.arange(batch + 1, dtype=torch.int32, device=dev) * lk
+        splits = max(1, min(lk // 128, -(-2 * sms // (batch * Hk))))
+        out = torch.empty_like(q)
+        lse = torch.empty((H, batch), dtype=torch.float32, device=dev)
+        ws = fa_varlen.new_workspace(int(fa_varlen.lib.fa_varlen_fwd_splitkv_workspace_size(batch, batch, H, Hk, D,
+                                                                                           splits)), dev)
+        call = lambda: fa_varlen.fa_varlen_fwd_splitkv(q, k, v, cu_q, 1, lk, D ** -0.5, True, splits, cu_seqlens_k=cu_k,
+                                                       out=out, softmax_lse=lse, workspace=ws, stream=stream)
+        for _ in range(3):
+            call()
+        evs = []
+        for _ in range(iters):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            call()
+            b.record(stream)
+            evs.append((a, b))
+        torch.cuda.synchronize(dev)
+        ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+        kv_bytes = 2 * batch * lk * Hk * D * 2
+        gbs = kv_bytes / (ms * 1e-3) / 1e9
+        res[f"decode {batch} seqs x {lk} keys, h32 kv8 d128, 1 query token, {splits} splits"] = {
+            "ms": ms, "kv_gbytes": kv_bytes / 1e9, "gbs": gbs, "pct_of_hbm_peak": 100 * gbs / hbm_peak_gbs}
         del q, k, v, out, lse, ws
     return res
 
