@@ -203,7 +203,7 @@ fa_status_t run_bwd(const void* dout, const void* q, const void* k, const void* 
 
   const int HD = num_heads * head_dim;
   const int HkD = num_heads_k * head_dim;
-  CUtensorMap tq, tk, tv, tdo;
+  fa::BwdMaps maps;
   const void* anyp = total_q > 0 ? q : k;
   const void* qp = total_q > 0 ? q : anyp;
   const void* dop = total_q > 0 ? dout : anyp;
@@ -215,8 +215,12 @@ fa_status_t run_bwd(const void* dout, const void* q, const void* k, const void* 
   // follow that tensor's head count.
   const int qcols = total_q > 0 ? HD : HkD;
   const int kcols = total_k > 0 ? HkD : HD;
-  if (!encode_map(&tq, qp, qrows, qcols, fa::kBwdBM) || !encode_map(&tdo, dop, qrows, qcols, fa::kBwdBM) ||
-      !encode_map(&tk, kp, krows, kcols, fa::kBwdBN) || !encode_map(&tv, vp, krows, kcols, fa::kBwdBN))
+  // dk / dv maps serve only stores of key tiles, which exist only when total_k > 0.
+  const void* dkp = total_k > 0 ? dk : anyp;
+  const void* dvp = total_k > 0 ? dv : anyp;
+  if (!encode_map(&maps.q, qp, qrows, qcols, fa::kBwdBM) || !encode_map(&maps.dout, dop, qrows, qcols, fa::kBwdBM) ||
+      !encode_map(&maps.k, kp, krows, kcols, fa::kBwdBN) || !encode_map(&maps.v, vp, krows, kcols, fa::kBwdBN) ||
+      !encode_map(&maps.dk, dkp, krows, kcols, fa::kBwdBN) || !encode_map(&maps.dv, dvp, krows, kcols, fa::kBwdBN))
     return FA_ERR_CUDA;
 
   const int sms = sm_count();
@@ -249,7 +253,7 @@ fa_status_t run_bwd(const void* dout, const void* q, const void* k, const void* 
   b.scale_log2 = softmax_scale * 1.4426950408889634f;
   b.grid = static_cast<int>(items < sms ? items : sms);
   if (timed_launch(stream, [&] { return fa::launch_bwd_preprocess(b, stream); }) != cudaSuccess ||
-      timed_launch(stream, [&] { return fa::launch_bwd_main(b, tq, tk, tv, tdo, stream); }) != cudaSuccess ||
+      timed_launch(stream, [&] { return fa::launch_bwd_main(b, maps, stream); }) != cudaSuccess ||
       timed_launch(stream, [&] { return fa::launch_bwd_convert(b, stream); }) != cudaSuccess)
     return FA_ERR_CUDA;
   return FA_OK;

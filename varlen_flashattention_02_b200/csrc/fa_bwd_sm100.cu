@@ -67,21 +67,6 @@ struct BwdSmem {
   static constexpr int kAlloc = kBytes + 1024;
 };
 
-struct Bars {
-  uint64_t kv_full, kv_empty;
-  uint64_t qdo_full[3], qdo_empty[3];
-  uint64_t st_full[2];
-  uint64_t ds_full[2], ds_empty[2];
-  uint64_t dq_full[2], dq_empty[2];
-  uint64_t dkv_full, dkv_empty;
-  uint64_t ld_full[3], ld_empty[3];
-  uint64_t drain;
-  ItemRing items;
-  uint32_t tmem_base;
-  int abort_flag;
-};
-static_assert(sizeof(Bars) <= 512, "barrier block fits its reserved space");
-
 // An item is (sequence, key/value head hk, key tile j). Its steps visit the
 // query tiles i0 .. i0+nt-1 that see the key tile, for each query head of
 // hk's group in turn: step s is query head h0 + s / nt, tile i0 + s % nt.
@@ -109,6 +94,22 @@ __device__ __forceinline__ Item get_item(const BwdArgs& a, const int2* pairs, in
   return it;
 }
 
+struct Bars {
+  uint64_t kv_full, kv_empty;
+  uint64_t qdo_full[3], qdo_empty[3];
+  uint64_t st_full[2];
+  uint64_t ds_full[2], ds_empty[2];
+  uint64_t dq_full[2], dq_empty[2];
+  uint64_t dkv_full, dv_empty, dk_empty;
+  uint64_t ld_full[3], ld_empty[3];
+  uint64_t drain;
+  ItemRing items;
+  Item item_data[kItemSlots];  // the published items, decoded once by the producer
+  uint32_t tmem_base;
+  int abort_flag;
+};
+static_assert(sizeof(Bars) <= 512, "barrier block fits its reserved space");
+
 // Query head and query tile of step s of an item.
 struct Step {
   int h, t;
@@ -135,6 +136,39 @@ __device__ __forceinline__ bool wait_dq_turn(const uint32_t* cnt, uint32_t j, co
   }
 }
 
+// Eight fp32 accumulator values (bit patterns) to eight bf16, times scale.
+__device__ __forceinline__ uint4 pack8_bf16(const uint32_t* y, float scale) {
+  uint4 w;
+  w.x = pack_bf16x2(__uint_as_float(y[0]) * scale, __uint_as_float(y[1]) * scale);
+  w.y = pack_bf16x2(__uint_as_float(y[2]) * scale, __uint_as_float(y[3]) * scale);
+  w.z = pack_bf16x2(__uint_as_float(y[4]) * scale, __uint_as_float(y[5]) * scale);
+  w.w = pack_bf16x2(__uint_as_float(y[6]) * scale, __uint_as_float(y[7]) * scale);
+  return w;
+}
+
+// One row of D accumulator values to bf16 in global memory, times scale.
+template <int D>
+__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_t (&x)[D / 32][32], float scale) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int e = 0; e < D / 8; ++e) d4[e] = pack8_bf16(x[e / 4] + 8 * (e % 4), scale);
+}
+
+// Row r of a [128 x D] bf16 tile into shared memory in the layout of the
+// 128-byte-swizzled TMA boxes (64 columns x 128 rows per box, box c at
+// c * 16 KB, 1024-byte aligned): the 16-byte unit u of a 128-byte row sits
+// at position u ^ (r % 8). The eight threads of a store phase therefore
+// write eight different bank groups.
+template <int D>
+__device__ __forceinline__ void stage_row_sw128(uint8_t* tile, const uint32_t (&x)[D / 32][32], float scale, int r) {
+  uint8_t* row = tile + r * 128;
+#pragma unroll
+  for (int e = 0; e < D / 8; ++e) {
+    const int c = e / 8, u = e % 8;
+    *reinterpret_cast<uint4*>(row + c * 16384 + ((u ^ (r & 7)) << 4)) = pack8_bf16(x[e / 4] + 8 * (e % 4), scale);
+  }
+}
+
 // DET: deterministic dQ. Every query tile receives its dQ contributions in
 // key-tile order j = 0, 1, ...: key tile j waits on the tile's counter for
 // its turn, adds, waits for the addition to land and advances the counter.
@@ -144,6 +178,7 @@ template <int D, bool CAUSAL, bool DET>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+               const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                const BwdArgs a) {
   using L = BwdSmem<D>;
   constexpr int NQ = L::kQStages;
@@ -174,7 +209,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.dq_empty[i], 4);
     }
     mbar_init(&bars.dkv_full, 1);
-    mbar_init(&bars.dkv_empty, 4);
+    mbar_init(&bars.dv_empty, 4);
+    mbar_init(&bars.dk_empty, 4);
     mbar_init(&bars.drain, 1);
     // Item consumers: MMA warp (1), row loaders (2), P/dS warps (4), drain warps (4).
     item_ring_init(bars.items, 11);
@@ -186,6 +222,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_do);
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tm_dk);
+    tma_prefetch_desc(&tm_dv);
   }
   if (warp == 1) {
     tmem_alloc(&bars.tmem_base, kTmemCols);
@@ -201,34 +241,61 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------------------------------------------------- producer
+      // It claims each item ahead of time (while the previous item's last
+      // Q/dO tiles are still in use), decodes it once for every role, warms
+      // L2 with its K/V tiles and loads the first Q/dO tiles before waiting
+      // for the K/V buffer, so an item's first step starts without an
+      // exposed load.
       uint32_t m = 0, p = 0, ni = 0;
+      auto load_qdo = [&](const Item& it, int s) -> bool {
+        const int st = p % NQ;
+        if (p >= NQ && !wait_bar(&bars.qdo_empty[st], ((p / NQ) - 1) & 1, ab)) return false;
+        const Step sp = item_step(it, s);
+        const int qrow = it.s.q0 + sp.t * BM;
+        uint8_t* sq = smem + L::kQdo + 2 * st * L::kQTile;
+        uint8_t* sdo = sq + L::kQTile;
+        mbar_arrive_expect_tx(&bars.qdo_full[st], 2 * L::kQTile);
+        for (int c = 0; c < L::kChunks; ++c) {
+          tma_load_2d(&tm_q, &bars.qdo_full[st], sq + c * L::kQChunk, sp.h * D + c * 64, qrow);
+          tma_load_2d(&tm_do, &bars.qdo_full[st], sdo + c * L::kQChunk, sp.h * D + c * 64, qrow);
+        }
+        ++p;
+        return true;
+      };
       for (;;) {
-        int idx;
-        if (!publish_item(bars.items, ni, &hdr->work_counter, n_items, idx, ab)) goto producer_done;
+        const int slot = ni % kItemSlots;
+        if (ni >= kItemSlots && !wait_bar(&bars.items.empty[slot], ((ni / kItemSlots) - 1) & 1, ab)) goto producer_done;
+        int idx = static_cast<int>(atomicAdd(&hdr->work_counter, 1u));
+        if (idx >= n_items) idx = -1;
+        Item it;
+        if (idx >= 0) {
+          it = get_item(a, pairs, idx);
+          bars.item_data[slot] = it;
+        }
+        *reinterpret_cast<volatile int*>(&bars.items.idx[slot]) = idx;
+        mbar_arrive(&bars.items.full[slot]);
+        ++ni;
         if (idx < 0) break;
-        const Item it = get_item(a, pairs, idx);
         if (it.n == 0) continue;
-        if (m > 0 && !wait_bar(&bars.kv_empty, (m - 1) & 1, ab)) goto producer_done;
         const int krow = it.s.k0 + it.j * BN;
+        if (m > 0)
+          for (int c = 0; c < L::kChunks; ++c) {
+            tma_prefetch_2d(&tm_k, it.hk * D + c * 64, krow);
+            tma_prefetch_2d(&tm_v, it.hk * D + c * 64, krow);
+          }
+        const int pre = it.n < NQ - 1 ? it.n : NQ - 1;
+        int s = 0;
+        for (; s < pre; ++s)
+          if (!load_qdo(it, s)) goto producer_done;
+        if (m > 0 && !wait_bar(&bars.kv_empty, (m - 1) & 1, ab)) goto producer_done;
         mbar_arrive_expect_tx(&bars.kv_full, 2 * L::kKTile);
         for (int c = 0; c < L::kChunks; ++c) {
           tma_load_2d(&tm_k, &bars.kv_full, smem + L::kK + c * L::kKChunk, it.hk * D + c * 64, krow);
           tma_load_2d(&tm_v, &bars.kv_full, smem + L::kV + c * L::kKChunk, it.hk * D + c * 64, krow);
         }
-        for (int s = 0; s < it.n; ++s, ++p) {
-          const int st = p % NQ;
-          if (p >= NQ && !wait_bar(&bars.qdo_empty[st], ((p / NQ) - 1) & 1, ab)) goto producer_done;
-          const Step sp = item_step(it, s);
-          const int qrow = it.s.q0 + sp.t * BM;
-          uint8_t* sq = smem + L::kQdo + 2 * st * L::kQTile;
-          uint8_t* sdo = sq + L::kQTile;
-          mbar_arrive_expect_tx(&bars.qdo_full[st], 2 * L::kQTile);
-          for (int c = 0; c < L::kChunks; ++c) {
-            tma_load_2d(&tm_q, &bars.qdo_full[st], sq + c * L::kQChunk, sp.h * D + c * 64, qrow);
-            tma_load_2d(&tm_do, &bars.qdo_full[st], sdo + c * L::kQChunk, sp.h * D + c * 64, qrow);
-          }
-        }
         ++m;
+        for (; s < it.n; ++s)
+          if (!load_qdo(it, s)) goto producer_done;
       }
     producer_done:
       if (m > 0) wait_bar_final(&bars.kv_full, (m - 1) & 1, ab);
@@ -255,9 +322,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       int slot;
       const int idx = consume_item<true>(bars.items, ni, slot, ab);
       if (idx < 0) break;
+      const Item it = bars.item_data[slot];
+      __syncwarp();
       if (elect_one()) mbar_arrive(&bars.items.empty[slot]);
       __syncwarp();
-      const Item it = get_item(a, pairs, idx);
       if (it.n == 0) continue;
       if (!wait_bar_warp(&bars.kv_full, m & 1, ab)) goto mma_done;
       tc_fence_after();
@@ -292,7 +360,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int pb = pp & 1;
           const int qs = pp % NQ;
           if (!wait_bar_warp(&bars.ds_full[pb], (pp >> 1) & 1, ab)) goto mma_done;
-          if (s == 1 && m > 0 && !wait_bar_warp(&bars.dkv_empty, (m - 1) & 1, ab)) goto mma_done;
+          // First step of an item: the drain group must have read the
+          // previous item's dV (then dK) out of TMEM.
+          if (s == 1 && m > 0 && !wait_bar_warp(&bars.dv_empty, (m - 1) & 1, ab)) goto mma_done;
           tc_fence_after();
           const uint64_t q_mn = qdo_mn0 + static_cast<uint64_t>((2 * qs * L::kQTile) >> 4);
           const uint64_t ds_k = ds_kmaj0 + static_cast<uint64_t>((pb * L::kDsTile) >> 4);
@@ -304,6 +374,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < BM / 16; ++kk)
               mma_ts(tmem + kColDV, tmem + kColS + pb * BM + kk * 8, q_mn + kQTileD + ((kk * 2048) >> 4), kIdKV,
                      (acc | kk) ? 1u : 0u);
+          }
+          __syncwarp();
+          if (s == 1 && m > 0 && !wait_bar_warp(&bars.dk_empty, (m - 1) & 1, ab)) goto mma_done;
+          tc_fence_after();
+          if (elect_one()) {
 #pragma unroll
             for (int kk = 0; kk < BM / 16; ++kk)
               mma_ss(tmem + kColDK, ds_k + ((kk * 32) >> 4), q_mn + ((kk * 2048) >> 4), kIdKV, (acc | kk) ? 1u : 0u);
@@ -338,9 +413,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int islot;
       const int idx = consume_item<true>(bars.items, ni, islot, ab);
       if (idx < 0) break;
+      const Item it = bars.item_data[islot];
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.items.empty[islot]);
-      const Item it = get_item(a, pairs, idx);
       for (int s = 0; s < it.n; ++s, ++p) {
         const int slot = p % NQ;
         if (p >= NQ && !wait_bar_warp(&bars.ld_empty[slot], ((p / NQ) - 1) & 1, ab)) goto loader_done;
@@ -374,9 +449,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int islot;
       const int idx = consume_item<true>(bars.items, ni, islot, ab);
       if (idx < 0) break;
+      const Item it = bars.item_data[islot];
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.items.empty[islot]);
-      const Item it = get_item(a, pairs, idx);
       const int kg = it.j * BN + kr;  // key index within the sequence
       const bool key_ok = kg < it.s.lk;
       const int diag = it.s.lk - it.s.lq;
@@ -455,8 +530,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Group-uniform: this group uses named barriers, so all four warps
       // must leave together (end of work, or an abort seen by any warp).
       if (!named_bar_and(1, 128, idx >= 0)) break;
+      const Item it = bars.item_data[islot];
+      __syncwarp();
       if (lane == 0) mbar_arrive(&bars.items.empty[islot]);
-      const Item it = get_item(a, pairs, idx);
       const int kg = it.j * BN + t;
       const bool key_ok = kg < it.s.lk;
       const size_t krow = (static_cast<size_t>(it.s.k0) + kg) * a.Hk + it.hk;
@@ -522,39 +598,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         st_release_gpu(det_prev, static_cast<uint32_t>(it.j) + 1u);
         det_prev = nullptr;
       }
-      // dK, dV of this key tile.
+      // dK, dV of this key tile. dV is read out of TMEM first and released
+      // at once, so the next item's first dV MMAs wait only for that read;
+      // dK follows. A whole tile leaves through TMA stores from the stage
+      // (the coalesced path, which keeps the load/store unit free for the
+      // P/dS warps); a tile cut by the end of its sequence is stored row by
+      // row, so that no row of the next sequence is touched.
       if (!named_bar_and(1, 128, wait_bar(&bars.dkv_full, m & 1, ab))) goto drain_done;
       tc_fence_after();
       {
-        uint4* dk = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.dk) + krow * D);
-        uint4* dv = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.dv) + krow * D);
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t x[32], y[32];
-          tmem_ld32(tmem + lane_base + kColDK + c * 32, x);
-          tmem_ld32(tmem + lane_base + kColDV + c * 32, y);
-          tmem_wait_ld();
-          if (key_ok) {
+        const bool whole = (it.j + 1) * BN <= it.s.lk;  // the same for the whole group
+        const int row0 = it.s.k0 + it.j * BN;
+        uint8_t* tile = smem + L::kStage;
+        uint32_t x[D / 32][32];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              uint4 wk, wv;
-              wk.x = pack_bf16x2(__uint_as_float(x[8 * e + 0]) * a.scale, __uint_as_float(x[8 * e + 1]) * a.scale);
-              wk.y = pack_bf16x2(__uint_as_float(x[8 * e + 2]) * a.scale, __uint_as_float(x[8 * e + 3]) * a.scale);
-              wk.z = pack_bf16x2(__uint_as_float(x[8 * e + 4]) * a.scale, __uint_as_float(x[8 * e + 5]) * a.scale);
-              wk.w = pack_bf16x2(__uint_as_float(x[8 * e + 6]) * a.scale, __uint_as_float(x[8 * e + 7]) * a.scale);
-              wv.x = pack_bf16x2(__uint_as_float(y[8 * e + 0]), __uint_as_float(y[8 * e + 1]));
-              wv.y = pack_bf16x2(__uint_as_float(y[8 * e + 2]), __uint_as_float(y[8 * e + 3]));
-              wv.z = pack_bf16x2(__uint_as_float(y[8 * e + 4]), __uint_as_float(y[8 * e + 5]));
-              wv.w = pack_bf16x2(__uint_as_float(y[8 * e + 6]), __uint_as_float(y[8 * e + 7]));
-              dk[c * 4 + e] = wk;
-              dv[c * 4 + e] = wv;
-            }
+        for (int c = 0; c < D / 32; ++c) tmem_ld32(tmem + lane_base + kColDV + c * 32, x[c]);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.dv_empty);
+        if (whole) {
+          if (t == 0) bulk_wait_group_read0();  // the last dQ reduction has read the stage
+          named_bar_sync(1, 128);
+          stage_row_sw128<D>(tile, x, 1.f, t);
+          fence_proxy_async_smem();
+          named_bar_sync(1, 128);
+          if (t == 0) {
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) tma_store_2d(&tm_dv, tile + c * 16384, it.hk * D + c * 64, row0);
+            bulk_commit_group();
           }
+        } else if (key_ok) {
+          store_row_bf16<D>(static_cast<__nv_bfloat16*>(a.dv) + krow * D, x, 1.f);
+        }
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) tmem_ld32(tmem + lane_base + kColDK + c * 32, x[c]);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.dk_empty);
+        if (whole) {
+          if (t == 0) bulk_wait_group_read0();  // the dV stores have read the stage
+          named_bar_sync(1, 128);
+          stage_row_sw128<D>(tile, x, a.scale, t);
+          fence_proxy_async_smem();
+          named_bar_sync(1, 128);
+          if (t == 0) {
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) tma_store_2d(&tm_dk, tile + c * 16384, it.hk * D + c * 64, row0);
+            bulk_commit_group();
+          }
+        } else if (key_ok) {
+          store_row_bf16<D>(static_cast<__nv_bfloat16*>(a.dk) + krow * D, x, a.scale);
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.dkv_empty);
       ++m;
     }
   drain_done:
@@ -638,13 +735,12 @@ __global__ void __launch_bounds__(256) bwd_convert_kernel(const BwdArgs a) {
 }
 
 template <int D, bool CAUSAL, bool DET>
-cudaError_t launch_main(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                        const CUtensorMap& tdo, cudaStream_t stream) {
+cudaError_t launch_main(const BwdArgs& a, const BwdMaps& m, cudaStream_t stream) {
   using L = BwdSmem<D>;
   auto kern = bwd_kernel<D, CAUSAL, DET>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
-  kern<<<a.grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, tdo, a);
+  kern<<<a.grid, kThreads, L::kAlloc, stream>>>(m.q, m.k, m.v, m.dout, m.dk, m.dv, a);
   return cudaGetLastError();
 }
 
@@ -662,19 +758,14 @@ cudaError_t launch_bwd_preprocess(const BwdArgs& a, cudaStream_t stream) {
 }
 
 template <bool DET>
-cudaError_t launch_main_det(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& tdo, cudaStream_t stream) {
+cudaError_t launch_main_det(const BwdArgs& a, const BwdMaps& m, cudaStream_t stream) {
   if (a.D == 64)
-    return a.causal ? launch_main<64, true, DET>(a, tq, tk, tv, tdo, stream)
-                    : launch_main<64, false, DET>(a, tq, tk, tv, tdo, stream);
-  return a.causal ? launch_main<128, true, DET>(a, tq, tk, tv, tdo, stream)
-                  : launch_main<128, false, DET>(a, tq, tk, tv, tdo, stream);
+    return a.causal ? launch_main<64, true, DET>(a, m, stream) : launch_main<64, false, DET>(a, m, stream);
+  return a.causal ? launch_main<128, true, DET>(a, m, stream) : launch_main<128, false, DET>(a, m, stream);
 }
 
-cudaError_t launch_bwd_main(const BwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& tdo, cudaStream_t stream) {
-  return a.deterministic ? launch_main_det<true>(a, tq, tk, tv, tdo, stream)
-                         : launch_main_det<false>(a, tq, tk, tv, tdo, stream);
+cudaError_t launch_bwd_main(const BwdArgs& a, const BwdMaps& m, cudaStream_t stream) {
+  return a.deterministic ? launch_main_det<true>(a, m, stream) : launch_main_det<false>(a, m, stream);
 }
 
 cudaError_t launch_bwd_convert(const BwdArgs& a, cudaStream_t stream) {

@@ -98,12 +98,15 @@ struct BwdArgs {
   int grid;
 };
 // Backward in three launches: preprocess (rowsum(dO*O) and zero the dQ
-// accumulator), main, dQ conversion. tm_q / tm_do: [rows, H*D], box 64 rows x
-// 64 columns; tm_k / tm_v: [rows, Hk*D], box 128 rows x 64 columns; all
-// 128-byte swizzle.
+// accumulator), main, dQ conversion. Tensor maps, all bf16 with 128-byte
+// swizzle and 64-column boxes: q / dout over [rows, H*D] with 64-row boxes
+// (loads); k / v over [rows, Hk*D] with 128-row boxes (loads); dk / dv over
+// [rows, Hk*D] with 128-row boxes (stores of whole key tiles).
+struct BwdMaps {
+  CUtensorMap q, k, v, dout, dk, dv;
+};
 cudaError_t launch_bwd_preprocess(const BwdArgs& a, cudaStream_t stream);
-cudaError_t launch_bwd_main(const BwdArgs& a, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
-                            const CUtensorMap& tm_v, const CUtensorMap& tm_do, cudaStream_t stream);
+cudaError_t launch_bwd_main(const BwdArgs& a, const BwdMaps& maps, cudaStream_t stream);
 cudaError_t launch_bwd_convert(const BwdArgs& a, cudaStream_t stream);
 
 }  // namespace fa
