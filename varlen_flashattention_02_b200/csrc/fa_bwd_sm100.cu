@@ -35,6 +35,8 @@
 // back to TMEM as bf16 and feeds the dV MMA directly; dS^T is written once to
 // shared memory in a layout that serves both the dK MMA (K-major A) and the
 // dQ^T MMA (MN-major B).
+#include <type_traits>
+
 #include "fa_common.cuh"
 #include "fa_kernels.h"
 
@@ -668,69 +670,102 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// The two streaming kernels around the main one take kUnits (row, head)
+// units per warp, consecutive in memory, and issue all their loads before
+// using any, so that enough bytes are in flight to run at HBM speed.
+constexpr int kUnits = 4;
+
 // Dv[h, r] = sum_c dO[r, h, c] * O[r, h, c] in fp32, and dQacc[h, r, :] = 0.
-// One warp per (row, head).
 template <int D>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdArgs a) {
-  const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  constexpr int E = D / 32;  // bf16 elements per lane: 4 (8 bytes) or 2 (4 bytes)
+  using V = typename std::conditional<E == 4, uint2, uint32_t>::type;
+  const long long units = static_cast<long long>(a.total_q) * a.H;
+  const long long u0 = ((static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5) * kUnits;
   const int lane = threadIdx.x & 31;
-  if (w >= static_cast<long long>(a.total_q) * a.H) return;
-  const int row = static_cast<int>(w / a.H), h = static_cast<int>(w % a.H);
-  const size_t base = static_cast<size_t>(w) * D;
-  constexpr int E = D / 32;  // bf16 elements per lane
-  const __nv_bfloat16* o = static_cast<const __nv_bfloat16*>(a.out) + base + lane * E;
-  const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(a.dout) + base + lane * E;
-  float acc = 0.f;
-  if constexpr (E == 4) {
-    const uint2 ov = *reinterpret_cast<const uint2*>(o), gv = *reinterpret_cast<const uint2*>(g);
-    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
-    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+  if (u0 >= units) return;
+  const V* o = reinterpret_cast<const V*>(static_cast<const __nv_bfloat16*>(a.out) + u0 * D) + lane;
+  const V* g = reinterpret_cast<const V*>(static_cast<const __nv_bfloat16*>(a.dout) + u0 * D) + lane;
+  V ov[kUnits], gv[kUnits];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const float2 x = __bfloat1622float2(o2[i]), y = __bfloat1622float2(g2[i]);
-      acc = fmaf(x.x, y.x, acc);
-      acc = fmaf(x.y, y.y, acc);
+  for (int i = 0; i < kUnits; ++i) {
+    if (u0 + i < units) {
+      ov[i] = o[i * 32];
+      gv[i] = g[i * 32];
+    } else {
+      ov[i] = V{};
+      gv[i] = V{};
     }
-  } else {
-    const uint32_t ov = *reinterpret_cast<const uint32_t*>(o), gv = *reinterpret_cast<const uint32_t*>(g);
-    const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ov));
-    const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv));
-    acc = fmaf(x.x, y.x, acc);
-    acc = fmaf(x.y, y.y, acc);
+  }
+  float acc[kUnits];
+#pragma unroll
+  for (int i = 0; i < kUnits; ++i) {
+    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov[i]);
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv[i]);
+    acc[i] = 0.f;
+#pragma unroll
+    for (int k = 0; k < E / 2; ++k) {
+      const float2 x = __bfloat1622float2(o2[k]), y = __bfloat1622float2(g2[k]);
+      acc[i] = fmaf(x.x, y.x, acc[i]);
+      acc[i] = fmaf(x.y, y.y, acc[i]);
+    }
   }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+    for (int i = 0; i < kUnits; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
   float* dvec = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + a.dvec_offset);
   float* dqacc = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + a.dqacc_offset);
-  if (lane == 0) {
-    dvec[static_cast<size_t>(h) * a.tq_pad + row] = acc;
-    reinterpret_cast<uint32_t*>(static_cast<char*>(a.workspace) + a.qcount_offset)[static_cast<size_t>(h) * a.tq_pad +
-                                                                                  row] = 0u;
+  uint32_t* qcount = reinterpret_cast<uint32_t*>(static_cast<char*>(a.workspace) + a.qcount_offset);
+#pragma unroll
+  for (int i = 0; i < kUnits; ++i) {
+    const long long u = u0 + i;
+    if (u >= units) break;
+    const int row = static_cast<int>(u / a.H), h = static_cast<int>(u % a.H);
+    const size_t hr = static_cast<size_t>(h) * a.tq_pad + row;
+    if (lane == 0) {
+      dvec[hr] = acc[i];
+      qcount[hr] = 0u;
+    }
+    float4* z = reinterpret_cast<float4*>(dqacc + hr * D);
+    for (int c = lane; c < D / 4; c += 32) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  float4* z = reinterpret_cast<float4*>(dqacc + (static_cast<size_t>(h) * a.tq_pad + row) * D);
-  for (int i = lane; i < D / 4; i += 32) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-// dQ[r, h, :] = bf16(scale * dQacc[h, r, :]). One warp per (row, head).
+// dQ[r, h, :] = bf16(scale * dQacc[h, r, :]).
 template <int D>
 __global__ void __launch_bounds__(256) bwd_convert_kernel(const BwdArgs a) {
-  const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  constexpr int E = D / 32;  // fp32 elements per lane: 4 (16 bytes) or 2 (8 bytes)
+  using F = typename std::conditional<E == 4, float4, float2>::type;
+  const long long units = static_cast<long long>(a.total_q) * a.H;
+  const long long u0 = ((static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5) * kUnits;
   const int lane = threadIdx.x & 31;
-  if (w >= static_cast<long long>(a.total_q) * a.H) return;
-  const int row = static_cast<int>(w / a.H), h = static_cast<int>(w % a.H);
-  const float* src = reinterpret_cast<const float*>(static_cast<const char*>(a.workspace) + a.dqacc_offset) +
-                     (static_cast<size_t>(h) * a.tq_pad + row) * D;
-  __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.dq) + static_cast<size_t>(w) * D;
-  constexpr int E = D / 32;
-  if constexpr (E == 4) {
-    const float4 v = reinterpret_cast<const float4*>(src)[lane];
-    uint2 o;
-    o.x = pack_bf16x2(v.x * a.scale, v.y * a.scale);
-    o.y = pack_bf16x2(v.z * a.scale, v.w * a.scale);
-    reinterpret_cast<uint2*>(dst)[lane] = o;
-  } else {
-    const float2 v = reinterpret_cast<const float2*>(src)[lane];
-    reinterpret_cast<uint32_t*>(dst)[lane] = pack_bf16x2(v.x * a.scale, v.y * a.scale);
+  if (u0 >= units) return;
+  const float* acc = reinterpret_cast<const float*>(static_cast<const char*>(a.workspace) + a.dqacc_offset);
+  F v[kUnits];
+#pragma unroll
+  for (int i = 0; i < kUnits; ++i) {
+    const long long u = u0 + i;
+    if (u < units) {
+      const int row = static_cast<int>(u / a.H), h = static_cast<int>(u % a.H);
+      v[i] = reinterpret_cast<const F*>(acc + (static_cast<size_t>(h) * a.tq_pad + row) * D)[lane];
+    } else {
+      v[i] = F{};
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kUnits; ++i) {
+    const long long u = u0 + i;
+    if (u >= units) break;
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.dq) + u * D;
+    if constexpr (E == 4) {
+      uint2 o;
+      o.x = pack_bf16x2(v[i].x * a.scale, v[i].y * a.scale);
+      o.y = pack_bf16x2(v[i].z * a.scale, v[i].w * a.scale);
+      reinterpret_cast<uint2*>(dst)[lane] = o;
+    } else {
+      reinterpret_cast<uint32_t*>(dst)[lane] = pack_bf16x2(v[i].x * a.scale, v[i].y * a.scale);
+    }
   }
 }
 
@@ -747,7 +782,7 @@ cudaError_t launch_main(const BwdArgs& a, const BwdMaps& m, cudaStream_t stream)
 }  // namespace
 
 cudaError_t launch_bwd_preprocess(const BwdArgs& a, cudaStream_t stream) {
-  const long long warps = static_cast<long long>(a.total_q) * a.H;
+  const long long warps = (static_cast<long long>(a.total_q) * a.H + kUnits - 1) / kUnits;
   const unsigned blocks = static_cast<unsigned>((warps + 7) / 8);
   if (blocks == 0) return cudaSuccess;
   if (a.D == 64)
@@ -769,7 +804,7 @@ cudaError_t launch_bwd_main(const BwdArgs& a, const BwdMaps& m, cudaStream_t str
 }
 
 cudaError_t launch_bwd_convert(const BwdArgs& a, cudaStream_t stream) {
-  const long long warps = static_cast<long long>(a.total_q) * a.H;
+  const long long warps = (static_cast<long long>(a.total_q) * a.H + kUnits - 1) / kUnits;
   const unsigned blocks = static_cast<unsigned>((warps + 7) / 8);
   if (blocks == 0) return cudaSuccess;
   if (a.D == 64)
