@@ -265,18 +265,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       for (;;) {
-        const int slot = ni % kItemSlots;
-        if (ni >= kItemSlots && !wait_bar(&bars.items.empty[slot], ((ni / kItemSlots) - 1) & 1, ab)) goto producer_done;
-        int idx = static_cast<int>(atomicAdd(&hdr->work_counter, 1u));
-        if (idx >= n_items) idx = -1;
+        int idx;
         Item it;
-        if (idx >= 0) {
-          it = get_item(a, pairs, idx);
+        auto decode = [&](int slot, int v) {
+          it = get_item(a, pairs, v);
           bars.item_data[slot] = it;
-        }
-        *reinterpret_cast<volatile int*>(&bars.items.idx[slot]) = idx;
-        mbar_arrive(&bars.items.full[slot]);
-        ++ni;
+        };
+        if (!publish_item_decoded(bars.items, ni, &hdr->work_counter, n_items, idx, ab, decode)) goto producer_done;
         if (idx < 0) break;
         if (it.n == 0) continue;
         const int krow = it.s.k0 + it.j * BN;

@@ -284,6 +284,25 @@ __device__ __forceinline__ bool publish_item(ItemRing& r, uint32_t& n, uint32_t*
   return true;
 }
 
+// Publisher that also decodes each claimed item once for all roles: for a
+// claimed index, `decode(slot, idx)` stores the decoded item beside the ring
+// before it is published (the mbarrier arrive orders those writes before the
+// consumers' wait), and consumers copy it out before releasing the slot.
+template <typename Decode>
+__device__ __forceinline__ bool publish_item_decoded(ItemRing& r, uint32_t& n, uint32_t* counter, int n_items,
+                                                     int& idx, const Abort& ab, Decode&& decode) {
+  const int slot = n % kItemSlots;
+  if (n >= kItemSlots && !wait_bar(&r.empty[slot], ((n / kItemSlots) - 1) & 1, ab)) return false;
+  int v = static_cast<int>(atomicAdd(counter, 1u));
+  if (v >= n_items) v = -1;
+  if (v >= 0) decode(slot, v);
+  *reinterpret_cast<volatile int*>(&r.idx[slot]) = v;
+  mbar_arrive(&r.full[slot]);
+  ++n;
+  idx = v;
+  return true;
+}
+
 // Consumer: wait for the n-th published item; returns its index, or -1 when
 // there is no more work (or the CTA is aborting). `slot` receives the ring
 // slot, on whose `empty` barrier the caller arrives once it has the index.

@@ -84,12 +84,25 @@ struct FwdSmem {
   static constexpr int kV = kK + kKStages * kTileBytes;     // V stage s at kV + s*tile
   static constexpr int kInvL = kV + kVStages * kTileBytes;  // fp32 [2][128]: 1/l per row
   static constexpr int kBar = kInvL + kQTiles * BM * 4;
-  static constexpr int kBytes = kBar + 512;
+  static constexpr int kBytes = kBar + 1024;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
   static constexpr int kSCol = 0;               // S of query tile w at columns w*BN
   static constexpr int kOCol = 2 * BN;          // O of query tile w at kOCol + w*D
 };
 static_assert(FwdSmem<128>::kAlloc <= 232448 && FwdSmem<64>::kAlloc <= 232448, "layout fits 227 KB");
+
+struct Item {
+  int b, h, t;  // t: 256-row block of the sequence
+  int hk;       // key/value head of query head h
+  SeqInfo s;
+  int nk[2];    // key tiles visible from query tile w (0 when the tile is empty)
+};
+
+// Decoded items travel through the item ring at head_dim 128 (the
+// producer decodes each item once and the other roles copy it); at head_dim
+// 64 every role decodes the index itself, which measured faster there.
+template <int D>
+constexpr bool kDecodedRing = D != 64;
 
 struct Bars {
   uint64_t q_full[2], q_empty[2];
@@ -99,17 +112,11 @@ struct Bars {
   uint64_t drain;
   uint64_t k_full[5], k_empty[5], v_full[5], v_empty[5];
   ItemRing items;
+  Item item_data[kItemSlots];  // the published items, decoded once by the producer
   uint32_t tmem_base;
   int abort_flag;
 };
-static_assert(sizeof(Bars) <= 512, "barrier block fits its reserved space");
-
-struct Item {
-  int b, h, t;  // t: 256-row block of the sequence
-  int hk;       // key/value head of query head h
-  SeqInfo s;
-  int nk[2];    // key tiles visible from query tile w (0 when the tile is empty)
-};
+static_assert(sizeof(Bars) <= 1024, "barrier block fits its reserved space");
 
 template <int KL>
 __device__ __forceinline__ Item get_item(const FwdArgs& a, const int2* pairs, int idx) {
@@ -143,9 +150,18 @@ __device__ __forceinline__ void qk_producer(const CUtensorMap* tm_q, const CUten
   uint32_t kc = 0, ni = 0, nq[2] = {0u, 0u};
   for (;;) {
     int idx;
-    if (!publish_item(bars.items, ni, &hdr->work_counter, n_items, idx, ab)) goto done;
+    Item it;
+    if constexpr (kDecodedRing<D>) {
+      auto decode = [&](int slot, int v) {
+        it = get_item<KL>(a, pairs, v);
+        bars.item_data[slot] = it;
+      };
+      if (!publish_item_decoded(bars.items, ni, &hdr->work_counter, n_items, idx, ab, decode)) goto done;
+    } else {
+      if (!publish_item(bars.items, ni, &hdr->work_counter, n_items, idx, ab)) goto done;
+      if (idx >= 0) it = get_item<KL>(a, pairs, idx);
+    }
     if (idx < 0) break;
-    const Item it = get_item<KL>(a, pairs, idx);
     const int nkb = max(it.nk[0], it.nk[1]);
     if (nkb == 0) continue;
 #pragma unroll
@@ -188,8 +204,8 @@ __device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, const FwdArg
     int slot;
     const int idx = consume_item<false>(bars.items, ni, slot, ab);
     if (idx < 0) break;
+    const Item it = kDecodedRing<D> ? bars.item_data[slot] : get_item<KL>(a, pairs, idx);
     mbar_arrive(&bars.items.empty[slot]);
-    const Item it = get_item<KL>(a, pairs, idx);
     const int nkb = max(it.nk[0], it.nk[1]);
     for (int j = 0; j < nkb; ++j, ++vc) {
       const int st = vc % NV;
@@ -244,9 +260,10 @@ __device__ __forceinline__ void mma_issuer(const FwdArgs& a, uint8_t* smem, Bars
     int slot;
     const int idx = consume_item<true>(bars.items, ni, slot, ab);
     if (idx < 0) break;
+    const Item it = kDecodedRing<D> ? bars.item_data[slot] : get_item<KL>(a, pairs, idx);
+    __syncwarp();
     if (elect_one()) mbar_arrive(&bars.items.empty[slot]);
     __syncwarp();
-    const Item it = get_item<KL>(a, pairs, idx);
     const int nkb = max(it.nk[0], it.nk[1]);
     if (nkb == 0) continue;
 #pragma unroll
@@ -340,9 +357,9 @@ __device__ __forceinline__ void softmax_role(const FwdArgs& a, uint8_t* smem, Ba
     int slot;
     const int idx = consume_item<true>(bars.items, ni, slot, ab);
     if (idx < 0) break;
+    const Item it = kDecodedRing<D> ? bars.item_data[slot] : get_item<KL>(a, pairs, idx);
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars.items.empty[slot]);
-    const Item it = get_item<KL>(a, pairs, idx);
     const int nk = it.nk[W];
     if (nk == 0) continue;  // the epilogue warpgroup writes empty rows
     const int tq = it.t * kQTiles + W;  // 128-row tile of the sequence
@@ -458,9 +475,9 @@ __device__ __forceinline__ void epilogue_role(const FwdArgs& a, uint8_t* smem, B
     int slot;
     const int idx = consume_item<true>(bars.items, ni, slot, ab);
     if (idx < 0) break;
+    const Item it = kDecodedRing<D> ? bars.item_data[slot] : get_item<KL>(a, pairs, idx);
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars.items.empty[slot]);
-    const Item it = get_item<KL>(a, pairs, idx);
 #pragma unroll
     for (int w = 0; w < 2; ++w) {
       const int r = (it.t * kQTiles + w) * BM + row;
