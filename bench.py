@@ -460,7 +460,7 @@ def decode_workloads(dev, stream, flush, hbm_peak_gbs, iters=10):
         v = torch.randn(batch * lk, Hk, D, device=dev, dtype=torch.bfloat16)
         cu_q = torch.arange(batch + 1, dtype=torch.int32, device=dev)
         cu_k = torch.arange(batch + 1, dtype=torch.int32, device=dev) * lk
-        splits = max(1, min(lk // 128, -(-2 * sms // (batch * Hk))))
+        splits = fa_varlen.fa_varlen_splitkv_num_splits(batch, 1, H, Hk, lk, sms)
         out = torch.empty_like(q)
         lse = torch.empty((H, batch), dtype=torch.float32, device=dev)
         ws = fa_varlen.new_workspace(int(fa_varlen.lib.fa_varlen_fwd_splitkv_workspace_size(batch, batch, H, Hk, D,

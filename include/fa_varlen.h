@@ -256,6 +256,20 @@ fa_status_t fa_varlen_fwd_splitkv(const void* q, const void* k, const void* v, c
                                   int causal, int num_splits, void* out, float* softmax_lse, void* workspace,
                                   size_t workspace_bytes, fa_cuda_stream_t stream);
 
+/* A split count for fa_varlen_fwd_splitkv (advisory; results do not depend
+ * on it). The work units of the split-KV forward are (sequence, key/value
+ * head, query tile, key range), taken by one persistent CTA per SM. This
+ * returns the smallest num_splits for which the units fill the SMs in
+ * nearly whole waves (at least 95% of the CTA-unit slots busy, the units
+ * being of equal size), keeping at least two 128-key tiles per range; if no
+ * count reaches that, the one with the best fill. A query tile holds
+ * 128 / (num_heads / num_heads_k) tokens of one sequence, so the unit count
+ * per range is taken as batch * num_heads_k * ceil(max_seqlen_q * group / 128).
+ * sm_count <= 0 uses the current device's SM count. Returns 1 for invalid
+ * arguments or when no device can be queried. Host only; no device work. */
+int fa_varlen_splitkv_num_splits(int batch, int max_seqlen_q, int num_heads, int num_heads_k, int max_seqlen_k,
+                                 int sm_count);
+
 /* Forward for callers that cannot allocate device memory. The pages have no
  * counterpart of this entry point; it exists for the library's users.
  *

@@ -154,3 +154,45 @@ def test_splitkv_rejects(lib):
     assert args(ctypes.byref(lay), 2, 256, 1) == 2
     assert lib.fa_varlen_fwd_splitkv_workspace_size(2, 64, 8, 3, 128, 2) == 0
     assert lib.fa_varlen_fwd_splitkv_workspace_size(2, 64, 8, 2, 128, 4) > 4 * 64 * 8 * 128 * 4
+
+
+def test_splitkv_num_splits(lib):
+    """The advisory split count: smallest count whose equal-sized units keep
+    at least 95% of the (SM x wave) slots busy, at least two 128-key tiles per
+    range, 1 for invalid arguments. Values worked by hand for 148 SMs."""
+    f = lib.fa_varlen_splitkv_num_splits
+    # 64 sequences x 8 kv heads = 512 units: 1 split fills 512/592 = 86%,
+    # 2 splits fill 1024/1036 = 98.8%.
+    assert f(64, 1, 32, 8, 8192, 148) == 2
+    # 4 x 8 = 32 units per split: 9 splits give 288 units in two waves
+    # (288/296 = 97.3%); 1..8 stay below 95%.
+    assert f(4, 1, 32, 8, 32768, 148) == 9
+    # A large batch already fills the SMs without splitting.
+    assert f(148 * 4, 1, 8, 8, 4096, 148) == 1
+    # Two key tiles per range at most: 300 keys = 3 tiles -> 1 split only.
+    assert f(1, 1, 8, 8, 300, 148) == 1
+    # Query tiles count: 64 tokens x group 4 = 2 tiles per sequence.
+    assert f(74, 64, 32, 8, 8192, 148) == f(148, 1, 32, 8, 8192, 148)
+    # Invalid arguments.
+    assert f(0, 1, 32, 8, 8192, 148) == 1
+    assert f(4, 1, 32, 7, 8192, 148) == 1
+    assert f(4, 1, 32, 8, 0, 148) == 1
+    # Exhaustive restatement over a grid of shapes.
+    for batch in (1, 3, 16):
+        for hk in (1, 2, 8):
+            for lk in (128, 1000, 20000):
+                for sms in (7, 148):
+                    per = batch * hk
+                    tiles = -(-lk // 128)
+                    cap = min(1024, max(1, tiles // 2))
+                    want, best = None, (0.0, 1)
+                    for s in range(1, cap + 1):
+                        u = per * s
+                        fill = u / (-(-u // sms) * sms)
+                        if fill >= 0.95:
+                            want = s
+                            break
+                        if fill > best[0]:
+                            best = (fill, s)
+                    assert f(batch, 1, hk, hk, lk, sms) == (want if want is not None else best[1])
+

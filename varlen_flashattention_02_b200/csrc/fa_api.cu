@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -295,6 +296,33 @@ bool kv_layout_ok(const fa_kv_layout_t* kv) {
 }  // namespace
 
 extern "C" {
+
+int fa_varlen_splitkv_num_splits(int batch, int max_seqlen_q, int num_heads, int num_heads_k, int max_seqlen_k,
+                                 int sm_count) {
+  if (batch <= 0 || max_seqlen_q <= 0 || num_heads <= 0 || num_heads_k <= 0 || num_heads % num_heads_k != 0 ||
+      max_seqlen_k <= 0)
+    return 1;
+  if (sm_count <= 0) sm_count = ::sm_count();
+  if (sm_count <= 0) return 1;
+  const long long group = num_heads / num_heads_k;
+  const long long q_tiles = (static_cast<long long>(max_seqlen_q) * group + 127) / 128;
+  const long long per_split = static_cast<long long>(batch) * num_heads_k * q_tiles;
+  const int k_tiles = (max_seqlen_k + 127) / 128;
+  const int max_splits = std::min(1024, std::max(1, k_tiles / 2));
+  int best = 1;
+  double best_fill = 0.0;
+  for (int s = 1; s <= max_splits; ++s) {
+    const long long units = per_split * s;
+    const long long slots = (units + sm_count - 1) / sm_count * sm_count;
+    const double fill = static_cast<double>(units) / static_cast<double>(slots);
+    if (fill >= 0.95) return s;
+    if (fill > best_fill) {
+      best_fill = fill;
+      best = s;
+    }
+  }
+  return best;
+}
 
 size_t fa_varlen_fwd_splitkv_workspace_size(int batch, int total_q, int num_heads, int num_heads_k, int head_dim,
                                             int num_splits) {

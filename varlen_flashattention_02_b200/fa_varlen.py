@@ -69,6 +69,8 @@ def _load():
     lib.fa_varlen_fwd_splitkv.argtypes = [P, P, P, P, ctypes.POINTER(KvLayout), I, I, I, I, I, I, I,
                                           ctypes.c_float, I, I, P, P, P, S, P]
     lib.fa_varlen_fwd_splitkv.restype = I
+    lib.fa_varlen_splitkv_num_splits.argtypes = [I, I, I, I, I, I]
+    lib.fa_varlen_splitkv_num_splits.restype = I
     lib.fa_varlen_fwd_kvcache.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, ctypes.c_float, I, P, P, P, S, P]
     lib.fa_varlen_fwd_kvcache.restype = I
     lib.fa_varlen_fwd_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, ctypes.c_float, I, P, P,
@@ -90,7 +92,7 @@ lib = _load()
 EXPORTED = ("fa_varlen_fwd_workspace_size", "fa_varlen_bwd_workspace_size", "fa_varlen_fwd",
             "fa_varlen_bwd", "fa_varlen_fwd_gqa", "fa_varlen_bwd_gqa", "fa_varlen_fwd_kvcache",
             "fa_varlen_fwd_paged", "fa_varlen_bwd_deterministic", "fa_varlen_fwd_splitkv",
-            "fa_varlen_fwd_splitkv_workspace_size", "fa_varlen_fwd_noalloc",
+            "fa_varlen_fwd_splitkv_workspace_size", "fa_varlen_splitkv_num_splits", "fa_varlen_fwd_noalloc",
             "fa_get_device_status", "fa_set_kernel_events", "fa_status_string")
 
 
@@ -335,6 +337,15 @@ def fa_varlen_fwd_paged(q, k_pages, v_pages, cu_seqlens_q, seqlens_k, block_tabl
     if rc != FA_OK:
         raise FaError(rc, "fa_varlen_fwd_paged")
     return out, softmax_lse
+
+
+def fa_varlen_splitkv_num_splits(batch: int, max_seqlen_q: int, num_heads: int, num_heads_k: int,
+                                 max_seqlen_k: int, sm_count: int = 0) -> int:
+    """Advisory split count for :func:`fa_varlen_fwd_splitkv` (same name in
+    the C ABI): the smallest count whose work units fill the SMs in nearly
+    whole waves. ``sm_count`` 0 queries the current device."""
+    return int(lib.fa_varlen_splitkv_num_splits(int(batch), int(max_seqlen_q), int(num_heads), int(num_heads_k),
+                                                int(max_seqlen_k), int(sm_count)))
 
 
 def fa_varlen_fwd_splitkv(q, k, v, cu_seqlens_q, max_seqlen_q: int, max_seqlen_k: int, softmax_scale: float,
