@@ -58,6 +58,32 @@ def max_over_ranks(x: float, device=None) -> float:
     return float(t.item())
 
 
+def head_range(heads: int, world: int, rank: int) -> tuple[int, int]:
+    """Heads [h0, h1) of rank ``rank`` when the heads of one problem are split
+    across ``world`` GPUs: contiguous, balanced (the first heads % world ranks
+    take one extra head). Every (sequence, head) unit is independent in both
+    directions, so the ranks exchange nothing; cu_seqlens is replicated."""
+    if world < 1 or not 0 <= rank < world or heads < world:
+        raise ValueError(f"cannot split {heads} heads over {world} ranks (rank {rank})")
+    base, extra = divmod(heads, world)
+    h0 = rank * base + min(rank, extra)
+    return h0, h0 + base + (1 if rank < extra else 0)
+
+
+def shard_heads(tensors: dict, h0: int, h1: int, kv_group: int = 1) -> dict:
+    """This rank's slice of packed [tokens, heads, d] arrays (bf16 bits):
+    query-side arrays (q, dout) take heads [h0, h1); key/value arrays take the
+    key/value heads those query heads read (h / kv_group). Contiguous copies,
+    so each slice is again a packed [tokens, h1 - h0, d] problem."""
+    if h0 % kv_group or h1 % kv_group:
+        raise ValueError("a rank's heads must cover whole key/value groups")
+    out = {}
+    for n, a in tensors.items():
+        lo, hi = (h0, h1) if n in ("q", "dout") else (h0 // kv_group, h1 // kv_group)
+        out[n] = np.ascontiguousarray(a[:, lo:hi, :])
+    return out
+
+
 def weak_scaling_value(world: int, flops_per_rank: float, max_ms_per_step: float) -> float:
     """Whole-job TFLOP/s: every rank did ``flops_per_rank`` per step; the job's
     step time is the slowest rank's."""
@@ -182,8 +208,18 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = bench_workload(args.tokens)
-    w.seed = w.seed + 1000 * rank  # same shape, own data per rank
-    t = w.tensors()
+    split_heads = args.split == "heads" and world > 1
+    heads_job = w.heads
+    if split_heads:
+        # One problem, its heads split across the ranks: every rank draws the
+        # same seeded batch and keeps its contiguous slice of heads.
+        F_job = fwd_flops(w.cu_q, w.cu_k, w.heads, w.head_dim, w.causal)
+        h0, h1 = head_range(w.heads, world, rank)
+        t = shard_heads(w.tensors(), h0, h1)
+        w.heads = h1 - h0
+    else:
+        w.seed = w.seed + 1000 * rank  # same shape, own data per rank
+        t = w.tensors()
     H, D = w.heads, w.head_dim
 
     def dev_bf16(bits):
@@ -274,9 +310,12 @@ def run_ours(args, rank, world, local_rank):
         "bwd_dq_convert": statistics.mean(evs[6].elapsed_time(evs[7]) for evs in bwd_ev),
     }
     tot_ms = max_over_ranks(sum(step_ms), dev)
-    F = fwd_flops(w.cu_q, w.cu_k, H, D, w.causal)
+    F = fwd_flops(w.cu_q, w.cu_k, H, D, w.causal)  # this rank's share
     ms_step = tot_ms / K
-    value = weak_scaling_value(world, 3.5 * F, ms_step)
+    if split_heads:
+        value = 3.5 * F_job / (ms_step * 1e-3) / 1e12  # the whole problem per slowest rank's step
+    else:
+        value = weak_scaling_value(world, 3.5 * F, ms_step)
 
     # ---- end to end through the public API with host buffers (pinned)
     host_in = {n: torch.from_numpy(t[n].view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -345,8 +384,9 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = max_over_ranks(e2e_ms, dev)
     if world > 1:
         dist.barrier()
+    e2e_value = (3.5 * F_job / (e2e_ms * 1e-3) / 1e12) if split_heads else weak_scaling_value(world, 3.5 * F, e2e_ms)
     e2e = None if not e2e_steps else {
-        "value": weak_scaling_value(world, 3.5 * F, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
         "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps,
         "pipelining": "step i+1's inputs copied in while step i computes; step i's gradients copied out "
                       "while step i+1 computes (copy streams, two device buffer sets)"}
@@ -364,13 +404,16 @@ def run_ours(args, rank, world, local_rank):
     fwd_k = statistics.mean(fwd_kern_ms)
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
-        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong" if split_heads else "weak",
+        "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded bf16 N(0,1); lengths from numpy default_rng)",
-        "config": {"workload": WORKLOAD, "total_tokens": w.total_q, "batch": w.batch, "heads": H,
+        "config": {"workload": WORKLOAD, "total_tokens": w.total_q, "batch": w.batch, "heads": heads_job,
                    "head_dim": D, "causal": True, "max_seqlen": w.max_seqlen_q,
                    "flops_fwd": F, "flop_convention": "fwd+bwd = 3.5 * F_fwd (bwd = 2.5 * F_fwd); causal halved",
                    "l2": "256 MiB buffer written between steps (and step inputs exceed L2)",
-                   "parallelism": f"weak: {world} independent replicas of the workload, no data-path collective"},
+                   "parallelism": (f"strong: heads split over {world} ranks (contiguous slices, cu_seqlens "
+                                   f"replicated, no data-path collective)" if split_heads else
+                                   f"weak: {world} independent replicas of the workload, no data-path collective")},
         "fwd_tflops": F / (statistics.mean(fwd_call_ms) * 1e-3) / 1e12,
         "bwd_tflops": 2.5 * F / (statistics.mean(bwd_call_ms) * 1e-3) / 1e12,
         "fwd_bwd_tflops_literal_2p5": weak_scaling_value(world, 2.5 * F, ms_step),
@@ -453,19 +496,19 @@ def decode_workloads(dev, stream, flush, hbm_peak_gbs, iters=10):
     res = {}
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     for batch, lk in ((64, 8192), (4, 32768)):
-        H, Hk, D = 32, 8, 128
-        rng = np.random.default_rng(9)
-        q = torch.from_numpy(synth.bf16_normal(rng, (batch, H, D)).view(np.int16)).view(torch.bfloat16).to(dev)
-        k = torch.randn(batch * lk, Hk, D, device=dev, dtype=torch.bfloat16)
-        v = torch.randn(batch * lk, Hk, D, device=dev, dtype=torch.bfloat16)
-        cu_q = torch.arange(batch + 1, dtype=torch.int32, device=dev)
-        cu_k = torch.arange(batch + 1, dtype=torch.int32, device=dev) * lk
+        # The same seeded inputs as the split-KV parity test at these shapes.
+        w = synth.decode_workload(batch, lk)
+        H, Hk, D = w.heads, w.kv_heads, w.head_dim
+        t = w.tensors()
+        q, k, v = (torch.from_numpy(t[n].view(np.int16)).view(torch.bfloat16).to(dev) for n in ("q", "k", "v"))
+        cu_q = torch.from_numpy(w.cu_q).to(dev)
+        cu_k = torch.from_numpy(w.cu_k).to(dev)
         splits = fa_varlen.fa_varlen_splitkv_num_splits(batch, 1, H, Hk, lk, sms)
         out = torch.empty_like(q)
         lse = torch.empty((H, batch), dtype=torch.float32, device=dev)
         ws = fa_varlen.new_workspace(int(fa_varlen.lib.fa_varlen_fwd_splitkv_workspace_size(batch, batch, H, Hk, D,
                                                                                            splits)), dev)
-        call = lambda: fa_varlen.fa_varlen_fwd_splitkv(q, k, v, cu_q, 1, lk, D ** -0.5, True, splits, cu_seqlens_k=cu_k,
+        call = lambda: fa_varlen.fa_varlen_fwd_splitkv(q, k, v, cu_q, 1, lk, w.scale, True, splits, cu_seqlens_k=cu_k,
                                                        out=out, softmax_lse=lse, workspace=ws, stream=stream)
         for _ in range(3):
             call()
@@ -583,6 +626,9 @@ def main():
     ap.add_argument("--no-aux", action="store_true", help="skip the forward-only workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--split", choices=("replicas", "heads"), default="replicas",
+                    help="N > 1: replicas = every rank runs the whole workload on its own data (weak scaling); "
+                         "heads = one workload, its heads split across the ranks (strong scaling)")
     ap.add_argument("--tokens", type=int, default=synth.TOTAL_TOKENS,
                     help="total tokens of the workload (default 16384; smaller only for profiling captures)")
     args = ap.parse_args()

@@ -41,9 +41,17 @@
  *                      non-decreasing, cu[batch] = total_q / total_k.
  * Element (row, h, c) of a packed tensor is at (row*num_heads + h)*head_dim + c.
  *
- * Supported: head_dim 64 or 128 (anything else returns FA_ERR_UNSUPPORTED;
- * there is no fallback path). q, k, v, out, dout, dq, dk, dv must be 16-byte
- * aligned. softmax_scale must be finite and > 0.
+ * Supported head dimensions (anything else returns FA_ERR_UNSUPPORTED;
+ * there is no fallback path):
+ *   - 64 and 128 on every entry point;
+ *   - 256 on the forwards (fa_varlen_fwd, _gqa, _kvcache, _paged, _noalloc)
+ *     and the backwards (fa_varlen_bwd, _gqa, _deterministic); the split-KV
+ *     forward (fa_varlen_fwd_splitkv) refuses it.
+ * The page "Flash-Atención y Flash-Atención-2" (FlashAttention-2 section)
+ * gives head dimensions "up to 256"; this library reads that as the three
+ * powers of two 64, 128 and 256 that tile into whole 64-column (128-byte)
+ * swizzled chunks. q, k, v, out, dout, dq, dk, dv must be 16-byte aligned.
+ * softmax_scale must be finite and > 0.
  *
  * Ownership and synchrony. The caller owns every buffer, including the
  * workspace (size from the *_workspace_size functions, any 256-byte-aligned
@@ -74,7 +82,7 @@ typedef struct CUstream_st* fa_cuda_stream_t;
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARGUMENT = 1, /* null pointer, negative size, bad scale, misaligned pointer */
-  FA_ERR_UNSUPPORTED = 2,      /* head_dim not in {64, 128}, or sizes beyond the limits below */
+  FA_ERR_UNSUPPORTED = 2,      /* head_dim not supported by the entry point, or sizes beyond the limits below */
   FA_ERR_WORKSPACE = 3,        /* workspace null, misaligned or smaller than required */
   FA_ERR_CUDA = 4,             /* a CUDA runtime call or launch failed */
   FA_ERR_BAD_SEQLENS = 5,      /* device: cu_seqlens not monotone, cu[0] != 0, cu[batch] != total,
@@ -263,8 +271,9 @@ fa_status_t fa_varlen_fwd_splitkv(const void* q, const void* k, const void* v, c
  * nearly whole waves (at least 95% of the CTA-unit slots busy, the units
  * being of equal size), keeping at least two 128-key tiles per range; if no
  * count reaches that, the one with the best fill. A query tile holds
- * 128 / (num_heads / num_heads_k) tokens of one sequence, so the unit count
- * per range is taken as batch * num_heads_k * ceil(max_seqlen_q * group / 128).
+ * tq = floor(128 / group) tokens of one sequence (group = num_heads /
+ * num_heads_k), so the unit count per range is taken as
+ * batch * num_heads_k * ceil(max_seqlen_q / tq).
  * sm_count <= 0 uses the current device's SM count. Returns 1 for invalid
  * arguments or when no device can be queried. Host only; no device work. */
 int fa_varlen_splitkv_num_splits(int batch, int max_seqlen_q, int num_heads, int num_heads_k, int max_seqlen_k,
@@ -283,10 +292,14 @@ int fa_varlen_splitkv_num_splits(int batch, int max_seqlen_q, int num_heads, int
  * every GPU loading the library holds until the process exits.
  *
  * - Returns FA_ERR_WORKSPACE, before any CUDA call, when the sizes need more
- *   scratch than that (fa_varlen_fwd_workspace_size(batch, total_q,
- *   num_heads, head_dim) > FA_NOALLOC_SCRATCH_BYTES; roughly
- *   total_q / 256 + 1.5 * batch must stay below about 32600).
- * - The first call on each device looks up the buffer's device address
+ *   scratch than that: fa_varlen_fwd_workspace_size(batch, total_q,
+ *   num_heads, head_dim) must not exceed FA_NOALLOC_SCRATCH_BYTES. That size
+ *   is about 256 + 4 * batch + 8 * (total_q / item_rows + batch) bytes,
+ *   item_rows being the query rows of one work item (256 for head_dim 64 and
+ *   128, 128 for head_dim 256), so total_q / item_rows + 1.5 * batch must
+ *   stay below about 32600.
+ * - The first call on each device (and the first after a device reset, which
+ *   creates a new context) looks up the buffer's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
  *   before any stream capture.
  * - All calls on a device share the one buffer, which keeps the last call's
@@ -315,6 +328,19 @@ fa_status_t fa_get_device_status(const void* workspace, fa_cuda_stream_t stream)
  * i < n_pairs. `events` holds cudaEvent_t handles created by the caller and
  * must stay valid while the hook is on. Pass NULL to turn it off. */
 void fa_set_kernel_events(void* const* events, int n_pairs);
+
+/* Test hook for the device-side failure detection; normal callers never need
+ * it. It applies to every later call made from the calling host thread.
+ * wait_limit_ns: the time after which every pipeline wait in the kernels
+ * gives up, records FA_ERR_DEVICE_TIMEOUT in the workspace status and makes
+ * the CTA stop (0 restores the default, 2 s). withhold_first_value_load != 0:
+ * the forward (fa_varlen_fwd, _gqa, _kvcache, _paged at head_dim 64 or 128)
+ * never issues the first value-tile load of its first work item and never
+ * posts that load's byte count, so the wait for it runs out; no load or MMA
+ * is left in flight, the call's outputs are undefined and the workspace
+ * status reads FA_ERR_DEVICE_TIMEOUT. The next call on the same workspace
+ * starts from a clean status. fa_set_test_hooks(0, 0) turns both off. */
+void fa_set_test_hooks(uint64_t wait_limit_ns, int withhold_first_value_load);
 
 /* Static, human-readable name of a status code. */
 const char* fa_status_string(fa_status_t status);

@@ -173,6 +173,15 @@ def test_splitkv_num_splits(lib):
     assert f(1, 1, 8, 8, 300, 148) == 1
     # Query tiles count: 64 tokens x group 4 = 2 tiles per sequence.
     assert f(74, 64, 32, 8, 8192, 148) == f(148, 1, 32, 8, 8192, 148)
+    # A group that does not divide 128: g = 3 packs floor(128/3) = 42 tokens
+    # per tile, so 128 tokens need 4 tiles (not ceil(3*128/128) = 3). With 2
+    # sequences x 8 kv heads that is 64 units per split; 9 splits fill
+    # 576/592 = 97.3% (3 tiles per sequence would have given 3 splits:
+    # 144/148). g = 6 packs 21 tokens: 64 tokens need 4 tiles, 3 sequences x
+    # 8 x 4 = 96 units, 3 splits fill 288/296 = 97.3%.
+    assert f(2, 128, 24, 8, 8192, 148) == 9
+    assert f(3, 64, 48, 8, 8192, 148) == 3
+    assert f(74, 42, 24, 8, 8192, 148) == f(74, 1, 24, 8, 8192, 148)  # 42 tokens: still one tile
     # Invalid arguments.
     assert f(0, 1, 32, 8, 8192, 148) == 1
     assert f(4, 1, 32, 7, 8192, 148) == 1

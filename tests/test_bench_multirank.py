@@ -55,3 +55,89 @@ def test_weak_scaling_value():
     # 2 ranks, 1e12 FLOP each per step, slowest step 2 ms -> 1000 TFLOP/s whole job.
     assert bench.weak_scaling_value(2, 1e12, 2.0) == pytest.approx(1000.0)
     assert bench.weak_scaling_value(1, 3.5e11, 1.0) == pytest.approx(350.0)
+
+
+def _head_split_worker(rank, world, port, out):
+    """One rank of a head-split problem: its slice of a small workload through
+    the oracle, then the slices gathered over gloo and reassembled on rank 0."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import bench
+    import oracle
+    from varlen_flashattention_02_b200 import synth
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = synth.make_workload("split", [70, 130, 1], [90, 130, 4], heads=6, head_dim=64, causal=True, seed=77)
+        h0, h1 = bench.head_range(w.heads, world, rank)
+        t = bench.shard_heads(w.tensors(), h0, h1)
+        o, l = oracle.fwd(t["q"], t["k"], t["v"], w.cu_q, w.cu_k, w.scale, True)
+        dq, dk, dv = oracle.bwd(t["q"], t["k"], t["v"], t["dout"], w.cu_q, w.cu_k, w.scale, True)
+        mine = [torch.from_numpy(np.ascontiguousarray(x)) for x in (o, l, dq, dk, dv)]
+        gathered = []
+        for x in mine:
+            parts = [torch.empty_like(x) for _ in range(world)]
+            dist.all_gather(parts, x)
+            gathered.append(parts)
+        if rank == 0:
+            full_o, full_l = oracle.fwd(*(w.tensors()[n] for n in ("q", "k", "v")), w.cu_q, w.cu_k, w.scale, True)
+            full_g = oracle.bwd(*(w.tensors()[n] for n in ("q", "k", "v", "dout")), w.cu_q, w.cu_k, w.scale, True)
+            # out, dq, dk, dv: [tokens, heads, d] -> concatenate along heads;
+            # lse: [heads, tokens] -> along its first axis.
+            ok = [np.array_equal(torch.cat(gathered[0], 1).numpy(), full_o),
+                  np.array_equal(torch.cat(gathered[1], 0).numpy(), full_l)]
+            ok += [np.array_equal(torch.cat(g, 1).numpy(), f) for g, f in zip(gathered[2:], full_g)]
+            out["ok"] = ok
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_head_split_reassembles_bitwise_gloo():
+    """Two gloo ranks split the heads of one problem (bench.py --split heads):
+    the per-rank results, gathered, equal the whole problem's bit for bit (no
+    exchange is needed because every (sequence, head) unit is independent)."""
+    import oracle
+
+    oracle.build()
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_head_split_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0
+    assert out["ok"] == [True] * 5
+
+
+def test_head_range():
+    import bench
+
+    assert [bench.head_range(16, 4, r) for r in range(4)] == [(0, 4), (4, 8), (8, 12), (12, 16)]
+    # Uneven: the first 16 % 3 = 1 rank takes one more head; the ranges tile [0, 16).
+    assert [bench.head_range(16, 3, r) for r in range(3)] == [(0, 6), (6, 11), (11, 16)]
+    assert bench.head_range(5, 1, 0) == (0, 5)
+    for bad in ((2, 4, 0), (16, 0, 0), (16, 2, 2)):
+        with pytest.raises(ValueError):
+            bench.head_range(*bad)
+
+
+def test_shard_heads_grouped():
+    import numpy as np
+
+    import bench
+
+    q = np.arange(3 * 8 * 2, dtype=np.uint16).reshape(3, 8, 2)
+    k = np.arange(3 * 2 * 2, dtype=np.uint16).reshape(3, 2, 2) + 1000
+    s = bench.shard_heads({"q": q, "k": k, "v": k, "dout": q}, 4, 8, kv_group=4)
+    assert np.array_equal(s["q"], q[:, 4:8]) and np.array_equal(s["k"], k[:, 1:2])
+    assert s["q"].flags.c_contiguous and s["k"].flags.c_contiguous
+    with pytest.raises(ValueError):
+        bench.shard_heads({"q": q}, 2, 6, kv_group=4)

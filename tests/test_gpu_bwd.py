@@ -67,8 +67,10 @@ def test_bwd_small(case, causal):
 def test_bwd_full_size_sampled(D):
     """The fwd+bwd workload (16384 tokens, lengths U{512..8192}, 16 heads,
     causal) at full size in the benchmark's launch configuration; whole
-    (sequence, head) units of the shortest sequences are checked against the
-    oracle and every gradient is checked to be finite."""
+    (sequence, head) units of the two shortest, the median and the longest
+    sequence (for this seed: all four, 685 to 6695 tokens; the longest key
+    tiles loop over the most query tiles) at the first and last head are
+    checked against the oracle, and every gradient is checked to be finite."""
     import torch
 
     w = synth.standard_workload(5)
@@ -77,8 +79,9 @@ def test_bwd_full_size_sampled(D):
                                 seed=w.seed)
     dq, dk, dv = _run_bwd(w)
     lens = np.diff(w.cu_q)
-    short = [int(b) for b in np.argsort(lens, kind="stable")[:2]]
-    units = [(b, h) for b in short for h in (0, w.heads - 1)]
+    order = [int(b) for b in np.argsort(lens, kind="stable")]
+    picked = sorted({order[0], order[1], order[len(order) // 2], order[-1]})
+    units = [(b, h) for b in picked for h in (0, w.heads - 1)]
     t = w.tensors()
     rq, rk, rv = oracle.bwd(t["q"], t["k"], t["v"], t["dout"], w.cu_q, w.cu_k, w.scale, w.causal, units=units)
     for b, h in units:

@@ -61,3 +61,35 @@ def test_bad_seqlens_reported(cu_q, cu_k, max_q):
     good = torch.tensor([0, 10, 20], dtype=torch.int32, device="cuda")
     fa_varlen.fa_varlen_fwd(q, k, v, good, good, 10, 10, 0.125, False, workspace=ws)
     assert fa_varlen.device_status(ws) == 0
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_device_timeout_reported(D):
+    """Failure detection on the device without any fault: with a 10 ms wait
+    limit and the test hook that withholds the first value-tile load of work
+    item 0, the MMA warp's bounded wait for that tile runs out; the CTA stops,
+    the workspace status reads FA_ERR_DEVICE_TIMEOUT, and the context stays
+    usable: the next ordinary call on the same workspace returns FA_OK with
+    parity."""
+    import torch
+
+    import oracle
+    from varlen_flashattention_02_b200 import fa_varlen
+
+    w = synth.make_workload("timeout", [700, 300, 129], heads=2, head_dim=D, causal=True, seed=61)
+    ws = fa_varlen.new_workspace(fa_varlen.fwd_workspace_size(w.batch, w.total_q, w.heads, w.head_dim), "cuda")
+    lib = fa_varlen.lib
+    lib.fa_set_test_hooks(10_000_000, 1)
+    try:
+        pu.run_fwd(w, workspace=ws)
+        assert fa_varlen.device_status(ws) == 6  # FA_ERR_DEVICE_TIMEOUT
+    finally:
+        lib.fa_set_test_hooks(0, 0)
+    (_, _, _), out, lse = pu.run_fwd(w, workspace=ws)
+    torch.cuda.synchronize()
+    assert fa_varlen.device_status(ws) == 0
+    t = w.tensors()
+    ro, rl = oracle.fwd(t["q"], t["k"], t["v"], w.cu_q, w.cu_k, w.scale, w.causal)
+    rows = np.repeat(np.arange(w.total_q), w.heads)
+    heads = np.tile(np.arange(w.heads), w.total_q)
+    pu.check_fwd(w, out, lse, ro, rl, rows, heads)

@@ -113,3 +113,22 @@ def test_splitkv_split_count_invariance():
     for o, l in outs[1:]:
         assert float((o.float() - outs[0][0].float()).abs().max()) < 1e-2
         assert float((l - outs[0][1]).abs().max()) < 1e-3
+
+
+@pytest.mark.parametrize("batch,keys,splits", [(64, 8192, 2), (4, 32768, 9)],
+                         ids=["64x8192-2splits", "4x32768-9splits"])
+def test_splitkv_decode_bench_shapes(batch, keys, splits):
+    """The benchmark's decode lines at full size, on the same seeded inputs:
+    one query token per sequence, 32 query heads over 8 key/value heads,
+    d=128, with the split counts the advisor picks for 148 SMs. Every output
+    row is compared with the oracle."""
+    from varlen_flashattention_02_b200 import fa_varlen
+
+    assert fa_varlen.fa_varlen_splitkv_num_splits(batch, 1, 32, 8, keys, 148) == splits
+    w = synth.decode_workload(batch, keys)
+    t = w.tensors()
+    q, k, v = (pu.to_dev(t[n]) for n in ("q", "k", "v"))
+    out, lse = fa_varlen.fa_varlen_fwd_splitkv(q, k, v, pu.cu_dev(w.cu_q), w.max_seqlen_q, w.max_seqlen_k, w.scale,
+                                               True, splits, cu_seqlens_k=pu.cu_dev(w.cu_k))
+    ref_out, ref_lse = oracle.fwd(t["q"], t["k"], t["v"], w.cu_q, w.cu_k, w.scale, True)
+    _check(t["q"], w.cu_q, out, lse, ref_out, ref_lse, w.heads, w.head_dim, True)

@@ -74,6 +74,14 @@ struct KernelEvents {
 };
 thread_local KernelEvents t_events;
 
+// Test hooks (per host thread): the wait limit of the kernels and the
+// withheld value load of fa_set_test_hooks.
+struct TestHooks {
+  uint64_t wait_ns = fa::kWaitTimeoutNs;
+  int withhold_v0 = 0;
+};
+thread_local TestHooks t_hooks;
+
 // Runs one launch, bracketed by the caller's timing events when the hook is on.
 template <class F>
 cudaError_t timed_launch(cudaStream_t stream, F&& launch) {
@@ -169,6 +177,8 @@ fa_status_t run_fwd(const void* q, const void* k, const void* v, const int32_t* 
   fa_args.causal = causal ? 1 : 0;
   fa_args.scale_log2 = softmax_scale * 1.4426950408889634f;
   fa_args.grid = static_cast<int>(items < sms ? items : sms);
+  fa_args.wait_ns = t_hooks.wait_ns;
+  fa_args.withhold_v0 = head_dim == 256 ? 0 : t_hooks.withhold_v0;
   auto launch = head_dim == 256 ? fa::launch_fwd_d256 : fa::launch_fwd;
   if (timed_launch(stream, [&] { return launch(fa_args, tq, tk, tv, stream); }) != cudaSuccess) return FA_ERR_CUDA;
   return FA_OK;
@@ -253,6 +263,7 @@ fa_status_t run_bwd(const void* dout, const void* q, const void* k, const void* 
   b.scale = softmax_scale;
   b.scale_log2 = softmax_scale * 1.4426950408889634f;
   b.grid = static_cast<int>(items < sms ? items : sms);
+  b.wait_ns = t_hooks.wait_ns;
   if (timed_launch(stream, [&] { return fa::launch_bwd_preprocess(b, stream); }) != cudaSuccess ||
       timed_launch(stream, [&] { return fa::launch_bwd_main(b, maps, stream); }) != cudaSuccess ||
       timed_launch(stream, [&] { return fa::launch_bwd_convert(b, stream); }) != cudaSuccess)
@@ -304,8 +315,12 @@ int fa_varlen_splitkv_num_splits(int batch, int max_seqlen_q, int num_heads, int
     return 1;
   if (sm_count <= 0) sm_count = ::sm_count();
   if (sm_count <= 0) return 1;
-  const long long group = num_heads / num_heads_k;
-  const long long q_tiles = (static_cast<long long>(max_seqlen_q) * group + 127) / 128;
+  const int group = num_heads / num_heads_k;
+  if (group > 128) return 1;
+  // A query tile holds tq = floor(128 / group) tokens of one sequence (the
+  // split-KV kernel's decomposition), so a sequence needs ceil(lq / tq) tiles.
+  const long long tq = 128 / group;
+  const long long q_tiles = (static_cast<long long>(max_seqlen_q) + tq - 1) / tq;
   const long long per_split = static_cast<long long>(batch) * num_heads_k * q_tiles;
   const int k_tiles = (max_seqlen_k + 127) / 128;
   const int max_splits = std::min(1024, std::max(1, k_tiles / 2));
@@ -393,6 +408,7 @@ fa_status_t fa_varlen_fwd_splitkv(const void* q, const void* k, const void* v, c
   d.causal = causal ? 1 : 0;
   d.scale_log2 = softmax_scale * 1.4426950408889634f;
   d.grid = static_cast<int>(items < sms ? items : sms);
+  d.wait_ns = t_hooks.wait_ns;
   if (timed_launch(stream, [&] { return fa::launch_decode(d, tq3, tk, tv, stream); }) != cudaSuccess ||
       timed_launch(stream, [&] { return fa::launch_decode_combine(d, stream); }) != cudaSuccess)
     return FA_ERR_CUDA;
@@ -507,6 +523,11 @@ fa_status_t fa_varlen_bwd_deterministic(const void* dout, const void* q, const v
   return run_bwd(dout, q, k, v, out, softmax_lse, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
                  max_seqlen_k, num_heads, num_heads_k, head_dim, softmax_scale, causal, dq, dk, dv, workspace,
                  workspace_bytes, stream, true);
+}
+
+void fa_set_test_hooks(uint64_t wait_limit_ns, int withhold_first_value_load) {
+  t_hooks.wait_ns = wait_limit_ns ? wait_limit_ns : fa::kWaitTimeoutNs;
+  t_hooks.withhold_v0 = withhold_first_value_load ? 1 : 0;
 }
 
 void fa_set_kernel_events(void* const* events, int n_pairs) {

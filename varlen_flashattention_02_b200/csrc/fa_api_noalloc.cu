@@ -12,9 +12,13 @@
 // caller-provided workspace.
 //
 // Host code cannot use the array's name as a device address (on the host it
-// is only a stand-in symbol). The address is looked up once per device with
-// cudaGetSymbolAddress, with that device current, on the first call made
-// while it is current, and cached.
+// is only a stand-in symbol). The address is looked up with
+// cudaGetSymbolAddress, with the device current, on the first call made on
+// each device, and cached together with the ID of the CUDA context it was
+// found in. A device reset (or any new primary context) reloads the module
+// and may move the array; the context then has a new ID, so the next call
+// looks the address up again instead of using a stale one.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -28,18 +32,49 @@ constexpr int kMaxDevices = 64;
 // Every GPU that loads the library holds this buffer until the process exits.
 static __device__ __align__(256) unsigned char g_fwd_scratch[FA_NOALLOC_SCRATCH_BYTES];
 
+struct Cached {
+  unsigned long long ctx_id;  // ID of the context the address belongs to (0: none yet)
+  void* addr;
+};
 std::mutex g_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
+Cached g_cache[kMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// ID of the calling thread's current context, or 0 if it cannot be told.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 // Device address of g_fwd_scratch on the current device (null on failure).
 void* scratch_on_current_device(int dev) {
   std::lock_guard<std::mutex> lock(g_mutex);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_fwd_scratch) != cudaSuccess) return nullptr;
-    g_scratch_addr[dev] = p;
-  }
-  return g_scratch_addr[dev];
+  const unsigned long long id = current_context_id();
+  if (id != 0 && g_cache[dev].ctx_id == id) return g_cache[dev].addr;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_fwd_scratch) != cudaSuccess) return nullptr;
+  // The lookup makes the device's primary context current if it was not.
+  g_cache[dev] = Cached{id != 0 ? id : current_context_id(), p};
+  return p;
 }
 
 }  // namespace

@@ -131,7 +131,7 @@ __device__ __forceinline__ bool wait_dq_turn(const uint32_t* cnt, uint32_t j, co
     for (int i = 0; i < 32; ++i)
       if (ld_acquire_gpu(cnt) >= j) return true;
     if (*ab.flag) return false;
-    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+    if (globaltimer_ns() - t0 > ab.limit_ns) {
       raise_abort(ab);
       return false;
     }
@@ -237,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
-  const Abort ab{&bars.abort_flag, &hdr->status};
+  const Abort ab{&bars.abort_flag, &hdr->status, a.wait_ns};
   const int n_items = (hdr->status == FA_OK) ? static_cast<int>(hdr->n_pairs) * a.Hk : 0;
 
   if (warp == 0) {

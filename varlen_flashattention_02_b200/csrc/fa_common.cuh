@@ -191,14 +191,16 @@ __host__ __device__ inline void bwd_q_tiles(int j, int lq, int lk, bool causal, 
 }
 
 // --------------------------------------------------------- bounded waits
-// Every pipeline wait gives up after this long, records
-// FA_ERR_DEVICE_TIMEOUT in the workspace status and raises the CTA's abort
-// flag so the other roles stop too.
+// Every pipeline wait gives up after a time limit (a kernel argument, this
+// long unless a test shortens it), records FA_ERR_DEVICE_TIMEOUT in the
+// workspace status and raises the CTA's abort flag so the other roles stop
+// too.
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
 
 struct Abort {
   volatile int* flag;  // shared memory, one per CTA
   uint32_t* status;    // workspace status word
+  uint64_t limit_ns;   // time limit of every wait
 };
 
 __device__ __forceinline__ void raise_abort(const Abort& ab) {
@@ -213,7 +215,7 @@ static __device__ __forceinline__ bool wait_slow(uint32_t addr, uint32_t parity,
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(addr, parity)) return true;
     if (*ab.flag) return false;
-    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+    if (globaltimer_ns() - t0 > ab.limit_ns) {
       raise_abort(ab);
       return false;
     }
@@ -237,7 +239,7 @@ __device__ __forceinline__ static bool wait_bar_final(uint64_t* bar, uint32_t pa
 #pragma unroll 1
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(addr, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+    if (globaltimer_ns() - t0 > ab.limit_ns) {
       raise_abort(ab);
       return false;
     }

@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
-  const Abort ab{&bars.abort_flag, &hdr->status};
+  const Abort ab{&bars.abort_flag, &hdr->status, a.wait_ns};
   const int n_items = (hdr->status == FA_OK) ? static_cast<int>(hdr->n_pairs) * a.Hk * a.splits : 0;
 
   if (warp == 0 && lane == 0) {

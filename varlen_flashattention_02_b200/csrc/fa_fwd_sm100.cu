@@ -200,6 +200,7 @@ __device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, const FwdArg
   using L = FwdSmem<D>;
   constexpr int NV = L::kVStages;
   uint32_t vc = 0, ni = 0;
+  uint32_t withheld = 0xffffffffu;  // test hook: the V load that was never issued
   for (;;) {
     int slot;
     const int idx = consume_item<false>(bars.items, ni, slot, ab);
@@ -212,6 +213,13 @@ __device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, const FwdArg
       const uint32_t use = vc / NV;
       const int vrow = KL == kKeysPaged ? key_tile_row(a.keys, it.b, it.s, j) : it.s.k0 + j * BN;
       if (use > 0 && !wait_bar(&bars.v_empty[st], (use - 1) & 1, ab)) goto done;
+      if (a.withhold_v0 && idx == 0 && j == 0) {
+        // Test hook: neither the load nor its expected bytes are posted, so
+        // the MMA warp's wait for this stage runs out (nothing is left in
+        // flight) and the CTA reports FA_ERR_DEVICE_TIMEOUT.
+        withheld = vc;
+        continue;
+      }
       mbar_arrive_expect_tx(&bars.v_full[st], L::kTileBytes);
       for (int c = 0; c < L::kChunks; ++c)
         tma_load_2d(tm_v, &bars.v_full[st], smem + L::kV + st * L::kTileBytes + c * kChunkBytes,
@@ -219,7 +227,8 @@ __device__ __forceinline__ void v_producer(const CUtensorMap* tm_v, const FwdArg
     }
   }
 done:
-  for (uint32_t i = (vc > NV ? vc - NV : 0); i < vc; ++i) wait_bar_final(&bars.v_full[i % NV], (i / NV) & 1, ab);
+  for (uint32_t i = (vc > NV ? vc - NV : 0); i < vc; ++i)
+    if (i != withheld) wait_bar_final(&bars.v_full[i % NV], (i / NV) & 1, ab);
 }
 
 // The MMA issuer. The whole warp runs this loop converged (all values
@@ -592,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
 
-  const Abort ab{&bars.abort_flag, &hdr->status};
+  const Abort ab{&bars.abort_flag, &hdr->status, a.wait_ns};
   const int n_items = (hdr->status == FA_OK) ? static_cast<int>(hdr->n_pairs) * a.H : 0;
 
   // Warpgroup index broadcast from lane 0 so that the compiler sees a

@@ -40,6 +40,8 @@ struct FwdArgs {
   int causal;
   float scale_log2;  // softmax_scale * log2(e)
   int grid;          // persistent CTAs
+  uint64_t wait_ns;  // time limit of every pipeline wait
+  int withhold_v0;   // test hook: the first V tile load of work item 0 is never issued
 };
 // tm_q: 2-D map over [rows, H*D] bf16; tm_k / tm_v over [rows, Hk*D]; box
 // 128 rows x 64 columns, 128-byte swizzle.
@@ -72,6 +74,7 @@ struct DecodeArgs {
   int causal;
   float scale_log2;
   int grid;
+  uint64_t wait_ns;  // time limit of every pipeline wait
 };
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tm_q3, const CUtensorMap& tm_k,
                           const CUtensorMap& tm_v, cudaStream_t stream);
@@ -96,6 +99,7 @@ struct BwdArgs {
   float scale;        // softmax_scale
   float scale_log2;   // softmax_scale * log2(e)
   int grid;
+  uint64_t wait_ns;   // time limit of every pipeline wait
 };
 // Backward in three launches: preprocess (rowsum(dO*O) and zero the dQ
 // accumulator), main, dQ conversion. Tensor maps, all bf16 with 128-byte

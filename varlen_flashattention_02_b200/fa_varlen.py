@@ -76,6 +76,8 @@ def _load():
     lib.fa_varlen_fwd_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, ctypes.c_float, I, P, P,
                                         P, S, P]
     lib.fa_varlen_fwd_paged.restype = I
+    lib.fa_set_test_hooks.argtypes = [ctypes.c_uint64, I]
+    lib.fa_set_test_hooks.restype = None
     lib.fa_get_device_status.argtypes = [P, P]
     lib.fa_get_device_status.restype = I
     lib.fa_varlen_fwd_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, ctypes.c_float, I, P, P, P]

@@ -128,6 +128,16 @@ def make_workload(name: str, lengths_q, lengths_k=None, heads=1, head_dim=64,
                     head_dim, float(scale), bool(causal), int(seed), with_grad, heads_k)
 
 
+def decode_workload(batch: int, keys: int, heads: int = 32, heads_k: int = 8, head_dim: int = 128,
+                    seed: int = 9) -> Workload:
+    """Token-by-token decoding: one query token per sequence against ``keys``
+    cached keys each (packed), grouped heads, causal (the single query is the
+    last position, so it sees every key). The split-KV benchmark lines and
+    their parity test use these inputs."""
+    return make_workload(f"decode-{batch}x{keys}-h{heads}-kv{heads_k}-d{head_dim}", [1] * batch, [keys] * batch,
+                         heads=heads, head_dim=head_dim, causal=True, seed=seed, heads_k=heads_k)
+
+
 def standard_workload(n: int, causal: bool | None = None, head_dim: int | None = None) -> Workload:
     """The five standard workloads, numbered 1..5.
 
