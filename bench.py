@@ -431,6 +431,7 @@ def run_ours(args, rank, world, local_rank):
     }
     if rank == 0 and not args.no_aux:
         result["fwd_by_workload"] = fwd_only_workloads(dev, stream, flush, peak)
+        result["bwd_by_workload"] = bwd_workloads(dev, stream, flush, peak)
         result["decode_by_workload"] = decode_workloads(dev, stream, flush, float(peaks["hbm_gbs"]))
     return result, w
 
@@ -481,6 +482,66 @@ def fwd_only_workloads(dev, stream, flush, peak, iters=10):
         F = fwd_flops(w.cu_q, w.cu_k, w.heads, w.head_dim, w.causal)
         res[name] = {"ms": ms, "tflops": F / (ms * 1e-3) / 1e12, "pct_of_peak": 100 * F / (ms * 1e-3) / 1e12 / peak}
         del q, k, v, out, lse, ws
+    return res
+
+
+def bwd_workloads(dev, stream, flush, peak, iters=10):
+    """Backward (and fwd+bwd) TFLOP/s of the fwd+bwd workload's lengths at the
+    other head dimensions and with grouped heads (same launch path as the
+    headline: the whole fa_varlen_bwd call, work list included)."""
+    import torch
+
+    from varlen_flashattention_02_b200 import fa_varlen
+
+    lens = synth.lengths_uniform(5, synth.TOTAL_TOKENS, 512, 8192)
+    specs = [("varlen-16k-U512..8192 (seed 5) h16 d64 causal",
+              lambda: synth.make_workload("d64", lens, heads=16, head_dim=64, causal=True, seed=5)),
+             ("grouped-query varlen-16k-U512..8192 (seed 5) h32 kv8 d128 causal",
+              lambda: synth.make_workload("gqa", lens, heads=32, head_dim=128, causal=True, seed=5, heads_k=8)),
+             ("varlen-16k-U512..8192 (seed 5) h16 d256 causal",
+              lambda: synth.make_workload("d256", lens, heads=16, head_dim=256, causal=True, seed=5))]
+    res = {}
+    for name, make in specs:
+        w = make()
+        t = w.tensors()
+        mk = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)
+        q, k, v, do = mk(t["q"]), mk(t["k"]), mk(t["v"]), mk(t["dout"])
+        cq, ck = torch.from_numpy(w.cu_q).to(dev), torch.from_numpy(w.cu_k).to(dev)
+        out = torch.empty_like(q)
+        lse = torch.empty((w.heads, w.total_q), dtype=torch.float32, device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        wsf = fa_varlen.new_workspace(fa_varlen.fwd_workspace_size(w.batch, w.total_q, w.heads, w.head_dim), dev)
+        wsb = fa_varlen.new_workspace(
+            fa_varlen.bwd_workspace_size(w.batch, w.total_q, w.total_k, w.heads, w.head_dim), dev)
+        fwd_fn = fa_varlen.fa_varlen_fwd_gqa if w.kv_heads != w.heads else fa_varlen.fa_varlen_fwd
+        bwd_fn = fa_varlen.fa_varlen_bwd_gqa if w.kv_heads != w.heads else fa_varlen.fa_varlen_bwd
+        fwd = lambda: fwd_fn(q, k, v, cq, ck, w.max_seqlen_q, w.max_seqlen_k, w.scale, True, out=out,
+                             softmax_lse=lse, workspace=wsf, stream=stream)
+        bwd = lambda: bwd_fn(do, q, k, v, out, lse, cq, ck, w.max_seqlen_q, w.max_seqlen_k, w.scale, True, dq=dq,
+                             dk=dk, dv=dv, workspace=wsb, stream=stream)
+        for _ in range(3):
+            fwd()
+            bwd()
+        tf, tb = [], []
+        for _ in range(iters):
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            flush.zero_()
+            evs[0].record(stream)
+            fwd()
+            evs[1].record(stream)
+            bwd()
+            evs[2].record(stream)
+            torch.cuda.synchronize(dev)
+            tf.append(evs[0].elapsed_time(evs[1]))
+            tb.append(evs[1].elapsed_time(evs[2]))
+        if fa_varlen.device_status(wsf) != 0 or fa_varlen.device_status(wsb) != 0:
+            raise RuntimeError(f"device status not OK in {name}")
+        F = fwd_flops(w.cu_q, w.cu_k, w.heads, w.head_dim, True)
+        ms_f, ms_b = statistics.mean(tf), statistics.mean(tb)
+        res[name] = {"fwd_ms": ms_f, "bwd_ms": ms_b, "bwd_tflops": 2.5 * F / (ms_b * 1e-3) / 1e12,
+                     "bwd_pct_of_peak": 100 * 2.5 * F / (ms_b * 1e-3) / 1e12 / peak,
+                     "fwd_bwd_tflops": 3.5 * F / ((ms_f + ms_b) * 1e-3) / 1e12}
+        del q, k, v, do, out, lse, dq, dk, dv, wsf, wsb
     return res
 
 
@@ -617,6 +678,23 @@ def run_reference(args):
     }
 
 
+def summary(r):
+    """The line's key figures again, compact, at its end: headline, forward
+    and backward of the headline workload, each other workload's % of peak."""
+    pct = lambda x: round(x, 1)
+    out = {"fwd_bwd_tflops": round(r["value"], 1), "pct_of_peak": {k: pct(v) for k, v in r["pct_of_peak"].items()
+                                                                   if k != "denominator"},
+           "kernel_ms": {k: round(v, 4) for k, v in r["kernel_ms"].items()},
+           "bwd_kernel_frac": round(r["roofline"]["frac"], 4)}
+    if "fwd_by_workload" in r:
+        out["fwd_pct_by_workload"] = {k: pct(v["pct_of_peak"]) for k, v in r["fwd_by_workload"].items()}
+    if "bwd_by_workload" in r:
+        out["bwd_pct_by_workload"] = {k: pct(v["bwd_pct_of_peak"]) for k, v in r["bwd_by_workload"].items()}
+    if "decode_by_workload" in r:
+        out["decode_pct_of_hbm"] = {k: pct(v["pct_of_hbm_peak"]) for k, v in r["decode_by_workload"].items()}
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -662,6 +740,7 @@ def main():
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline:
                 result["cpu_baseline"] = cpu_baseline(w)
+            result["summary"] = summary(result)
             print(json.dumps(result), flush=True)
     finally:
         if world > 1:

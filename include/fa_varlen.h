@@ -114,7 +114,9 @@ fa_status_t fa_varlen_fwd(const void* q, const void* k, const void* v, const int
  * Recomputes the probabilities from softmax_lse; writes dq, dk, dv.
  * The query gradient is accumulated with fp32 atomic reductions, so dq may
  * differ in the last bits between runs (fa_varlen_bwd_deterministic does
- * not). */
+ * not). head_dim 64, 128 or 256; at 256 the work runs as two passes over
+ * the same work list (dv first, then dk and dq), which the caller does not
+ * see: the arguments, workspace size and results are the same. */
 fa_status_t fa_varlen_bwd(const void* dout, const void* q, const void* k, const void* v, const void* out,
                           const float* softmax_lse, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
                           int batch, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int num_heads,
@@ -151,7 +153,7 @@ fa_status_t fa_varlen_bwd_gqa(const void* dout, const void* q, const void* k, co
 /* Deterministic backward (same arguments and results as fa_varlen_bwd_gqa).
  * The page "Flash-Atención y Flash-Atención-2" (backward paragraph) has the
  * column workers aggregate the query gradient with atomic additions, whose
- * order, and so whose rounding, changes from run to run. Here every 64-row
+ * order, and so whose rounding, changes from run to run. Here every 128-row
  * query tile receives its dQ contributions in key-tile order: key tile j
  * waits (on a per-tile counter in the workspace) until key tiles 0 .. j-1
  * have added theirs. dq, dk and dv are then bitwise identical from run to
@@ -251,7 +253,8 @@ typedef struct {
  *    128-row tile, so each key/value tile is read once per group;
  *  - each tile's key tiles are divided into num_splits ranges processed in
  *    parallel; each writes a normalised partial output and its logsumexp
- *    into the workspace (fp32) and a combine kernel merges them
+ *    into the workspace (fp32), and the CTA that finishes a tile's last
+ *    range merges them, counting finished ranges in the workspace
  *    (num_splits = 1 writes out directly).
  * head_dim 64 or 128 (FA_ERR_UNSUPPORTED otherwise). The workspace must
  * hold fa_varlen_fwd_splitkv_workspace_size(...) bytes (0 = invalid sizes).

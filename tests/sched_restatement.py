@@ -12,7 +12,7 @@ from __future__ import annotations
 
 FWD_BM = FWD_BN = 128
 FWD_ITEM_ROWS = 256
-BWD_BN, BWD_BM = 128, 64
+BWD_BN, BWD_BM = 128, 128
 HEADER = 256
 BINS = 2048
 

@@ -63,7 +63,7 @@ def _fwd(lib, **over):
 
 
 @pytest.mark.parametrize("over,code", [
-    (dict(D=96), 2), (dict(D=192), 2), (dict(D=512), 2), (dict(batch=0), 1), (dict(H=0), 1), (dict(total_q=-1), 1),
+    (dict(D=96), 2), (dict(D=192), 2), (dict(D=512), 2), (dict(D=256, ws_bytes=64), 3), (dict(batch=0), 1), (dict(H=0), 1), (dict(total_q=-1), 1),
     (dict(scale=0.0), 1), (dict(scale=float("inf")), 1), (dict(scale=-1.0), 1), (dict(q=None), 1),
     (dict(cu_q=None), 1), (dict(q=FAKE + 8), 1), (dict(out=FAKE + 2), 1), (dict(ws=None), 3),
     (dict(ws=FAKE + 16), 3), (dict(ws_bytes=64), 3),
@@ -83,7 +83,7 @@ def _bwd(lib, **over):
 
 
 @pytest.mark.parametrize("over,code", [
-    (dict(D=32), 2), (dict(D=256), 2), (dict(batch=-3), 1), (dict(scale=float("nan")), 1), (dict(do=None), 1), (dict(dk=None), 1),
+    (dict(D=32), 2), (dict(D=192), 2), (dict(D=256, ws_bytes=1024), 3), (dict(batch=-3), 1), (dict(scale=float("nan")), 1), (dict(do=None), 1), (dict(dk=None), 1),
     (dict(dv=FAKE + 4), 1), (dict(ws_bytes=1024), 3),
 ], ids=lambda x: str(x))
 def test_bwd_rejects(lib, over, code):
@@ -152,6 +152,10 @@ def test_splitkv_rejects(lib):
     assert args(None, 2, 8, 1) == 1
     assert args(ctypes.byref(lay), 0, 8, 1) == 1
     assert args(ctypes.byref(lay), 2, 256, 1) == 2
+    # head_dim 256 is refused by the split-KV forward (the other forwards and
+    # the backwards accept it).
+    assert lib.fa_varlen_fwd_splitkv(FAKE, FAKE, FAKE, FAKE, ctypes.byref(lay), 2, 64, 32, 32, 8, 1, 256, 0.1, 1, 2,
+                                     FAKE, FAKE, FAKE, 1 << 20, None) == 2
     assert lib.fa_varlen_fwd_splitkv_workspace_size(2, 64, 8, 3, 128, 2) == 0
     assert lib.fa_varlen_fwd_splitkv_workspace_size(2, 64, 8, 2, 128, 4) > 4 * 64 * 8 * 128 * 4
 

@@ -132,3 +132,26 @@ def test_splitkv_decode_bench_shapes(batch, keys, splits):
                                                True, splits, cu_seqlens_k=pu.cu_dev(w.cu_k))
     ref_out, ref_lse = oracle.fwd(t["q"], t["k"], t["v"], w.cu_q, w.cu_k, w.scale, True)
     _check(t["q"], w.cu_q, out, lse, ref_out, ref_lse, w.heads, w.head_dim, True)
+
+
+def test_splitkv_workspace_reused():
+    """The CTA that finishes a unit's last split merges the partials, counted
+    in the workspace; the work-list kernel zeroes the counts at every call, so
+    calls that reuse one workspace (different inputs, different split counts)
+    each match the oracle."""
+    import torch
+
+    from varlen_flashattention_02_b200 import fa_varlen
+
+    lq, lk, H, Hk, D = [1, 2, 1], [3000, 777, 4096], 16, 4, 128
+    ws = fa_varlen.new_workspace(int(fa_varlen.lib.fa_varlen_fwd_splitkv_workspace_size(3, 4, H, Hk, D, 8)), "cuda")
+    for seed, splits in ((851, 8), (852, 3), (853, 8)):
+        w = synth.make_workload("reuse", lq, lk, heads=H, head_dim=D, causal=True, seed=seed, heads_k=Hk)
+        t = w.tensors()
+        q, k, v = (pu.to_dev(t[n]) for n in ("q", "k", "v"))
+        out, lse = fa_varlen.fa_varlen_fwd_splitkv(q, k, v, pu.cu_dev(w.cu_q), w.max_seqlen_q, w.max_seqlen_k,
+                                                   w.scale, True, splits, cu_seqlens_k=pu.cu_dev(w.cu_k),
+                                                   workspace=ws)
+        torch.cuda.synchronize()
+        ref_out, ref_lse = oracle.fwd(t["q"], t["k"], t["v"], w.cu_q, w.cu_k, w.scale, True)
+        _check(t["q"], w.cu_q, out, lse, ref_out, ref_lse, H, D, True)

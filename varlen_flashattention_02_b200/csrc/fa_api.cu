@@ -194,7 +194,6 @@ fa_status_t run_bwd(const void* dout, const void* q, const void* k, const void* 
   fa_status_t st = check_sizes(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, num_heads, num_heads_k,
                                head_dim, softmax_scale);
   if (st != FA_OK) return st;
-  if (head_dim == 256) return FA_ERR_UNSUPPORTED;  // the backward supports head_dim 64 and 128
   if (!cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARGUMENT;
   if (total_q > 0 && (!q || !dout || !out || !softmax_lse || !dq || !aligned16(q) || !aligned16(dout) ||
                       !aligned16(out) || !aligned16(dq)))
@@ -229,10 +228,21 @@ fa_status_t run_bwd(const void* dout, const void* q, const void* k, const void* 
   // dk / dv maps serve only stores of key tiles, which exist only when total_k > 0.
   const void* dkp = total_k > 0 ? dk : anyp;
   const void* dvp = total_k > 0 ? dv : anyp;
-  if (!encode_map(&maps.q, qp, qrows, qcols, fa::kBwdBM) || !encode_map(&maps.dout, dop, qrows, qcols, fa::kBwdBM) ||
-      !encode_map(&maps.k, kp, krows, kcols, fa::kBwdBN) || !encode_map(&maps.v, vp, krows, kcols, fa::kBwdBN) ||
-      !encode_map(&maps.dk, dkp, krows, kcols, fa::kBwdBN) || !encode_map(&maps.dv, dvp, krows, kcols, fa::kBwdBN))
+  // head_dim 256 runs a dV pass over 128-row query tiles and a dK/dQ pass
+  // over 64-row query tiles (fa_bwd_d256_sm100.cu); its dK/dV leave as rows.
+  fa::BwdMapsD256 maps256;
+  if (head_dim == 256) {
+    if (!encode_map(&maps256.q128, qp, qrows, qcols, 128) || !encode_map(&maps256.do128, dop, qrows, qcols, 128) ||
+        !encode_map(&maps256.q64, qp, qrows, qcols, 64) || !encode_map(&maps256.do64, dop, qrows, qcols, 64) ||
+        !encode_map(&maps256.k, kp, krows, kcols, fa::kBwdBN) || !encode_map(&maps256.v, vp, krows, kcols, fa::kBwdBN))
+      return FA_ERR_CUDA;
+  } else if (!encode_map(&maps.q, qp, qrows, qcols, fa::kBwdBM) ||
+             !encode_map(&maps.dout, dop, qrows, qcols, fa::kBwdBM) ||
+             !encode_map(&maps.k, kp, krows, kcols, fa::kBwdBN) || !encode_map(&maps.v, vp, krows, kcols, fa::kBwdBN) ||
+             !encode_map(&maps.dk, dkp, krows, kcols, fa::kBwdBN) ||
+             !encode_map(&maps.dv, dvp, krows, kcols, fa::kBwdBN)) {
     return FA_ERR_CUDA;
+  }
 
   const int sms = sm_count();
   if (sms <= 0) return FA_ERR_CUDA;
@@ -265,16 +275,21 @@ fa_status_t run_bwd(const void* dout, const void* q, const void* k, const void* 
   b.grid = static_cast<int>(items < sms ? items : sms);
   b.wait_ns = t_hooks.wait_ns;
   if (timed_launch(stream, [&] { return fa::launch_bwd_preprocess(b, stream); }) != cudaSuccess ||
-      timed_launch(stream, [&] { return fa::launch_bwd_main(b, maps, stream); }) != cudaSuccess ||
+      timed_launch(stream,
+                   [&] {
+                     return head_dim == 256 ? fa::launch_bwd_d256(b, maps256, stream)
+                                            : fa::launch_bwd_main(b, maps, stream);
+                   }) != cudaSuccess ||
       timed_launch(stream, [&] { return fa::launch_bwd_convert(b, stream); }) != cudaSuccess)
     return FA_ERR_CUDA;
   return FA_OK;
 }
 
 // Workspace of the split-KV forward: header, per-sequence offsets and the
-// (sequence, token tile) list, then the split partials.
+// (sequence, token tile) list, then the split partials and, per (pair,
+// key/value head) unit, the count of its finished splits.
 struct DecodeLayout {
-  size_t seq_off, pairs, opart, lpart, total;
+  size_t seq_off, pairs, opart, lpart, done, total;
   int max_pairs, tq;
 };
 DecodeLayout decode_layout(int batch, int total_q, int H, int Hk, int D, int splits) {
@@ -292,6 +307,8 @@ DecodeLayout decode_layout(int batch, int total_q, int H, int Hk, int D, int spl
     off = fa::align_up(off + sizeof(float) * splits * rows * D, 256);
     L.lpart = off;
     off = fa::align_up(off + sizeof(float) * splits * rows, 256);
+    L.done = off;
+    off = fa::align_up(off + sizeof(uint32_t) * 4 * static_cast<size_t>(L.max_pairs) * Hk, 256);
   }
   L.total = off;
   return L;
@@ -371,6 +388,10 @@ fa_status_t fa_varlen_fwd_splitkv(const void* q, const void* k, const void* v, c
   t_events.next = 0;
   fa::SchedArgs sa{cu_seqlens_q, keys, batch, total_q, total_k, max_seqlen_q, max_seqlen_k,
                    causal ? 1 : 0, 0, L.tq, 0, workspace, L.seq_off, L.pairs, L.max_pairs};
+  if (num_splits > 1) {  // the split counters start every call at zero
+    sa.zero_words = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + L.done);
+    sa.n_zero = 4 * L.max_pairs * num_heads_k;  // one count per unit and 32-row quarter
+  }
   if (timed_launch(stream, [&] { return fa::launch_sched_prep(sa, stream); }) != cudaSuccess) return FA_ERR_CUDA;
   if (total_q == 0) return FA_OK;
 
@@ -396,6 +417,7 @@ fa_status_t fa_varlen_fwd_splitkv(const void* q, const void* k, const void* v, c
   char* ws = static_cast<char*>(workspace);
   d.opart = num_splits > 1 ? reinterpret_cast<float*>(ws + L.opart) : nullptr;
   d.lpart = num_splits > 1 ? reinterpret_cast<float*>(ws + L.lpart) : nullptr;
+  d.unit_done = num_splits > 1 ? reinterpret_cast<uint32_t*>(ws + L.done) : nullptr;
   d.workspace = workspace;
   d.pairs_offset = L.pairs;
   d.H = num_heads;
@@ -409,8 +431,7 @@ fa_status_t fa_varlen_fwd_splitkv(const void* q, const void* k, const void* v, c
   d.scale_log2 = softmax_scale * 1.4426950408889634f;
   d.grid = static_cast<int>(items < sms ? items : sms);
   d.wait_ns = t_hooks.wait_ns;
-  if (timed_launch(stream, [&] { return fa::launch_decode(d, tq3, tk, tv, stream); }) != cudaSuccess ||
-      timed_launch(stream, [&] { return fa::launch_decode_combine(d, stream); }) != cudaSuccess)
+  if (timed_launch(stream, [&] { return fa::launch_decode(d, tq3, tk, tv, stream); }) != cudaSuccess)
     return FA_ERR_CUDA;
   return FA_OK;
 }

@@ -1,4 +1,4 @@
-// fa_bwd_sm100.cu -- backward varlen attention for sm_100a.
+// fa_bwd_sm100.cu -- backward varlen attention for sm_100a (head_dim 64, 128).
 //
 // Three kernels per call, after the work-list preparation (key-tile mode):
 //  1. preprocess: Dv_i = sum_c dO_ic * O_ic (fp32, [H, rows]) and zero the
@@ -7,7 +7,7 @@
 //     key-tile) items, longest first, from a global counter. For 128 keys
 //     K_j, V_j of one key/value head it loops over the query heads that read
 //     that head (one, or a group under grouped-query attention) and the
-//     64-row query tiles that see the keys, recomputing the probabilities
+//     128-row query tiles that see the keys, recomputing the probabilities
 //     from the saved logsumexp instead of storing them:
 //        S^T  = K_j Q_i^T,  P^T = exp2(S^T*scale*log2e - lse_i*log2e)
 //        dP^T = V_j dO_i^T, dS^T = P^T * (dP^T - Dv_i)
@@ -26,15 +26,21 @@
 // sequence offsets and lengths from the cumulative arrays). The gradient
 // formulas are the chain rule of softmax attention (the pages print none).
 //
-// B200 design: persistent longest-first scheduling; warp specialisation
-// (warp 0 TMA, warp 1 MMA issue, warps 2-3 stage logsumexp/Dv rows,
-// warps 4-7 compute P^T and dS^T with one thread per key row, warps 8-11
-// drain dQ^T from TMEM into bulk fp32 reductions and write dK/dV); dK, dV
-// and the per-step S^T, dP^T tiles live in TMEM (S^T and dP^T double-
-// buffered so the next step's QK^T overlaps this step's softmax); P^T goes
-// back to TMEM as bf16 and feeds the dV MMA directly; dS^T is written once to
-// shared memory in a layout that serves both the dK MMA (K-major A) and the
-// dQ^T MMA (MN-major B).
+// B200 design. Each step works on 128 keys x 128 queries, so every MMA is
+// M = 128 with N = 128 (or N = head_dim): five groups of D/16 or 8 MMAs per
+// step. Warp roles (16 warps): warp 0 TMA loads and item claims, warp 1 MMA
+// issue, warps 2-3 stage logsumexp/Dv rows, two P/dS warpgroups (warps 4-7:
+// queries 0-63 of the step, warps 8-11: queries 64-127; one thread per key
+// row = TMEM lane), warps 12-15 drain dQ^T into bulk fp32 reductions and
+// write dK/dV. Tensor memory holds dK, dV, S^T and dP^T; P^T and dS^T are
+// written back over their S^T columns as bf16 so that both the dV and the dK
+// MMA read their A operand from TMEM; dS^T also goes to shared memory once,
+// as the B operand of dQ^T = K^T dS^T, whose result reuses the dP^T columns.
+// Once a step's MMAs have completed, its Q/dO stage (exactly the size of the
+// step's fp32 dQ tile) is the staging area of that step's dQ reduction, and
+// at an item's end of its dK/dV stores; the drain group then hands the stage
+// back to the loader. At head_dim 128 shared memory holds K, V, two Q/dO
+// stages and the dS^T tile: the whole 227 KB.
 #include <type_traits>
 
 #include "fa_common.cuh"
@@ -45,29 +51,37 @@ namespace {
 
 constexpr int BN = kBwdBN;  // keys per item
 constexpr int BM = kBwdBM;  // queries per step
-constexpr int kThreads = 384;
+static_assert(BN == 128 && BM == 128, "one 128 x 128 tile per step");
+constexpr int kThreads = 512;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kColDK = 0, kColDV = 128, kColS = 256, kColDP = 384;  // TMEM column map
+// TMEM column map: dK, dV (D columns each), S^T (P^T at +0/+64, dS^T at
+// +32/+96 as bf16 pairs, one 64-query half per P/dS warpgroup), dP^T (then
+// dQ^T: D lanes x 128 query columns).
+constexpr int kColDK = 0, kColDV = 128, kColS = 256, kColDP = 384;
+constexpr int kPdsWarp0 = 4, kDrainWarp0 = 12;
 
 template <int D>
 struct BwdSmem {
-  static constexpr int kQStages = 3;  // Q/dO stages (and logsumexp/Dv slots) in flight
+  static constexpr int kQStages = D == 64 ? 3 : 2;  // Q/dO stages (and logsumexp/Dv slots) in flight
   static constexpr int kChunks = D / 64;
   static constexpr int kKChunk = BN * 128;  // [128 rows x 64 bf16] swizzled chunk
-  static constexpr int kQChunk = BM * 128;  // [ 64 rows x 64 bf16]
+  static constexpr int kQChunk = BM * 128;
   static constexpr int kKTile = kChunks * kKChunk;
   static constexpr int kQTile = kChunks * kQChunk;
-  static constexpr int kDsTile = BN * BM * 2;  // dS^T [128 keys x 64 queries] bf16
+  static constexpr int kDsHalf = BN * 64 * 2;  // dS^T [128 keys x 64 queries] bf16, one swizzled chunk
+  static constexpr int kDsTile = 2 * kDsHalf;
   static constexpr int kK = 0;
   static constexpr int kV = kK + kKTile;
   static constexpr int kQdo = kV + kKTile;  // stage s: Q at kQdo + 2s*QTile, dO after it
   static constexpr int kDs = kQdo + 2 * kQStages * kQTile;
-  static constexpr int kStage = kDs + 2 * kDsTile;   // fp32 dQ [64 x D]
-  static constexpr int kLd = kStage + BM * D * 4;    // kQStages slots x (lse[64], dv[64]) fp32
+  static constexpr int kLd = kDs + kDsTile;  // slots x (lse[128], dv[128]) fp32
   static constexpr int kBar = kLd + kQStages * 2 * BM * 4;
   static constexpr int kBytes = kBar + 512;
-  static constexpr int kAlloc = kBytes + 1024;
 };
+static_assert(BwdSmem<128>::kBytes <= 232448 && BwdSmem<64>::kBytes <= 232448, "layout fits 227 KB");
+// A Q/dO stage holds a step's fp32 dQ tile (128 queries x D) and a key
+// tile's bf16 dV and dK (2 x 128 x D).
+static_assert(2 * BwdSmem<128>::kQTile == BM * 128 * 4 && 2 * BwdSmem<64>::kQTile == BM * 64 * 4, "stage");
 
 // An item is (sequence, key/value head hk, key tile j). Its steps visit the
 // query tiles i0 .. i0+nt-1 that see the key tile, for each query head of
@@ -99,10 +113,10 @@ __device__ __forceinline__ Item get_item(const BwdArgs& a, const int2* pairs, in
 struct Bars {
   uint64_t kv_full, kv_empty;
   uint64_t qdo_full[3], qdo_empty[3];
-  uint64_t st_full[2];
-  uint64_t ds_full[2], ds_empty[2];
-  uint64_t dq_full[2], dq_empty[2];
-  uint64_t dkv_full, dv_empty, dk_empty;
+  uint64_t s_full, dp_full;   // S^T, dP^T of the step in TMEM
+  uint64_t p_full, ds_full;   // P^T (TMEM), dS^T (TMEM and shared) written
+  uint64_t dq_full, dq_free;  // dQ^T in TMEM; read out by the drain group
+  uint64_t dkv_full, dv_free, dk_free;
   uint64_t ld_full[3], ld_empty[3];
   uint64_t drain;
   ItemRing items;
@@ -148,27 +162,21 @@ __device__ __forceinline__ uint4 pack8_bf16(const uint32_t* y, float scale) {
   return w;
 }
 
-// One row of D accumulator values to bf16 in global memory, times scale.
-template <int D>
-__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_t (&x)[D / 32][32], float scale) {
+// One 64-column chunk of a dK or dV row (TMEM values), times scale, as bf16:
+// either into row r of a 128-byte-swizzled [128 rows x 64 columns] TMA box
+// (the 16-byte unit u of a row sits at u ^ (r % 8), so the eight threads of
+// a store phase write eight different bank groups), or straight to global
+// memory (a row of a tile cut by the end of its sequence).
+__device__ __forceinline__ void chunk_to_box(uint8_t* box, const uint32_t (&x)[2][32], float scale, int r) {
+  uint8_t* row = box + r * 128;
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+    *reinterpret_cast<uint4*>(row + ((u ^ (r & 7)) << 4)) = pack8_bf16(x[u / 4] + 8 * (u % 4), scale);
+}
+__device__ __forceinline__ void chunk_to_global(__nv_bfloat16* dst, const uint32_t (&x)[2][32], float scale) {
   uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-  for (int e = 0; e < D / 8; ++e) d4[e] = pack8_bf16(x[e / 4] + 8 * (e % 4), scale);
-}
-
-// Row r of a [128 x D] bf16 tile into shared memory in the layout of the
-// 128-byte-swizzled TMA boxes (64 columns x 128 rows per box, box c at
-// c * 16 KB, 1024-byte aligned): the 16-byte unit u of a 128-byte row sits
-// at position u ^ (r % 8). The eight threads of a store phase therefore
-// write eight different bank groups.
-template <int D>
-__device__ __forceinline__ void stage_row_sw128(uint8_t* tile, const uint32_t (&x)[D / 32][32], float scale, int r) {
-  uint8_t* row = tile + r * 128;
-#pragma unroll
-  for (int e = 0; e < D / 8; ++e) {
-    const int c = e / 8, u = e % 8;
-    *reinterpret_cast<uint4*>(row + c * 16384 + ((u ^ (r & 7)) << 4)) = pack8_bf16(x[e / 4] + 8 * (e % 4), scale);
-  }
+  for (int u = 0; u < 8; ++u) d4[u] = pack8_bf16(x[u / 4] + 8 * (u % 4), scale);
 }
 
 // DET: deterministic dQ. Every query tile receives its dQ contributions in
@@ -184,8 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                const BwdArgs a) {
   using L = BwdSmem<D>;
   constexpr int NQ = L::kQStages;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
   Bars& bars = *reinterpret_cast<Bars*>(smem + L::kBar);
   auto* hdr = reinterpret_cast<WsHeader*>(a.workspace);
   const int2* pairs = reinterpret_cast<const int2*>(static_cast<const char*>(a.workspace) + a.pairs_offset);
@@ -194,28 +201,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* qcount = reinterpret_cast<uint32_t*>(static_cast<char*>(a.workspace) + a.qcount_offset);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  // The layout uses the whole opt-in shared memory with no alignment slack:
+  // the swizzled tiles need a 1024-byte-aligned base. The dynamic window
+  // starts aligned on this architecture; if it ever did not, the call
+  // reports an error instead of computing garbage.
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicCAS(&hdr->status, 0u, static_cast<uint32_t>(FA_ERR_CUDA));
+    return;
+  }
+
   if (threadIdx.x == 0) {
     mbar_init(&bars.kv_full, 1);
     mbar_init(&bars.kv_empty, 1);
-    for (int i = 0; i < L::kQStages; ++i) {
+    for (int i = 0; i < NQ; ++i) {
       mbar_init(&bars.qdo_full[i], 1);
       mbar_init(&bars.qdo_empty[i], 1);
       mbar_init(&bars.ld_full[i], 2);
-      mbar_init(&bars.ld_empty[i], 4);
+      mbar_init(&bars.ld_empty[i], 8);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars.st_full[i], 1);
-      mbar_init(&bars.ds_full[i], 4);
-      mbar_init(&bars.ds_empty[i], 1);
-      mbar_init(&bars.dq_full[i], 1);
-      mbar_init(&bars.dq_empty[i], 4);
-    }
+    mbar_init(&bars.s_full, 1);
+    mbar_init(&bars.dp_full, 1);
+    mbar_init(&bars.p_full, 8);
+    mbar_init(&bars.ds_full, 8);
+    mbar_init(&bars.dq_full, 1);
+    mbar_init(&bars.dq_free, 4);
     mbar_init(&bars.dkv_full, 1);
-    mbar_init(&bars.dv_empty, 4);
-    mbar_init(&bars.dk_empty, 4);
+    mbar_init(&bars.dv_free, 4);
+    mbar_init(&bars.dk_free, 4);
     mbar_init(&bars.drain, 1);
-    // Item consumers: MMA warp (1), row loaders (2), P/dS warps (4), drain warps (4).
-    item_ring_init(bars.items, 11);
+    // Item consumers: MMA warp (1), row loaders (2), P/dS warps (8), drain warps (4).
+    item_ring_init(bars.items, 15);
     bars.abort_flag = 0;
     fence_mbar_init();
   }
@@ -225,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_do);
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == kDrainWarp0 && lane == 0) {
     tma_prefetch_desc(&tm_dk);
     tma_prefetch_desc(&tm_dv);
   }
@@ -301,19 +316,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     // The whole warp runs this loop converged; one elected lane issues each
-    // group of MMAs and the commits. Descriptors are built once and advanced
-    // by constant offsets.
-    constexpr uint32_t kIdS = idesc_bf16_f32(BN, BM, false, false);   // S^T, dP^T: 128 x 64, K = D
-    constexpr uint32_t kIdKV = idesc_bf16_f32(BN, D, false, true);    // dV, dK: 128 x D, K = 64
-    constexpr uint32_t kIdQ = idesc_bf16_f32(128, BM, true, true);    // dQ^T: 128 (>= D) x 64, K = 128
+    // group of MMAs and the commits. Per step p, in issue order (the tensor
+    // pipe executes one thread's MMAs in order, so an MMA may overwrite TMEM
+    // columns that earlier-issued MMAs read):
+    //   S^T = K Q^T; [dQ^T of p-1 read out] dP^T = V dO^T; [P^T written]
+    //   dV += P^T dO; [dS^T written] dK += dS^T Q; dQ^T = K^T dS^T.
+    constexpr uint32_t kIdS = idesc_bf16_f32(BN, BM, false, false);  // S^T, dP^T: 128 x 128, K = D
+    constexpr uint32_t kIdKV = idesc_bf16_f32(BN, D, false, true);   // dV, dK: 128 x D, K = 128 queries
+    constexpr uint32_t kIdQ = idesc_bf16_f32(128, BM, true, true);   // dQ^T: 128 (>= D) x 128, K = 128 keys
     const uint64_t k_kmaj = smem_desc_sw128(smem_u32(smem + L::kK), 16, 1024);
     const uint64_t v_kmaj = smem_desc_sw128(smem_u32(smem + L::kV), 16, 1024);
+    // At head_dim 64 the second 64-row half of M reads the first again
+    // (lanes 64-127 of dQ^T are then ignored).
     const uint64_t k_mn = smem_desc_sw128(smem_u32(smem + L::kK), D == 128 ? L::kKChunk : 0, 1024);
     const uint64_t qdo_kmaj0 = smem_desc_sw128(smem_u32(smem + L::kQdo), 16, 1024);
     const uint64_t qdo_mn0 = smem_desc_sw128(smem_u32(smem + L::kQdo), L::kQChunk, 1024);
-    const uint64_t ds_kmaj0 = smem_desc_sw128(smem_u32(smem + L::kDs), 16, 1024);
-    const uint64_t ds_mn0 = smem_desc_sw128(smem_u32(smem + L::kDs), 0, 1024);
-    constexpr uint64_t kQTileD = L::kQTile >> 4;    // descriptor step between Q and dO of a stage
+    const uint64_t ds_mn = smem_desc_sw128(smem_u32(smem + L::kDs), L::kDsHalf, 1024);
+    constexpr uint64_t kQTileD = L::kQTile >> 4;  // descriptor step between Q and dO of a stage
     uint32_t m = 0, p = 0, ni = 0;
     for (;;) {
       int slot;
@@ -326,85 +345,84 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (it.n == 0) continue;
       if (!wait_bar_warp(&bars.kv_full, m & 1, ab)) goto mma_done;
       tc_fence_after();
-      for (int s = 0; s <= it.n; ++s) {
-        if (s < it.n) {
-          const uint32_t ps = p + s;
-          const int st = ps & 1;      // TMEM S^T / dP^T buffer
-          const int qs = ps % NQ;     // Q/dO stage
-          if (!wait_bar_warp(&bars.qdo_full[qs], (ps / NQ) & 1, ab)) goto mma_done;
-          if (ps >= 2 && !wait_bar_warp(&bars.dq_empty[st], ((ps >> 1) - 1) & 1, ab)) goto mma_done;
-          tc_fence_after();
-          const uint64_t q_desc = qdo_kmaj0 + static_cast<uint64_t>((2 * qs * L::kQTile) >> 4);
-          if (elect_one()) {
+      for (int s = 0; s < it.n; ++s, ++p) {
+        const int qs = p % NQ;
+        // Descriptors are rebuilt from opaque copies where they are used, so
+        // that the compiler does not keep every offset form in registers.
+        const uint64_t q_kmaj = opaque_u64(qdo_kmaj0) + static_cast<uint64_t>((2 * qs * L::kQTile) >> 4);
+        const uint64_t q_mn = opaque_u64(qdo_mn0) + static_cast<uint64_t>((2 * qs * L::kQTile) >> 4);
+        if (!wait_bar_warp(&bars.qdo_full[qs], (p / NQ) & 1, ab)) goto mma_done;
+        tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint64_t oa = ((kk >> 2) * L::kKChunk + (kk & 3) * 32) >> 4;
-              const uint64_t ob = ((kk >> 2) * L::kQChunk + (kk & 3) * 32) >> 4;
-              mma_ss(tmem + kColS + st * BM, k_kmaj + oa, q_desc + ob, kIdS, kk > 0);
-            }
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint64_t oa = ((kk >> 2) * L::kKChunk + (kk & 3) * 32) >> 4;
-              const uint64_t ob = ((kk >> 2) * L::kQChunk + (kk & 3) * 32) >> 4;
-              mma_ss(tmem + kColDP + st * BM, v_kmaj + oa, q_desc + kQTileD + ob, kIdS, kk > 0);
-            }
-            mma_commit(&bars.st_full[st]);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t o = ((kk >> 2) * L::kKChunk + (kk & 3) * 32) >> 4;
+            mma_ss(tmem + kColS, opaque_u64(k_kmaj) + o, q_kmaj + o, kIdS, kk > 0);
           }
-          __syncwarp();
+          mma_commit(&bars.s_full);
         }
-        if (s > 0) {
-          const uint32_t pp = p + s - 1;
-          const int pb = pp & 1;
-          const int qs = pp % NQ;
-          if (!wait_bar_warp(&bars.ds_full[pb], (pp >> 1) & 1, ab)) goto mma_done;
-          // First step of an item: the drain group must have read the
-          // previous item's dV (then dK) out of TMEM.
-          if (s == 1 && m > 0 && !wait_bar_warp(&bars.dv_empty, (m - 1) & 1, ab)) goto mma_done;
-          tc_fence_after();
-          const uint64_t q_mn = qdo_mn0 + static_cast<uint64_t>((2 * qs * L::kQTile) >> 4);
-          const uint64_t ds_k = ds_kmaj0 + static_cast<uint64_t>((pb * L::kDsTile) >> 4);
-          const uint64_t ds_mn = ds_mn0 + static_cast<uint64_t>((pb * L::kDsTile) >> 4);
-          const uint32_t acc = (s > 1) ? 1u : 0u;
-          if (elect_one()) {
-            // dV += P^T dO (P^T from TMEM, dO MN-major); dK += dS^T Q.
+        __syncwarp();
+        // dP^T goes where the previous step's dQ^T is until the drain group
+        // has read it out.
+        if (p > 0 && !wait_bar_warp(&bars.dq_free, (p - 1) & 1, ab)) goto mma_done;
+        tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-            for (int kk = 0; kk < BM / 16; ++kk)
-              mma_ts(tmem + kColDV, tmem + kColS + pb * BM + kk * 8, q_mn + kQTileD + ((kk * 2048) >> 4), kIdKV,
-                     (acc | kk) ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t o = ((kk >> 2) * L::kKChunk + (kk & 3) * 32) >> 4;
+            mma_ss(tmem + kColDP, opaque_u64(v_kmaj) + o, q_kmaj + kQTileD + o, kIdS, kk > 0);
           }
-          __syncwarp();
-          if (s == 1 && m > 0 && !wait_bar_warp(&bars.dk_empty, (m - 1) & 1, ab)) goto mma_done;
-          tc_fence_after();
-          if (elect_one()) {
-#pragma unroll
-            for (int kk = 0; kk < BM / 16; ++kk)
-              mma_ss(tmem + kColDK, ds_k + ((kk * 32) >> 4), q_mn + ((kk * 2048) >> 4), kIdKV, (acc | kk) ? 1u : 0u);
-            // dQ^T = K^T dS^T into the dP^T columns of this step.
-#pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk)
-              mma_ss(tmem + kColDP + pb * BM, k_mn + ((kk * 2048) >> 4), ds_mn + ((kk * 2048) >> 4), kIdQ, kk > 0);
-            mma_commit(&bars.dq_full[pb]);
-            mma_commit(&bars.qdo_empty[qs]);
-            mma_commit(&bars.ds_empty[pb]);
-          }
-          __syncwarp();
+          mma_commit(&bars.dp_full);
         }
+        __syncwarp();
+        if (!wait_bar_warp(&bars.p_full, p & 1, ab)) goto mma_done;
+        // First step of an item: the drain group must have read the previous
+        // item's dV (then dK) out of TMEM.
+        if (s == 0 && m > 0 && !wait_bar_warp(&bars.dv_free, (m - 1) & 1, ab)) goto mma_done;
+        tc_fence_after();
+        const uint32_t acc = s > 0 ? 1u : 0u;
+        if (elect_one()) {
+          // dV += P^T dO: P^T bf16 in TMEM (16 queries = 8 columns per MMA;
+          // queries 64-127 start 64 columns further), dO MN-major.
+#pragma unroll
+          for (int kk = 0; kk < BM / 16; ++kk)
+            mma_ts(tmem + kColDV, tmem + kColS + (kk >> 2) * 64 + (kk & 3) * 8,
+                   q_mn + kQTileD + ((kk * 2048) >> 4), kIdKV, (acc | kk) ? 1u : 0u);
+        }
+        __syncwarp();
+        if (!wait_bar_warp(&bars.ds_full, p & 1, ab)) goto mma_done;
+        if (s == 0 && m > 0 && !wait_bar_warp(&bars.dk_free, (m - 1) & 1, ab)) goto mma_done;
+        tc_fence_after();
+        if (elect_one()) {
+          // dK += dS^T Q (dS^T bf16 in TMEM, 32 columns after its P^T).
+#pragma unroll
+          for (int kk = 0; kk < BM / 16; ++kk)
+            mma_ts(tmem + kColDK, tmem + kColS + (kk >> 2) * 64 + 32 + (kk & 3) * 8, q_mn + ((kk * 2048) >> 4),
+                   kIdKV, (acc | kk) ? 1u : 0u);
+          // dQ^T = K^T dS^T (dS^T from shared memory) into the dP^T columns.
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            mma_ss(tmem + kColDP, opaque_u64(k_mn) + ((kk * 2048) >> 4), opaque_u64(ds_mn) + ((kk * 2048) >> 4), kIdQ,
+                   kk > 0);
+          mma_commit(&bars.dq_full);
+        }
+        __syncwarp();
       }
       if (elect_one()) {
         mma_commit(&bars.dkv_full);
         mma_commit(&bars.kv_empty);
       }
       __syncwarp();
-      p += it.n;
       ++m;
     }
   mma_done:
     if (elect_one()) mma_commit(&bars.drain);
     __syncwarp();
     wait_bar_final(&bars.drain, 0, ab);
-  } else if (warp < 4) {
+  } else if (warp < kPdsWarp0) {
     // ------------------------------------------------------------ lse / Dv rows
-    const int r = threadIdx.x - 64;  // query row within the tile, 0..63
+    // Two rows per thread (r and r + 64) of the step's 128 query rows.
+    const int r = threadIdx.x - 64;
     uint32_t p = 0, ni = 0;
     for (;;) {
       int islot;
@@ -417,30 +435,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int slot = p % NQ;
         if (p >= NQ && !wait_bar_warp(&bars.ld_empty[slot], ((p / NQ) - 1) & 1, ab)) goto loader_done;
         const Step sp = item_step(it, s);
-        const int qi = sp.t * BM + r;  // row within the sequence
-        // Stored negated and in base 2: -lse*log2(e); -inf for rows outside
-        // the sequence or without a visible key, which makes their P exactly 0.
-        float nlse2 = -INFINITY, dv = 0.f;
-        if (qi < it.s.lq) {
-          const size_t gq = static_cast<size_t>(it.s.q0) + qi;
-          const float l = __ldg(a.lse + static_cast<size_t>(sp.h) * a.total_q + gq);
-          if (l != -INFINITY) {
-            nlse2 = -l * 1.4426950408889634f;
-            dv = __ldg(dvec + static_cast<size_t>(sp.h) * a.tq_pad + gq);
-          }
-        }
         float* ld = reinterpret_cast<float*>(smem + L::kLd) + slot * 2 * BM;
-        ld[r] = nlse2;
-        ld[BM + r] = dv;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int rr = r + 64 * u;
+          const int qi = sp.t * BM + rr;  // row within the sequence
+          // Stored negated and in base 2: -lse*log2(e); -inf for rows outside
+          // the sequence or without a visible key, which makes their P exactly 0.
+          float nlse2 = -INFINITY, dv = 0.f;
+          if (qi < it.s.lq) {
+            const size_t gq = static_cast<size_t>(it.s.q0) + qi;
+            const float l = __ldg(a.lse + static_cast<size_t>(sp.h) * a.total_q + gq);
+            if (l != -INFINITY) {
+              nlse2 = -l * 1.4426950408889634f;
+              dv = __ldg(dvec + static_cast<size_t>(sp.h) * a.tq_pad + gq);
+            }
+          }
+          ld[rr] = nlse2;
+          ld[BM + rr] = dv;
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.ld_full[slot]);
       }
     }
   loader_done:;
-  } else if (warp < 8) {
+  } else if (warp < kDrainWarp0) {
     // ------------------------------------------------------------ P^T, dS^T
-    const int kr = threadIdx.x - 128;  // key row in the tile == TMEM lane
+    // Warpgroup qh owns queries 64*qh .. 64*qh+63 of every step; thread = key
+    // row = TMEM lane. Phase 1: P^T from S^T (handed to the dV MMA at once);
+    // phase 2: dS^T from dP^T and the bf16 P^T values kept in registers.
+    const int qh = (warp - kPdsWarp0) >> 2;
+    const int kr = (threadIdx.x - kPdsWarp0 * 32) & 127;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t t_s = tmem + lane_base + kColS + qh * 64;    // S^T of my queries; P^T, dS^T after it
+    const uint32_t t_dp = tmem + lane_base + kColDP + qh * 64;  // dP^T of my queries
+    uint8_t* ds_row = smem + L::kDs + qh * L::kDsHalf + kr * 128;
     uint32_t p = 0, ni = 0;
     for (;;) {
       int islot;
@@ -453,48 +482,71 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool key_ok = kg < it.s.lk;
       const int diag = it.s.lk - it.s.lq;
       for (int s = 0; s < it.n; ++s, ++p) {
-        const int pb = p & 1;
-        if (!wait_bar_warp(&bars.st_full[pb], (p >> 1) & 1, ab)) goto compute_done;
         const int slot = p % NQ;
+        if (!wait_bar_warp(&bars.s_full, p & 1, ab)) goto compute_done;
         if (!wait_bar_warp(&bars.ld_full[slot], (p / NQ) & 1, ab)) goto compute_done;
-        if (p >= 2 && !wait_bar_warp(&bars.ds_empty[pb], ((p >> 1) - 1) & 1, ab)) goto compute_done;
         tc_fence_after();
-        const float* ld = reinterpret_cast<const float*>(smem + L::kLd) + slot * 2 * BM;
-        const int row0 = item_step(it, s).t * BM;  // first query row of the step
+        const float* ld = reinterpret_cast<const float*>(smem + L::kLd) + slot * 2 * BM + qh * 64;
+        const int row0 = item_step(it, s).t * BM + qh * 64;  // first query row of my half
         // Visible iff kg <= row + diag, i.e. e >= kg - diag - row0; keys past
         // the sequence see nothing.
         int e_min = CAUSAL ? kg - diag - row0 : 0;
-        if (!key_ok) e_min = BM;
-        uint8_t* ds_row = smem + L::kDs + pb * L::kDsTile + kr * 128;
+        if (!key_ok) e_min = 64;
         const uint64_t sc2 = f2_make(a.scale_log2, a.scale_log2);
+        // P^T of my 64 queries as bf16 pairs: written to TMEM for the dV MMA
+        // and kept in registers for dS^T, so that dS^T is formed from exactly
+        // the probabilities the dV MMA uses.
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < BM / 32; ++c) {
-          uint32_t sv[32], dpv[32];
-          tmem_ld32(tmem + lane_base + kColS + pb * BM + c * 32, sv);
-          tmem_ld32(tmem + lane_base + kColDP + pb * BM + c * 32, dpv);
+        for (int c = 0; c < 2; ++c) {
+          uint32_t sv[32];
+          tmem_ld32(t_s + c * 32, sv);
           tmem_wait_ld();
-          uint32_t pk[16], dsk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const int q = c * 32 + e;
-            // Pairs of query columns share packed f32x2 arithmetic.
             const uint64_t nl2 = *reinterpret_cast<const uint64_t*>(ld + q);
-            const uint64_t dv2 = *reinterpret_cast<const uint64_t*>(ld + BM + q);
             float x0, x1;
             f2_split(f2_fma(f2_make(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sc2, nl2), x0, x1);
             float p0 = ex2_approx(x0);
             float p1 = ex2_approx(x1);
             if (q < e_min) p0 = 0.f;
             if (q + 1 < e_min) p1 = 0.f;
-            const uint64_t p2 = f2_make(p0, p1);
+            pk[q / 2] = pack_bf16x2(p0, p1);
+          }
+          // P^T into the first 32 columns of my S^T half; the second chunk
+          // writes columns the first chunk has already read.
+          tmem_st16(t_s + c * 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[c * 16]));
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.p_full);
+        // dS^T of the previous step has been read by its dQ^T MMAs: S^T of
+        // this step was issued after them and has completed.
+        if (!wait_bar_warp(&bars.dp_full, p & 1, ab)) goto compute_done;
+        tc_fence_after();
+        const uint64_t* dv2p = reinterpret_cast<const uint64_t*>(ld + BM);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t dpv[32];
+          tmem_ld32(t_dp + c * 32, dpv);
+          tmem_wait_ld();
+          uint32_t dsk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int q = c * 32 + e;
             float d0, d1;
-            f2_split(f2_mul(p2, f2_sub(f2_make(__uint_as_float(dpv[e]), __uint_as_float(dpv[e + 1])), dv2)), d0, d1);
-            pk[e / 2] = pack_bf16x2(p0, p1);
+            const uint32_t pp = pk[q / 2];  // bf16 pair -> two exact fp32 values
+            f2_split(f2_mul(f2_make(__uint_as_float(pp << 16), __uint_as_float(pp & 0xffff0000u)),
+                            f2_sub(f2_make(__uint_as_float(dpv[e]), __uint_as_float(dpv[e + 1])), dv2p[q / 2])),
+                     d0, d1);
             dsk[e / 2] = pack_bf16x2(d0, d1);
           }
-          // P^T (bf16 pairs) into the first 32 columns of this step's S^T.
-          tmem_st16(tmem + lane_base + kColS + pb * BM + c * 16, pk);
-          // dS^T row kr, queries c*32 .. c*32+31: four 16-byte chunks, 128-byte swizzle.
+          // dS^T into TMEM (A operand of dK) and into shared memory, row kr,
+          // queries c*32 .. c*32+31: four 16-byte units, 128-byte swizzle
+          // (B operand of dQ^T).
+          tmem_st16(t_s + 32 + c * 16, dsk);
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int chunk = (c * 4 + u) ^ (kr & 7);
@@ -507,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&bars.ds_full[pb]);
+          mbar_arrive(&bars.ds_full);
           mbar_arrive(&bars.ld_empty[slot]);
         }
       }
@@ -515,10 +567,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   compute_done:;
   } else {
     // ------------------------------------------------------------ dQ drain, dK/dV
-    const int t = threadIdx.x - 256;  // 0..127: TMEM lane (d for dQ^T, key row for dK/dV)
-    const int q4 = warp & 3;
-    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
-    float* stage = reinterpret_cast<float*>(smem + L::kStage);
+    const int t = threadIdx.x - kDrainWarp0 * 32;  // 0..127: TMEM lane (d for dQ^T, key row for dK/dV)
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     uint32_t p = 0, m = 0, ni = 0;
     uint32_t* det_prev = nullptr;  // deterministic mode: counter whose turn is still to be passed on
     for (;;) {
@@ -542,36 +592,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         continue;
       }
+      int qs = 0;  // Q/dO stage of the current step: its staging area
       for (int s = 0; s < it.n; ++s, ++p) {
-        const int pb = p & 1;
         // Group-wide decision: every warp of this group reaches the vote, so
         // none is left waiting on the named barriers below.
-        if (!named_bar_and(1, 128, wait_bar(&bars.dq_full[pb], (p >> 1) & 1, ab))) goto drain_done;
+        if (!named_bar_and(1, 128, wait_bar(&bars.dq_full, p & 1, ab))) goto drain_done;
         tc_fence_after();
-        uint32_t v0[32], v1[32];
-        tmem_ld32(tmem + lane_base + kColDP + pb * BM, v0);
-        tmem_ld32(tmem + lane_base + kColDP + pb * BM + 32, v1);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.dq_empty[pb]);
-        // The previous bulk reduction must have finished reading the stage.
-        if (t == 0) bulk_wait_group_read0();
-        named_bar_sync(1, 128);
-        if (t < D) {
+        // Every MMA of the step has completed, so its Q/dO stage is free:
+        // the step's fp32 dQ tile (128 x D) is staged there and leaves with
+        // one bulk reduction (128 consecutive rows of one head are one
+        // contiguous block of the head-major accumulator).
+        qs = static_cast<int>(p % NQ);
+        float* stage = reinterpret_cast<float*>(smem + L::kQdo + 2 * qs * L::kQTile);
+        const Step sp = item_step(it, s);
+        const size_t q0 = static_cast<size_t>(it.s.q0) + static_cast<size_t>(sp.t) * BM;
+        uint32_t* cnt = qcount + static_cast<size_t>(sp.h) * a.tq_pad + q0;
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(tmem + lane_base + kColDP + h * 64, v0);
+          tmem_ld32(tmem + lane_base + kColDP + h * 64 + 32, v1);
+          tmem_wait_ld();
+          if (h == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.dq_free);
+          }
+          if (t < D) {
+            float* st = stage + h * 64 * D;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) stage[e * D + t] = __uint_as_float(v0[e]);
+            for (int e = 0; e < 32; ++e) st[e * D + t] = __uint_as_float(v0[e]);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) stage[(32 + e) * D + t] = __uint_as_float(v1[e]);
+            for (int e = 0; e < 32; ++e) st[(32 + e) * D + t] = __uint_as_float(v1[e]);
+          }
         }
         fence_proxy_async_smem();
         named_bar_sync(1, 128);
         if (t == 0) {
-          const Step sp = item_step(it, s);
-          const size_t q0 = static_cast<size_t>(it.s.q0) + static_cast<size_t>(sp.t) * BM;
-          uint32_t* cnt = qcount + static_cast<size_t>(sp.h) * a.tq_pad + q0;
-          const bool turn = !DET || wait_dq_turn(cnt, static_cast<uint32_t>(it.j), ab);
-          if (turn) {
+          // Deterministic mode: this query tile's turn first (a wait that
+          // runs out raises the abort flag, and nothing more is added).
+          if (DET) wait_dq_turn(cnt, static_cast<uint32_t>(it.j), ab);
+          if (!*ab.flag) {
             if (DET) fence_proxy_async_global();
             bulk_reduce_add_f32(dqacc + (static_cast<size_t>(sp.h) * a.tq_pad + q0) * D, stage, BM * D * 4);
             bulk_commit_group();
@@ -587,6 +648,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               det_prev = cnt;
             }
           }
+          // Hand the stage back to the loader once the reduction has read
+          // it (an item's last stage serves the dK/dV stores first).
+          if (s + 1 < it.n) {
+            bulk_wait_group_read0();
+            mbar_arrive(&bars.qdo_empty[qs]);
+          }
         }
       }
       if (DET && t == 0 && det_prev) {
@@ -597,62 +664,64 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // dK, dV of this key tile. dV is read out of TMEM first and released
       // at once, so the next item's first dV MMAs wait only for that read;
-      // dK follows. A whole tile leaves through TMA stores from the stage
-      // (the coalesced path, which keeps the load/store unit free for the
-      // P/dS warps); a tile cut by the end of its sequence is stored row by
-      // row, so that no row of the next sequence is touched.
+      // dK follows. A whole tile leaves through TMA stores from the last
+      // step's stage (the coalesced path, which keeps the load/store unit
+      // free for the P/dS warps): dV in its first half, dK in its second; a
+      // tile cut by the end of its sequence is stored row by row, so that no
+      // row of the next sequence is touched.
       if (!named_bar_and(1, 128, wait_bar(&bars.dkv_full, m & 1, ab))) goto drain_done;
       tc_fence_after();
       {
         const bool whole = (it.j + 1) * BN <= it.s.lk;  // the same for the whole group
         const int row0 = it.s.k0 + it.j * BN;
-        uint8_t* tile = smem + L::kStage;
-        uint32_t x[D / 32][32];
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) tmem_ld32(tmem + lane_base + kColDV + c * 32, x[c]);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.dv_empty);
+        uint8_t* stage = smem + L::kQdo + 2 * qs * L::kQTile;
         if (whole) {
-          if (t == 0) bulk_wait_group_read0();  // the last dQ reduction has read the stage
+          // The last dQ reduction must have read the stage.
+          if (t == 0) bulk_wait_group_read0();
           named_bar_sync(1, 128);
-          stage_row_sw128<D>(tile, x, 1.f, t);
-          fence_proxy_async_smem();
-          named_bar_sync(1, 128);
-          if (t == 0) {
-#pragma unroll
-            for (int c = 0; c < D / 64; ++c) tma_store_2d(&tm_dv, tile + c * 16384, it.hk * D + c * 64, row0);
-            bulk_commit_group();
-          }
-        } else if (key_ok) {
-          store_row_bf16<D>(static_cast<__nv_bfloat16*>(a.dv) + krow * D, x, 1.f);
         }
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) tmem_ld32(tmem + lane_base + kColDK + c * 32, x[c]);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.dk_empty);
-        if (whole) {
-          if (t == 0) bulk_wait_group_read0();  // the dV stores have read the stage
-          named_bar_sync(1, 128);
-          stage_row_sw128<D>(tile, x, a.scale, t);
-          fence_proxy_async_smem();
-          named_bar_sync(1, 128);
-          if (t == 0) {
-#pragma unroll
-            for (int c = 0; c < D / 64; ++c) tma_store_2d(&tm_dk, tile + c * 16384, it.hk * D + c * 64, row0);
-            bulk_commit_group();
+#pragma unroll 1
+        for (int g = 0; g < 2; ++g) {  // g = 0: dV, g = 1: dK (times scale)
+          const int col = g == 0 ? kColDV : kColDK;
+          const float sc = g == 0 ? 1.f : a.scale;
+          __nv_bfloat16* gdst = static_cast<__nv_bfloat16*>(g == 0 ? a.dv : a.dk) + krow * D;
+          uint8_t* box = stage + g * L::kQTile;  // bf16 boxes of [128 rows x 64 columns], 16 KB apart
+#pragma unroll 1
+          for (int c = 0; c < D / 64; ++c) {
+            uint32_t x[2][32];
+            tmem_ld32(tmem + lane_base + col + c * 64, x[0]);
+            tmem_ld32(tmem + lane_base + col + c * 64 + 32, x[1]);
+            tmem_wait_ld();
+            if (c == D / 64 - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(g == 0 ? &bars.dv_free : &bars.dk_free);
+            }
+            if (whole)
+              chunk_to_box(box + c * 16384, x, sc, t);
+            else if (key_ok)
+              chunk_to_global(gdst + c * 64, x, sc);
           }
-        } else if (key_ok) {
-          store_row_bf16<D>(static_cast<__nv_bfloat16*>(a.dk) + krow * D, x, a.scale);
+          if (whole) {
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            if (t == 0) {
+              const CUtensorMap* map = g == 0 ? &tm_dv : &tm_dk;
+#pragma unroll
+              for (int c = 0; c < D / 64; ++c) tma_store_2d(map, box + c * 16384, it.hk * D + c * 64, row0);
+              bulk_commit_group();
+            }
+          }
+        }
+        if (t == 0) {
+          bulk_wait_group_read0();  // the stores (and the last reduction) have read the stage
+          mbar_arrive(&bars.qdo_empty[qs]);
         }
       }
       ++m;
     }
   drain_done:
-    // Bulk reductions still reading the stage must finish before exit.
+    // Bulk operations still reading shared memory must finish before exit.
     if (t == 0) bulk_wait_group0();
   }
 
@@ -667,14 +736,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // The two streaming kernels around the main one take kUnits (row, head)
 // units per warp, consecutive in memory, and issue all their loads before
-// using any, so that enough bytes are in flight to run at HBM speed.
+// using any, so that enough bytes are in flight to run at HBM speed. They
+// serve every head dimension (64, 128, 256): lane l of a warp handles
+// elements l*E .. l*E+E-1 of a row of D = 32*E.
 constexpr int kUnits = 4;
+
+template <int N>
+struct Words;  // N 32-bit words in one vector access
+template <>
+struct Words<1> {
+  using T = uint32_t;
+};
+template <>
+struct Words<2> {
+  using T = uint2;
+};
+template <>
+struct Words<4> {
+  using T = uint4;
+};
 
 // Dv[h, r] = sum_c dO[r, h, c] * O[r, h, c] in fp32, and dQacc[h, r, :] = 0.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdArgs a) {
-  constexpr int E = D / 32;  // bf16 elements per lane: 4 (8 bytes) or 2 (4 bytes)
-  using V = typename std::conditional<E == 4, uint2, uint32_t>::type;
+  constexpr int E = D / 32;  // bf16 elements per lane: 2, 4 or 8 (4, 8 or 16 bytes)
+  using V = typename Words<E / 2>::T;
   const long long units = static_cast<long long>(a.total_q) * a.H;
   const long long u0 = ((static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5) * kUnits;
   const int lane = threadIdx.x & 31;
@@ -730,37 +816,35 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdArgs a) {
 // dQ[r, h, :] = bf16(scale * dQacc[h, r, :]).
 template <int D>
 __global__ void __launch_bounds__(256) bwd_convert_kernel(const BwdArgs a) {
-  constexpr int E = D / 32;  // fp32 elements per lane: 4 (16 bytes) or 2 (8 bytes)
-  using F = typename std::conditional<E == 4, float4, float2>::type;
+  constexpr int E = D / 32;          // fp32 elements per lane: 2, 4 or 8
+  constexpr int W = E < 4 ? E : 4;   // words per vector load
+  constexpr int NL = E / W;          // vector loads per lane and unit
+  using F = typename Words<W>::T;
+  using O = typename Words<E / 2>::T;
   const long long units = static_cast<long long>(a.total_q) * a.H;
   const long long u0 = ((static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5) * kUnits;
   const int lane = threadIdx.x & 31;
   if (u0 >= units) return;
   const float* acc = reinterpret_cast<const float*>(static_cast<const char*>(a.workspace) + a.dqacc_offset);
-  F v[kUnits];
+  F v[kUnits][NL];
 #pragma unroll
   for (int i = 0; i < kUnits; ++i) {
     const long long u = u0 + i;
-    if (u < units) {
-      const int row = static_cast<int>(u / a.H), h = static_cast<int>(u % a.H);
-      v[i] = reinterpret_cast<const F*>(acc + (static_cast<size_t>(h) * a.tq_pad + row) * D)[lane];
-    } else {
-      v[i] = F{};
-    }
+    const int row = static_cast<int>(u / a.H), h = static_cast<int>(u % a.H);
+    const F* src = reinterpret_cast<const F*>(acc + (static_cast<size_t>(h) * a.tq_pad + row) * D) + lane * NL;
+#pragma unroll
+    for (int l = 0; l < NL; ++l) v[i][l] = u < units ? src[l] : F{};
   }
 #pragma unroll
   for (int i = 0; i < kUnits; ++i) {
     const long long u = u0 + i;
     if (u >= units) break;
-    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.dq) + u * D;
-    if constexpr (E == 4) {
-      uint2 o;
-      o.x = pack_bf16x2(v[i].x * a.scale, v[i].y * a.scale);
-      o.y = pack_bf16x2(v[i].z * a.scale, v[i].w * a.scale);
-      reinterpret_cast<uint2*>(dst)[lane] = o;
-    } else {
-      reinterpret_cast<uint32_t*>(dst)[lane] = pack_bf16x2(v[i].x * a.scale, v[i].y * a.scale);
-    }
+    const float* x = reinterpret_cast<const float*>(&v[i][0]);
+    O o;
+    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+    for (int k = 0; k < E / 2; ++k) ow[k] = pack_bf16x2(x[2 * k] * a.scale, x[2 * k + 1] * a.scale);
+    reinterpret_cast<O*>(static_cast<__nv_bfloat16*>(a.dq) + u * D)[lane] = o;
   }
 }
 
@@ -768,9 +852,9 @@ template <int D, bool CAUSAL, bool DET>
 cudaError_t launch_main(const BwdArgs& a, const BwdMaps& m, cudaStream_t stream) {
   using L = BwdSmem<D>;
   auto kern = bwd_kernel<D, CAUSAL, DET>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
   if (e != cudaSuccess) return e;
-  kern<<<a.grid, kThreads, L::kAlloc, stream>>>(m.q, m.k, m.v, m.dout, m.dk, m.dv, a);
+  kern<<<a.grid, kThreads, L::kBytes, stream>>>(m.q, m.k, m.v, m.dout, m.dk, m.dv, a);
   return cudaGetLastError();
 }
 
@@ -782,8 +866,10 @@ cudaError_t launch_bwd_preprocess(const BwdArgs& a, cudaStream_t stream) {
   if (blocks == 0) return cudaSuccess;
   if (a.D == 64)
     bwd_preprocess_kernel<64><<<blocks, 256, 0, stream>>>(a);
-  else
+  else if (a.D == 128)
     bwd_preprocess_kernel<128><<<blocks, 256, 0, stream>>>(a);
+  else
+    bwd_preprocess_kernel<256><<<blocks, 256, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -804,8 +890,10 @@ cudaError_t launch_bwd_convert(const BwdArgs& a, cudaStream_t stream) {
   if (blocks == 0) return cudaSuccess;
   if (a.D == 64)
     bwd_convert_kernel<64><<<blocks, 256, 0, stream>>>(a);
-  else
+  else if (a.D == 128)
     bwd_convert_kernel<128><<<blocks, 256, 0, stream>>>(a);
+  else
+    bwd_convert_kernel<256><<<blocks, 256, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

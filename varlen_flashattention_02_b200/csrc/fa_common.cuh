@@ -22,16 +22,17 @@ constexpr int kFwdItemRows = 256;
 // 128-row query tile per CTA only.
 __host__ __device__ inline int fwd_item_rows(int D) { return D > 128 ? kFwdBM : kFwdItemRows; }
 // Backward tiles: a work item is 128 key rows of one (sequence, head);
-// queries stream through in tiles of 64.
+// queries stream through in tiles of 128.
 constexpr int kBwdBN = 128;
-constexpr int kBwdBM = 64;
+constexpr int kBwdBM = 128;
 
 // Per-call device state at the start of the workspace.
 struct WsHeader {
-  uint32_t status;        // fa_status_t of the device side of the call
-  uint32_t n_pairs;       // number of (sequence, tile) pairs in `pairs`
-  uint32_t work_counter;  // next work item to hand out (reset by the scheduler)
-  uint32_t reserved[61];
+  uint32_t status;         // fa_status_t of the device side of the call
+  uint32_t n_pairs;        // number of (sequence, tile) pairs in `pairs`
+  uint32_t work_counter;   // next work item to hand out (reset by the scheduler)
+  uint32_t work_counter2;  // the same, for a second kernel over the same list (head_dim 256 backward)
+  uint32_t reserved[60];
 };
 static_assert(sizeof(WsHeader) == 256, "header is one 256-byte block");
 
@@ -173,10 +174,11 @@ __host__ __device__ inline int fwd_k_tiles(int row_end, int lq, int lk, bool cau
   return n < nk ? static_cast<int>(n) : nk;
 }
 
-// Range [begin, end) of backward query tiles (kBwdBM rows) that see at least
+// Range [begin, end) of backward query tiles (bm rows) that see at least
 // one key of key tile j (keys j*BN ..).
-__host__ __device__ inline void bwd_q_tiles(int j, int lq, int lk, bool causal, int* begin, int* end) {
-  const int nq = (lq + kBwdBM - 1) / kBwdBM;
+__host__ __device__ inline void bwd_q_tiles(int j, int lq, int lk, bool causal, int* begin, int* end,
+                                            int bm = kBwdBM) {
+  const int nq = (lq + bm - 1) / bm;
   *end = nq;
   *begin = 0;
   if (lk <= 0 || lq <= 0) {
@@ -186,7 +188,7 @@ __host__ __device__ inline void bwd_q_tiles(int j, int lq, int lk, bool causal, 
   if (causal) {
     long long first = static_cast<long long>(j) * kBwdBN - (lk - lq);
     if (first < 0) first = 0;
-    *begin = first >= lq ? nq : static_cast<int>(first / kBwdBM);
+    *begin = first >= lq ? nq : static_cast<int>(first / bm);
   }
 }
 

@@ -146,6 +146,9 @@ __device__ __forceinline__ void bulk_wait_group_read0() {
 __device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // All but the most recent bulk async-group have completed.
 __device__ __forceinline__ void bulk_wait_group1() { asm volatile("cp.async.bulk.wait_group 1;" ::: "memory"); }
+// All but the two (four) most recent bulk async-groups have completed.
+__device__ __forceinline__ void bulk_wait_group2() { asm volatile("cp.async.bulk.wait_group 2;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_group4() { asm volatile("cp.async.bulk.wait_group 4;" ::: "memory"); }
 // Orders this thread's generic-proxy and async-proxy (bulk copy) accesses to
 // global memory with respect to each other.
 __device__ __forceinline__ void fence_proxy_async_global() {
