@@ -253,8 +253,7 @@ typedef struct {
  *    128-row tile, so each key/value tile is read once per group;
  *  - each tile's key tiles are divided into num_splits ranges processed in
  *    parallel; each writes a normalised partial output and its logsumexp
- *    into the workspace (fp32), and the CTA that finishes a tile's last
- *    range merges them, counting finished ranges in the workspace
+ *    into the workspace (fp32) and a combine kernel merges them
  *    (num_splits = 1 writes out directly).
  * head_dim 64 or 128 (FA_ERR_UNSUPPORTED otherwise). The workspace must
  * hold fa_varlen_fwd_splitkv_workspace_size(...) bytes (0 = invalid sizes).

@@ -286,10 +286,9 @@ fa_status_t run_bwd(const void* dout, const void* q, const void* k, const void* 
 }
 
 // Workspace of the split-KV forward: header, per-sequence offsets and the
-// (sequence, token tile) list, then the split partials and, per (pair,
-// key/value head) unit, the count of its finished splits.
+// (sequence, token tile) list, then the split partials.
 struct DecodeLayout {
-  size_t seq_off, pairs, opart, lpart, done, total;
+  size_t seq_off, pairs, opart, lpart, total;
   int max_pairs, tq;
 };
 DecodeLayout decode_layout(int batch, int total_q, int H, int Hk, int D, int splits) {
@@ -307,8 +306,6 @@ DecodeLayout decode_layout(int batch, int total_q, int H, int Hk, int D, int spl
     off = fa::align_up(off + sizeof(float) * splits * rows * D, 256);
     L.lpart = off;
     off = fa::align_up(off + sizeof(float) * splits * rows, 256);
-    L.done = off;
-    off = fa::align_up(off + sizeof(uint32_t) * 4 * static_cast<size_t>(L.max_pairs) * Hk, 256);
   }
   L.total = off;
   return L;
@@ -388,10 +385,6 @@ fa_status_t fa_varlen_fwd_splitkv(const void* q, const void* k, const void* v, c
   t_events.next = 0;
   fa::SchedArgs sa{cu_seqlens_q, keys, batch, total_q, total_k, max_seqlen_q, max_seqlen_k,
                    causal ? 1 : 0, 0, L.tq, 0, workspace, L.seq_off, L.pairs, L.max_pairs};
-  if (num_splits > 1) {  // the split counters start every call at zero
-    sa.zero_words = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + L.done);
-    sa.n_zero = 4 * L.max_pairs * num_heads_k;  // one count per unit and 32-row quarter
-  }
   if (timed_launch(stream, [&] { return fa::launch_sched_prep(sa, stream); }) != cudaSuccess) return FA_ERR_CUDA;
   if (total_q == 0) return FA_OK;
 
@@ -417,7 +410,6 @@ fa_status_t fa_varlen_fwd_splitkv(const void* q, const void* k, const void* v, c
   char* ws = static_cast<char*>(workspace);
   d.opart = num_splits > 1 ? reinterpret_cast<float*>(ws + L.opart) : nullptr;
   d.lpart = num_splits > 1 ? reinterpret_cast<float*>(ws + L.lpart) : nullptr;
-  d.unit_done = num_splits > 1 ? reinterpret_cast<uint32_t*>(ws + L.done) : nullptr;
   d.workspace = workspace;
   d.pairs_offset = L.pairs;
   d.H = num_heads;
@@ -431,7 +423,8 @@ fa_status_t fa_varlen_fwd_splitkv(const void* q, const void* k, const void* v, c
   d.scale_log2 = softmax_scale * 1.4426950408889634f;
   d.grid = static_cast<int>(items < sms ? items : sms);
   d.wait_ns = t_hooks.wait_ns;
-  if (timed_launch(stream, [&] { return fa::launch_decode(d, tq3, tk, tv, stream); }) != cudaSuccess)
+  if (timed_launch(stream, [&] { return fa::launch_decode(d, tq3, tk, tv, stream); }) != cudaSuccess ||
+      timed_launch(stream, [&] { return fa::launch_decode_combine(d, stream); }) != cudaSuccess)
     return FA_ERR_CUDA;
   return FA_OK;
 }

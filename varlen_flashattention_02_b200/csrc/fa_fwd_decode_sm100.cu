@@ -17,8 +17,7 @@
 //    group;
 //  * the key tiles of an item are split into `splits` ranges processed by
 //    different CTAs; each writes its normalised partial output and its
-//    logsumexp, and whichever CTA finishes a unit's last split merges them
-//    (an arrival count per unit and warp; no separate combine launch):
+//    logsumexp, and the combine kernel merges them:
 //      lse = log sum_s exp(lse_s),  out = sum_s exp(lse_s - lse) * out_s.
 // Roles: one warp loads Q and K (and hands out items), one loads V, one
 // issues the MMAs, four (one thread per tile row) run the softmax and the
@@ -70,56 +69,6 @@ struct Item {
   SeqInfo s;
   int j0, j1;           // key tiles [j0, j1) of this split
 };
-
-// out = sum_s exp(lse_s - lse) * out_s with lse = log sum_s exp(lse_s), for
-// one (query token, head) row; lse_at: its index in the [H, total_q]
-// logsumexp array. Partial rows are fp32 and already normalised.
-template <int D>
-__device__ __forceinline__ void combine_row(const DecodeArgs& a, size_t orow, size_t lse_at) {
-  const size_t stride = static_cast<size_t>(a.total_q) * a.H;
-  const volatile float* lp = a.lpart;
-  float mx = -INFINITY;
-  for (int s = 0; s < a.splits; ++s) mx = fmaxf(mx, lp[s * stride + orow]);
-  float sum = 0.f;
-  if (mx != -INFINITY)
-    for (int s = 0; s < a.splits; ++s) {
-      const float ls = lp[s * stride + orow];
-      if (ls != -INFINITY) sum += __expf(ls - mx);
-    }
-  const float inv = sum > 0.f ? 1.f / sum : 0.f;
-  uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + orow * D);
-#pragma unroll 1
-  for (int c = 0; c < D / 32; ++c) {
-    float acc[32];
-#pragma unroll
-    for (int e = 0; e < 32; ++e) acc[e] = 0.f;
-    if (mx != -INFINITY)
-      for (int s = 0; s < a.splits; ++s) {
-        const float ls = lp[s * stride + orow];
-        if (ls == -INFINITY) continue;
-        const float f = __expf(ls - mx) * inv;
-        const volatile float4* src = reinterpret_cast<const volatile float4*>(a.opart + (s * stride + orow) * D) + c * 8;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float4 x = make_float4(src[e].x, src[e].y, src[e].z, src[e].w);
-          acc[4 * e + 0] = fmaf(f, x.x, acc[4 * e + 0]);
-          acc[4 * e + 1] = fmaf(f, x.y, acc[4 * e + 1]);
-          acc[4 * e + 2] = fmaf(f, x.z, acc[4 * e + 2]);
-          acc[4 * e + 3] = fmaf(f, x.w, acc[4 * e + 3]);
-        }
-      }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      uint4 w;
-      w.x = pack_bf16x2(acc[8 * e + 0], acc[8 * e + 1]);
-      w.y = pack_bf16x2(acc[8 * e + 2], acc[8 * e + 3]);
-      w.z = pack_bf16x2(acc[8 * e + 4], acc[8 * e + 5]);
-      w.w = pack_bf16x2(acc[8 * e + 6], acc[8 * e + 7]);
-      dst[c * 4 + e] = w;
-    }
-  }
-  a.lse[lse_at] = sum > 0.f ? mx + logf(sum) : -INFINITY;
-}
 
 template <int KL>
 __device__ __forceinline__ Item get_item(const DecodeArgs& a, const int2* pairs, int idx) {
@@ -468,22 +417,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           else
             a.lse[static_cast<size_t>(h) * a.total_q + it.s.q0 + r] = lse_nat;
         }
-        // Split partials: the warp that finishes the last of a unit's splits
-        // for its 32 rows merges them (each warp counts on its own, so no
-        // warp ever waits for another). Every split of a unit has the same
-        // rows, so warps without a row to write take no part.
-        if (split_out && __any_sync(0xffffffffu, row_ok)) {
-          __threadfence();  // this lane's partial row is visible before the count moves
-          __syncwarp();
-          uint32_t* cnt = a.unit_done + static_cast<size_t>(idx / a.splits) * 4 + (warp & 3);
-          uint32_t prev = 0;
-          if (lane == 0) prev = atomicAdd(cnt, 1u);
-          prev = __shfl_sync(0xffffffffu, prev, 0);
-          if (prev == static_cast<uint32_t>(a.splits - 1)) {
-            __threadfence();  // the other splits' rows, published before their counts moved
-            if (row_ok) combine_row<D>(a, orow, static_cast<size_t>(h) * a.total_q + it.s.q0 + r);
-          }
-        }
       }
       if (nk > 0) {
         tc_fence_before();
@@ -501,6 +434,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// out = sum_s exp(lse_s - lse) * out_s with lse = log sum_s exp(lse_s), one
+// warp per (query token, head) row.
+template <int D>
+__global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeArgs a) {
+  const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long rows = static_cast<long long>(a.total_q) * a.H;
+  if (w >= rows) return;
+  const size_t stride = static_cast<size_t>(rows);
+  float mx = -INFINITY;
+  for (int s = 0; s < a.splits; ++s) mx = fmaxf(mx, a.lpart[s * stride + w]);
+  constexpr int E = D / 32;  // channels per lane
+  float acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  float sum = 0.f;
+  if (mx != -INFINITY) {
+    for (int s = 0; s < a.splits; ++s) {
+      const float ls = a.lpart[s * stride + w];
+      if (ls == -INFINITY) continue;
+      const float f = __expf(ls - mx);
+      sum += f;
+      const float* src = a.opart + (s * stride + w) * D + lane * E;
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = fmaf(f, src[e], acc[e]);
+    }
+  }
+  const float inv = sum > 0.f ? 1.f / sum : 0.f;
+  __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + w * D + lane * E;
+#pragma unroll
+  for (int e = 0; e < E; e += 2) *reinterpret_cast<uint32_t*>(dst + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+  if (lane == 0) {
+    const long long row = w / a.H;
+    const int h = static_cast<int>(w - row * a.H);
+    a.lse[static_cast<size_t>(h) * a.total_q + row] = sum > 0.f ? mx + logf(sum) : -INFINITY;
   }
 }
 
@@ -532,6 +503,17 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tq, const CUte
     case kKeysSlots: return launch_layout<kKeysSlots>(a, tq, tk, tv, stream);
     default: return launch_layout<kKeysPacked>(a, tq, tk, tv, stream);
   }
+}
+
+cudaError_t launch_decode_combine(const DecodeArgs& a, cudaStream_t stream) {
+  const long long warps = static_cast<long long>(a.total_q) * a.H;
+  const unsigned blocks = static_cast<unsigned>((warps + 7) / 8);
+  if (blocks == 0 || a.splits <= 1) return cudaSuccess;
+  if (a.D == 64)
+    decode_combine_kernel<64><<<blocks, 256, 0, stream>>>(a);
+  else
+    decode_combine_kernel<128><<<blocks, 256, 0, stream>>>(a);
+  return cudaGetLastError();
 }
 
 }  // namespace fa

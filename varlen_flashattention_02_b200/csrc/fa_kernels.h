@@ -25,8 +25,6 @@ struct SchedArgs {
   void* workspace;
   size_t seq_off_offset, pairs_offset;
   int max_pairs;
-  uint32_t* zero_words;  // optional: per-call counters the kernel sets to 0 (null: none)
-  int n_zero;
 };
 cudaError_t launch_sched_prep(const SchedArgs& a, cudaStream_t stream);
 
@@ -58,8 +56,8 @@ cudaError_t launch_fwd_d256(const FwdArgs& a, const CUtensorMap& tm_q, const CUt
 // the rows of one tile (the decode path): an item is (sequence, key/value
 // head, tile of tq = 128 / group query tokens, key split); its 128 rows are
 // (token, head-in-group) pairs. With splits > 1 every split writes a
-// normalised partial output and its logsumexp (fp32), and the CTA that
-// finishes a unit's last split merges them into out and lse. tm_q3: 3-D map over q as [tokens, H, D] with box (64, group,
+// normalised partial output and its logsumexp (fp32) and the combine kernel
+// merges them. tm_q3: 3-D map over q as [tokens, H, D] with box (64, group,
 // tq); tm_k / tm_v as for launch_fwd.
 struct DecodeArgs {
   const int32_t* cu_q;
@@ -68,7 +66,6 @@ struct DecodeArgs {
   float* lse;       // fp32 [H, total_q]
   float* opart;     // fp32 [splits, total_q * H, D] (splits > 1)
   float* lpart;     // fp32 [splits, total_q * H]    (splits > 1)
-  uint32_t* unit_done;  // splits > 1: [units, 4] finished splits per unit and 32-row quarter (zeroed by the scheduler)
   void* workspace;  // header + pairs
   size_t pairs_offset;
   int H, Hk, group, D, total_q;
@@ -81,6 +78,7 @@ struct DecodeArgs {
 };
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tm_q3, const CUtensorMap& tm_k,
                           const CUtensorMap& tm_v, cudaStream_t stream);
+cudaError_t launch_decode_combine(const DecodeArgs& a, cudaStream_t stream);
 
 struct BwdArgs {
   const int32_t* cu_q;

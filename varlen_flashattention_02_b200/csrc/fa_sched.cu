@@ -94,7 +94,6 @@ __global__ void __launch_bounds__(kThreads) sched_prep_kernel(SchedArgs a) {
     if (!cache && (a.keys.cu_k[0] != 0 || a.keys.cu_k[a.batch] != a.total_k)) s_err = 1;
   }
   for (int i = tid; i < kBins; i += kThreads) s_hist[i] = 0;
-  for (int i = tid; i < a.n_zero; i += kThreads) a.zero_words[i] = 0u;
   __syncthreads();
   for (int b = tid; b < a.batch; b += kThreads) {
     const int lq = a.cu_q[b + 1] - a.cu_q[b];
