@@ -112,7 +112,10 @@ __device__ __forceinline__ Item get_item(const BwdArgs& a, const int2* pairs, in
 
 struct Bars {
   uint64_t kv_full, kv_empty;
-  uint64_t qdo_full[3], qdo_empty[3];
+  // Q and dO halves of each stage, filled and released separately: the
+  // drain hands the Q half back as soon as the first half of the step's dQ
+  // reduction has read it, so the next Q load starts early.
+  uint64_t q_full[3], q_empty[3], do_full[3], do_empty[3];
   uint64_t s_full, dp_full;   // S^T, dP^T of the step in TMEM
   uint64_t p_full, ds_full;   // P^T (TMEM), dS^T (TMEM and shared) written
   uint64_t dq_full, dq_free;  // dQ^T in TMEM; read out by the drain group
@@ -214,8 +217,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars.kv_full, 1);
     mbar_init(&bars.kv_empty, 1);
     for (int i = 0; i < NQ; ++i) {
-      mbar_init(&bars.qdo_full[i], 1);
-      mbar_init(&bars.qdo_empty[i], 1);
+      mbar_init(&bars.q_full[i], 1);
+      mbar_init(&bars.q_empty[i], 1);
+      mbar_init(&bars.do_full[i], 1);
+      mbar_init(&bars.do_empty[i], 1);
       mbar_init(&bars.ld_full[i], 2);
       mbar_init(&bars.ld_empty[i], 8);
     }
@@ -266,16 +271,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t m = 0, p = 0, ni = 0;
       auto load_qdo = [&](const Item& it, int s) -> bool {
         const int st = p % NQ;
-        if (p >= NQ && !wait_bar(&bars.qdo_empty[st], ((p / NQ) - 1) & 1, ab)) return false;
         const Step sp = item_step(it, s);
         const int qrow = it.s.q0 + sp.t * BM;
         uint8_t* sq = smem + L::kQdo + 2 * st * L::kQTile;
         uint8_t* sdo = sq + L::kQTile;
-        mbar_arrive_expect_tx(&bars.qdo_full[st], 2 * L::kQTile);
-        for (int c = 0; c < L::kChunks; ++c) {
-          tma_load_2d(&tm_q, &bars.qdo_full[st], sq + c * L::kQChunk, sp.h * D + c * 64, qrow);
-          tma_load_2d(&tm_do, &bars.qdo_full[st], sdo + c * L::kQChunk, sp.h * D + c * 64, qrow);
-        }
+        const uint32_t ph = ((p / NQ) - 1) & 1;
+        if (p >= NQ && !wait_bar(&bars.q_empty[st], ph, ab)) return false;
+        mbar_arrive_expect_tx(&bars.q_full[st], L::kQTile);
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_2d(&tm_q, &bars.q_full[st], sq + c * L::kQChunk, sp.h * D + c * 64, qrow);
+        if (p >= NQ && !wait_bar(&bars.do_empty[st], ph, ab)) return false;
+        mbar_arrive_expect_tx(&bars.do_full[st], L::kQTile);
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_2d(&tm_do, &bars.do_full[st], sdo + c * L::kQChunk, sp.h * D + c * 64, qrow);
         ++p;
         return true;
       };
@@ -311,7 +319,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     producer_done:
       if (m > 0) wait_bar_final(&bars.kv_full, (m - 1) & 1, ab);
-      for (uint32_t i = (p > NQ ? p - NQ : 0); i < p; ++i) wait_bar_final(&bars.qdo_full[i % NQ], (i / NQ) & 1, ab);
+      for (uint32_t i = (p > NQ ? p - NQ : 0); i < p; ++i) {
+        wait_bar_final(&bars.q_full[i % NQ], (i / NQ) & 1, ab);
+        wait_bar_final(&bars.do_full[i % NQ], (i / NQ) & 1, ab);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -351,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // that the compiler does not keep every offset form in registers.
         const uint64_t q_kmaj = opaque_u64(qdo_kmaj0) + static_cast<uint64_t>((2 * qs * L::kQTile) >> 4);
         const uint64_t q_mn = opaque_u64(qdo_mn0) + static_cast<uint64_t>((2 * qs * L::kQTile) >> 4);
-        if (!wait_bar_warp(&bars.qdo_full[qs], (p / NQ) & 1, ab)) goto mma_done;
+        if (!wait_bar_warp(&bars.q_full[qs], (p / NQ) & 1, ab)) goto mma_done;
         tc_fence_after();
         if (elect_one()) {
 #pragma unroll
@@ -365,6 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // dP^T goes where the previous step's dQ^T is until the drain group
         // has read it out.
         if (p > 0 && !wait_bar_warp(&bars.dq_free, (p - 1) & 1, ab)) goto mma_done;
+        if (!wait_bar_warp(&bars.do_full[qs], (p / NQ) & 1, ab)) goto mma_done;
         tc_fence_after();
         if (elect_one()) {
 #pragma unroll
@@ -599,14 +611,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!named_bar_and(1, 128, wait_bar(&bars.dq_full, p & 1, ab))) goto drain_done;
         tc_fence_after();
         // Every MMA of the step has completed, so its Q/dO stage is free:
-        // the step's fp32 dQ tile (128 x D) is staged there and leaves with
-        // one bulk reduction (128 consecutive rows of one head are one
-        // contiguous block of the head-major accumulator).
+        // the step's fp32 dQ tile (128 x D) is staged there, queries 0-63
+        // over the Q half and 64-127 over the dO half (128 consecutive rows
+        // of one head are one contiguous block of the head-major
+        // accumulator). Each half leaves with its own bulk reduction as soon
+        // as it is staged, and the Q half goes back to the loader once its
+        // reduction has read it, so the next Q tile loads while the second
+        // half is still being reduced. The deterministic mode adds the whole
+        // tile at once, in its query tile's turn.
         qs = static_cast<int>(p % NQ);
         float* stage = reinterpret_cast<float*>(smem + L::kQdo + 2 * qs * L::kQTile);
         const Step sp = item_step(it, s);
         const size_t q0 = static_cast<size_t>(it.s.q0) + static_cast<size_t>(sp.t) * BM;
         uint32_t* cnt = qcount + static_cast<size_t>(sp.h) * a.tq_pad + q0;
+        float* gdq = dqacc + (static_cast<size_t>(sp.h) * a.tq_pad + q0) * D;
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
           uint32_t v0[32], v1[32];
@@ -618,25 +636,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars.dq_free);
           }
+          float* st = stage + h * 64 * D;
           if (t < D) {
-            float* st = stage + h * 64 * D;
 #pragma unroll
             for (int e = 0; e < 32; ++e) st[e * D + t] = __uint_as_float(v0[e]);
 #pragma unroll
             for (int e = 0; e < 32; ++e) st[(32 + e) * D + t] = __uint_as_float(v1[e]);
           }
+          if (!DET) {
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            if (t == 0 && !*ab.flag) {
+              bulk_reduce_add_f32(gdq + h * 64 * D, st, 64 * D * 4);
+              bulk_commit_group();
+            }
+          }
         }
-        fence_proxy_async_smem();
-        named_bar_sync(1, 128);
-        if (t == 0) {
-          // Deterministic mode: this query tile's turn first (a wait that
-          // runs out raises the abort flag, and nothing more is added).
-          if (DET) wait_dq_turn(cnt, static_cast<uint32_t>(it.j), ab);
-          if (!*ab.flag) {
-            if (DET) fence_proxy_async_global();
-            bulk_reduce_add_f32(dqacc + (static_cast<size_t>(sp.h) * a.tq_pad + q0) * D, stage, BM * D * 4);
-            bulk_commit_group();
-            if (DET) {
+        if (DET) {
+          fence_proxy_async_smem();
+          named_bar_sync(1, 128);
+          if (t == 0) {
+            // This query tile's turn first (a wait that runs out raises the
+            // abort flag, and nothing more is added).
+            wait_dq_turn(cnt, static_cast<uint32_t>(it.j), ab);
+            if (!*ab.flag) {
+              fence_proxy_async_global();
+              bulk_reduce_add_f32(gdq, stage, BM * D * 4);
+              bulk_commit_group();
               // Pass the previous step's turn on once its addition has been
               // performed (it was issued a step ago, so this rarely waits);
               // this step's turn passes on at the next step or item end.
@@ -648,12 +674,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               det_prev = cnt;
             }
           }
-          // Hand the stage back to the loader once the reduction has read
-          // it (an item's last stage serves the dK/dV stores first).
-          if (s + 1 < it.n) {
+        }
+        // Hand the stage back to the loader half by half once the reductions
+        // have read it (an item's last stage serves the dK/dV stores first).
+        if (t == 0 && s + 1 < it.n) {
+          if (DET)
             bulk_wait_group_read0();
-            mbar_arrive(&bars.qdo_empty[qs]);
-          }
+          else
+            bulk_wait_group_read1();
+          mbar_arrive(&bars.q_empty[qs]);
+          bulk_wait_group_read0();
+          mbar_arrive(&bars.do_empty[qs]);
         }
       }
       if (DET && t == 0 && det_prev) {
@@ -715,7 +746,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (t == 0) {
           bulk_wait_group_read0();  // the stores (and the last reduction) have read the stage
-          mbar_arrive(&bars.qdo_empty[qs]);
+          mbar_arrive(&bars.q_empty[qs]);
+          mbar_arrive(&bars.do_empty[qs]);
         }
       }
       ++m;
