@@ -96,6 +96,12 @@ cudaError_t timed_launch(cudaStream_t stream, F&& launch) {
   return cudaSuccess;
 }
 
+// Each kernel of a call after the work-list kernel is launched as a
+// programmatic dependent of the one before it (its launch and prologue
+// overlap that kernel's tail), except while the per-kernel timing hook is
+// on: its events sit between the launches and time each kernel alone.
+bool chained() { return t_events.events == nullptr; }
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int sm_count() {
@@ -179,6 +185,7 @@ fa_status_t run_fwd(const void* q, const void* k, const void* v, const int32_t* 
   fa_args.grid = static_cast<int>(items < sms ? items : sms);
   fa_args.wait_ns = t_hooks.wait_ns;
   fa_args.withhold_v0 = head_dim == 256 ? 0 : t_hooks.withhold_v0;
+  fa_args.chained = chained() ? 1 : 0;
   auto launch = head_dim == 256 ? fa::launch_fwd_d256 : fa::launch_fwd;
   if (timed_launch(stream, [&] { return launch(fa_args, tq, tk, tv, stream); }) != cudaSuccess) return FA_ERR_CUDA;
   return FA_OK;
@@ -274,6 +281,7 @@ fa_status_t run_bwd(const void* dout, const void* q, const void* k, const void* 
   b.scale_log2 = softmax_scale * 1.4426950408889634f;
   b.grid = static_cast<int>(items < sms ? items : sms);
   b.wait_ns = t_hooks.wait_ns;
+  b.chained = chained() ? 1 : 0;
   if (timed_launch(stream, [&] { return fa::launch_bwd_preprocess(b, stream); }) != cudaSuccess ||
       timed_launch(stream,
                    [&] {
@@ -423,6 +431,7 @@ fa_status_t fa_varlen_fwd_splitkv(const void* q, const void* k, const void* v, c
   d.scale_log2 = softmax_scale * 1.4426950408889634f;
   d.grid = static_cast<int>(items < sms ? items : sms);
   d.wait_ns = t_hooks.wait_ns;
+  d.chained = chained() ? 1 : 0;
   if (timed_launch(stream, [&] { return fa::launch_decode(d, tq3, tk, tv, stream); }) != cudaSuccess ||
       timed_launch(stream, [&] { return fa::launch_decode_combine(d, stream); }) != cudaSuccess)
     return FA_ERR_CUDA;

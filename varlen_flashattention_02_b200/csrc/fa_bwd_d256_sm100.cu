@@ -152,6 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int2* pairs = reinterpret_cast<const int2*>(static_cast<const char*>(a.workspace) + a.pairs_offset);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if ((smem_u32(smem) & 1023u) != 0) {  // swizzled tiles need a 1024-byte-aligned base
+    griddep_wait();
     if (threadIdx.x == 0) atomicCAS(&hdr->status, 0u, static_cast<uint32_t>(FA_ERR_CUDA));
     return;
   }
@@ -185,6 +186,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&bars.tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  // The kernel launched behind this one may be scheduled now (it waits for
+  // this grid before it touches any of its results).
+  griddep_launch_dependents();
+  // Everything above is local to the CTA; the work list, the inputs and the
+  // outputs are touched only after the kernel before this one has finished.
+  griddep_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -474,6 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* qcount = reinterpret_cast<uint32_t*>(static_cast<char*>(a.workspace) + a.qcount_offset);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if ((smem_u32(smem) & 1023u) != 0) {
+    griddep_wait();
     if (threadIdx.x == 0) atomicCAS(&hdr->status, 0u, static_cast<uint32_t>(FA_ERR_CUDA));
     return;
   }
@@ -511,6 +519,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&bars.tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  // The kernel launched behind this one may be scheduled now (it waits for
+  // this grid before it touches any of its results).
+  griddep_launch_dependents();
+  // Everything above is local to the CTA; the work list, the inputs and the
+  // outputs are touched only after the kernel before this one has finished.
+  griddep_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -883,13 +897,13 @@ cudaError_t launch_bwd_d256(const BwdArgs& a, const BwdMapsD256& m, cudaStream_t
   cudaError_t e;
   auto k1 = a.causal ? dv::kernel<true> : dv::kernel<false>;
   if ((e = prepare(k1, dv::kBytes)) != cudaSuccess) return e;
-  k1<<<a.grid, dv::kThreads, dv::kBytes, stream>>>(m.q128, m.k, m.do128, a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = launch_kernel(k1, a.grid, dv::kThreads, dv::kBytes, stream, a.chained != 0, m.q128, m.k, m.do128, a)) !=
+      cudaSuccess)
+    return e;
   auto k2 = a.causal ? (a.deterministic ? dkq::kernel<true, true> : dkq::kernel<true, false>)
                      : (a.deterministic ? dkq::kernel<false, true> : dkq::kernel<false, false>);
   if ((e = prepare(k2, dkq::kBytes)) != cudaSuccess) return e;
-  k2<<<a.grid, dkq::kThreads, dkq::kBytes, stream>>>(m.q64, m.k, m.v, m.do64, a);
-  return cudaGetLastError();
+  return launch_kernel(k2, a.grid, dkq::kThreads, dkq::kBytes, stream, a.chained != 0, m.q64, m.k, m.v, m.do64, a);
 }
 
 }  // namespace fa

@@ -209,6 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // starts aligned on this architecture; if it ever did not, the call
   // reports an error instead of computing garbage.
   if ((smem_u32(smem) & 1023u) != 0) {
+    griddep_wait();
     if (threadIdx.x == 0) atomicCAS(&hdr->status, 0u, static_cast<uint32_t>(FA_ERR_CUDA));
     return;
   }
@@ -253,6 +254,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&bars.tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  // The kernel launched behind this one may be scheduled now (it waits for
+  // this grid before it touches any of its results).
+  griddep_launch_dependents();
+  // Everything above is local to the CTA; the work list, the inputs and the
+  // outputs are touched only after the kernel before this one has finished.
+  griddep_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -790,7 +797,7 @@ struct Words<4> {
 
 // Dv[h, r] = sum_c dO[r, h, c] * O[r, h, c] in fp32, and dQacc[h, r, :] = 0.
 template <int D>
-__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdArgs a) {
+__device__ __forceinline__ void preprocess_rows(const BwdArgs& a) {
   constexpr int E = D / 32;  // bf16 elements per lane: 2, 4 or 8 (4, 8 or 16 bytes)
   using V = typename Words<E / 2>::T;
   const long long units = static_cast<long long>(a.total_q) * a.H;
@@ -845,9 +852,21 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdArgs a) {
   }
 }
 
+// Reads only the caller's tensors and writes only its own workspace regions,
+// so it runs while the work-list kernel before it is still working; it waits
+// for that kernel before it exits, so that its own completion, which the
+// main kernel waits for, implies the work list's.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const BwdArgs a) {
+  griddep_launch_dependents();
+  preprocess_rows<D>(a);
+  griddep_wait();
+}
+
 // dQ[r, h, :] = bf16(scale * dQacc[h, r, :]).
 template <int D>
 __global__ void __launch_bounds__(256) bwd_convert_kernel(const BwdArgs a) {
+  griddep_wait();  // the accumulator comes from the main kernel before this one
   constexpr int E = D / 32;          // fp32 elements per lane: 2, 4 or 8
   constexpr int W = E < 4 ? E : 4;   // words per vector load
   constexpr int NL = E / W;          // vector loads per lane and unit
@@ -886,8 +905,8 @@ cudaError_t launch_main(const BwdArgs& a, const BwdMaps& m, cudaStream_t stream)
   auto kern = bwd_kernel<D, CAUSAL, DET>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
   if (e != cudaSuccess) return e;
-  kern<<<a.grid, kThreads, L::kBytes, stream>>>(m.q, m.k, m.v, m.dout, m.dk, m.dv, a);
-  return cudaGetLastError();
+  return launch_kernel(kern, a.grid, kThreads, L::kBytes, stream, a.chained != 0, m.q, m.k, m.v, m.dout, m.dk, m.dv,
+                       a);
 }
 
 }  // namespace
@@ -896,13 +915,8 @@ cudaError_t launch_bwd_preprocess(const BwdArgs& a, cudaStream_t stream) {
   const long long warps = (static_cast<long long>(a.total_q) * a.H + kUnits - 1) / kUnits;
   const unsigned blocks = static_cast<unsigned>((warps + 7) / 8);
   if (blocks == 0) return cudaSuccess;
-  if (a.D == 64)
-    bwd_preprocess_kernel<64><<<blocks, 256, 0, stream>>>(a);
-  else if (a.D == 128)
-    bwd_preprocess_kernel<128><<<blocks, 256, 0, stream>>>(a);
-  else
-    bwd_preprocess_kernel<256><<<blocks, 256, 0, stream>>>(a);
-  return cudaGetLastError();
+  auto kern = a.D == 64 ? bwd_preprocess_kernel<64> : a.D == 128 ? bwd_preprocess_kernel<128> : bwd_preprocess_kernel<256>;
+  return launch_kernel(kern, blocks, 256, 0, stream, a.chained != 0, a);
 }
 
 template <bool DET>
@@ -920,13 +934,8 @@ cudaError_t launch_bwd_convert(const BwdArgs& a, cudaStream_t stream) {
   const long long warps = (static_cast<long long>(a.total_q) * a.H + kUnits - 1) / kUnits;
   const unsigned blocks = static_cast<unsigned>((warps + 7) / 8);
   if (blocks == 0) return cudaSuccess;
-  if (a.D == 64)
-    bwd_convert_kernel<64><<<blocks, 256, 0, stream>>>(a);
-  else if (a.D == 128)
-    bwd_convert_kernel<128><<<blocks, 256, 0, stream>>>(a);
-  else
-    bwd_convert_kernel<256><<<blocks, 256, 0, stream>>>(a);
-  return cudaGetLastError();
+  auto kern = a.D == 64 ? bwd_convert_kernel<64> : a.D == 128 ? bwd_convert_kernel<128> : bwd_convert_kernel<256>;
+  return launch_kernel(kern, blocks, 256, 0, stream, a.chained != 0, a);
 }
 
 }  // namespace fa

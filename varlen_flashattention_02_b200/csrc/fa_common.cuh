@@ -320,4 +320,26 @@ __device__ __forceinline__ int consume_item(ItemRing& r, uint32_t& n, int& slot,
   return *reinterpret_cast<volatile int*>(&r.idx[slot]);
 }
 
+// kern<<<grid, block, smem, stream>>>(args...). With `chained` the grid is a
+// programmatic dependent of the kernel before it in the stream: it may be
+// scheduled (and run its prologue: barriers, tensor memory, descriptor
+// prefetch) while that kernel still runs, and every one of its threads
+// executes griddep_wait() before it reads or writes memory that kernel (or
+// anything before it) touches.
+template <class... KArgs, class... Args>
+inline cudaError_t launch_kernel(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                                 cudaStream_t stream, bool chained, const Args&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr = {};
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = chained ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 }  // namespace fa

@@ -124,6 +124,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&bars.tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  // Everything above is local to the CTA; the work list, the inputs and the
+  // outputs are touched only after the work-list kernel has finished.
+  griddep_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -422,8 +425,7 @@ cudaError_t launch_one(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMa
   auto kern = fwd_d256_kernel<CAUSAL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   if (e != cudaSuccess) return e;
-  kern<<<a.grid, kThreads, kSmemAlloc, stream>>>(tq, tk, tv, a);
-  return cudaGetLastError();
+  return launch_kernel(kern, a.grid, kThreads, kSmemAlloc, stream, a.chained != 0, tq, tk, tv, a);
 }
 
 }  // namespace

@@ -132,6 +132,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&bars.tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  // The kernel launched behind this one may be scheduled now (it waits for
+  // this grid before it touches any of its results).
+  griddep_launch_dependents();
+  // Everything above is local to the CTA; the work list, the inputs and the
+  // outputs are touched only after the kernel before this one has finished.
+  griddep_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -438,31 +444,53 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // out = sum_s exp(lse_s - lse) * out_s with lse = log sum_s exp(lse_s), one
-// warp per (query token, head) row.
+// warp per (query token, head) row. The splits are handled 32 at a time:
+// lane s loads split s's logsumexp, the maximum and the sum of the weights
+// are warp reductions, and the partial outputs (a 16-byte vector per lane at
+// d = 128) are loaded back to back, so that the latency of the partials is
+// paid about once instead of once per split. A split that saw no key
+// (logsumexp -inf) has weight 0 and its partial, which it did not write, is
+// not used.
 template <int D>
 __global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeArgs a) {
+  griddep_wait();  // the partials come from the decode kernel before this one
   const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const long long rows = static_cast<long long>(a.total_q) * a.H;
   if (w >= rows) return;
   const size_t stride = static_cast<size_t>(rows);
-  float mx = -INFINITY;
-  for (int s = 0; s < a.splits; ++s) mx = fmaxf(mx, a.lpart[s * stride + w]);
   constexpr int E = D / 32;  // channels per lane
+  using Vec = typename std::conditional<E == 4, float4, float2>::type;
+  static_assert(E == 2 || E == 4, "d = 64 or 128");
+  float mx = -INFINITY;
+  for (int s0 = 0; s0 < a.splits; s0 += 32)
+    if (s0 + lane < a.splits) mx = fmaxf(mx, a.lpart[(s0 + lane) * stride + w]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   float acc[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.f;
   float sum = 0.f;
   if (mx != -INFINITY) {
-    for (int s = 0; s < a.splits; ++s) {
-      const float ls = a.lpart[s * stride + w];
-      if (ls == -INFINITY) continue;
-      const float f = __expf(ls - mx);
+    for (int s0 = 0; s0 < a.splits; s0 += 32) {
+      const float ls = s0 + lane < a.splits ? a.lpart[(s0 + lane) * stride + w] : -INFINITY;
+      const float f = ls == -INFINITY ? 0.f : __expf(ls - mx);
       sum += f;
-      const float* src = a.opart + (s * stride + w) * D + lane * E;
+      const int n = a.splits - s0 < 32 ? a.splits - s0 : 32;
+      const float* src = a.opart + ((static_cast<size_t>(s0) * stride + w) * D + lane * E);
+#pragma unroll 8
+      for (int i = 0; i < n; ++i) {
+        const float fi = __shfl_sync(0xffffffffu, f, i);
+        const Vec x = *reinterpret_cast<const Vec*>(src + static_cast<size_t>(i) * stride * D);
+        const float* xv = reinterpret_cast<const float*>(&x);
+        if (fi != 0.f) {
 #pragma unroll
-      for (int e = 0; e < E; ++e) acc[e] = fmaf(f, src[e], acc[e]);
+          for (int e = 0; e < E; ++e) acc[e] = fmaf(fi, xv[e], acc[e]);
+        }
+      }
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   }
   const float inv = sum > 0.f ? 1.f / sum : 0.f;
   __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + w * D + lane * E;
@@ -482,8 +510,7 @@ cudaError_t launch_one(const DecodeArgs& a, const CUtensorMap& tq, const CUtenso
   auto kern = decode_kernel<D, CAUSAL, KL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
-  kern<<<a.grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
-  return cudaGetLastError();
+  return launch_kernel(kern, a.grid, kThreads, L::kAlloc, stream, a.chained != 0, tq, tk, tv, a);
 }
 
 template <int KL>
@@ -509,11 +536,8 @@ cudaError_t launch_decode_combine(const DecodeArgs& a, cudaStream_t stream) {
   const long long warps = static_cast<long long>(a.total_q) * a.H;
   const unsigned blocks = static_cast<unsigned>((warps + 7) / 8);
   if (blocks == 0 || a.splits <= 1) return cudaSuccess;
-  if (a.D == 64)
-    decode_combine_kernel<64><<<blocks, 256, 0, stream>>>(a);
-  else
-    decode_combine_kernel<128><<<blocks, 256, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(a.D == 64 ? decode_combine_kernel<64> : decode_combine_kernel<128>, blocks, 256, 0, stream,
+                       a.chained != 0, a);
 }
 
 }  // namespace fa

@@ -596,6 +596,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&bars.tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  // Everything above is local to the CTA; the work list, the inputs and the
+  // outputs are touched only after the work-list kernel has finished.
+  griddep_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -655,8 +658,7 @@ cudaError_t launch_one(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMa
   if (launch_regs != static_cast<int>(kRegsLaunch)) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
-  kern<<<a.grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
-  return cudaGetLastError();
+  return launch_kernel(kern, a.grid, kThreads, L::kAlloc, stream, a.chained != 0, tq, tk, tv, a);
 }
 
 template <int KL>

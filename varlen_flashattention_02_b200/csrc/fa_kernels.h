@@ -42,6 +42,7 @@ struct FwdArgs {
   int grid;          // persistent CTAs
   uint64_t wait_ns;  // time limit of every pipeline wait
   int withhold_v0;   // test hook: the first V tile load of work item 0 is never issued
+  int chained;       // launched as a programmatic dependent of the work-list kernel
 };
 // tm_q: 2-D map over [rows, H*D] bf16; tm_k / tm_v over [rows, Hk*D]; box
 // 128 rows x 64 columns, 128-byte swizzle.
@@ -75,6 +76,7 @@ struct DecodeArgs {
   float scale_log2;
   int grid;
   uint64_t wait_ns;  // time limit of every pipeline wait
+  int chained;       // decode chained to the work-list kernel, combine to decode
 };
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tm_q3, const CUtensorMap& tm_k,
                           const CUtensorMap& tm_v, cudaStream_t stream);
@@ -100,6 +102,7 @@ struct BwdArgs {
   float scale_log2;   // softmax_scale * log2(e)
   int grid;
   uint64_t wait_ns;   // time limit of every pipeline wait
+  int chained;        // each launch a programmatic dependent of the one before it
 };
 // Backward in three launches: preprocess (rowsum(dO*O) and zero the dQ
 // accumulator), main, dQ conversion. Tensor maps, all bf16 with 128-byte

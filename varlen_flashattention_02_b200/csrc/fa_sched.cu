@@ -82,6 +82,9 @@ __global__ void __launch_bounds__(kThreads) sched_prep_kernel(SchedArgs a) {
   auto* pairs = reinterpret_cast<int2*>(static_cast<char*>(a.workspace) + a.pairs_offset);
   const int tid = threadIdx.x;
   const bool causal = a.causal != 0;
+  // The attention kernel launched behind this one may take its SMs and run
+  // its prologue now; it waits for this grid before it reads the work list.
+  griddep_launch_dependents();
 
   const bool cache = a.keys.seqlens_k != nullptr;
   if (tid == 0) {

@@ -328,6 +328,16 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
+// Programmatic dependent launch. griddep_wait: the grids this one was
+// launched behind have completed and their memory operations are visible
+// (returns at once in a grid launched without the dependency attribute).
+// griddep_launch_dependents: grids launched behind this one may start as
+// soon as every CTA of this grid has executed it or exited.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Three-input maximum (sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
