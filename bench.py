@@ -432,7 +432,7 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and not args.no_aux:
         result["fwd_by_workload"] = fwd_only_workloads(dev, stream, flush, peak)
         result["bwd_by_workload"] = bwd_workloads(dev, stream, flush, peak)
-        result["decode_by_workload"] = decode_workloads(dev, stream, flush, float(peaks["hbm_gbs"]))
+        result["decode_by_workload"] = decode_workloads(dev, stream, float(peaks["hbm_gbs"]))
     return result, w
 
 
@@ -545,11 +545,15 @@ def bwd_workloads(dev, stream, flush, peak, iters=10):
     return res
 
 
-def decode_workloads(dev, stream, flush, hbm_peak_gbs, iters=10):
+def decode_workloads(dev, stream, hbm_peak_gbs, iters=20):
     """Split-KV decoding: one query token per sequence against a long key/value
     cache, 32 query heads over 8 key/value heads, d=128. The bound is HBM: the
     figure is the K/V bytes the call must read over its time, against the
-    measured copy bandwidth."""
+    measured copy bandwidth. The key/value cache is 4x to 17x the L2, so no
+    flush runs between calls (a write flush would leave L2 full of dirty lines
+    whose write-back this DRAM-bound call would then pay for); the calls are
+    queued back to back and timed together, so that host-side launch work
+    never leaves the device idle inside the timed region."""
     import torch
 
     from varlen_flashattention_02_b200 import fa_varlen
@@ -573,20 +577,21 @@ def decode_workloads(dev, stream, flush, hbm_peak_gbs, iters=10):
                                                        out=out, softmax_lse=lse, workspace=ws, stream=stream)
         for _ in range(3):
             call()
-        evs = []
-        for _ in range(iters):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            call()
-            b.record(stream)
-            evs.append((a, b))
         torch.cuda.synchronize(dev)
-        ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(iters):
+            call()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        if fa_varlen.device_status(ws) != 0:
+            raise RuntimeError("device status not OK after the decode calls")
+        ms = a.elapsed_time(b) / iters
         kv_bytes = 2 * batch * lk * Hk * D * 2
         gbs = kv_bytes / (ms * 1e-3) / 1e9
         res[f"decode {batch} seqs x {lk} keys, h32 kv8 d128, 1 query token, {splits} splits"] = {
-            "ms": ms, "kv_gbytes": kv_bytes / 1e9, "gbs": gbs, "pct_of_hbm_peak": 100 * gbs / hbm_peak_gbs}
+            "ms": ms, "kv_gbytes": kv_bytes / 1e9, "gbs": gbs, "pct_of_hbm_peak": 100 * gbs / hbm_peak_gbs,
+            "timing": f"{iters} calls back to back, no L2 flush (K/V {kv_bytes / 2**20:.0f} MiB > 126 MB L2)"}
         del q, k, v, out, lse, ws
     return res
 

@@ -447,10 +447,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 // warp per (query token, head) row. The splits are handled 32 at a time:
 // lane s loads split s's logsumexp, the maximum and the sum of the weights
 // are warp reductions, and the partial outputs (a 16-byte vector per lane at
-// d = 128) are loaded back to back, so that the latency of the partials is
-// paid about once instead of once per split. A split that saw no key
-// (logsumexp -inf) has weight 0 and its partial, which it did not write, is
-// not used.
+// d = 128) are loaded eight at a time before any of them is used, so that
+// the latency of the partials is paid once per eight splits instead of once
+// per split. A split that saw no key (logsumexp -inf, partial written as
+// zeros) has weight 0 and is skipped.
 template <int D>
 __global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeArgs a) {
   griddep_wait();  // the partials come from the decode kernel before this one
@@ -478,14 +478,21 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeArgs a)
       sum += f;
       const int n = a.splits - s0 < 32 ? a.splits - s0 : 32;
       const float* src = a.opart + ((static_cast<size_t>(s0) * stride + w) * D + lane * E);
-#pragma unroll 8
-      for (int i = 0; i < n; ++i) {
-        const float fi = __shfl_sync(0xffffffffu, f, i);
-        const Vec x = *reinterpret_cast<const Vec*>(src + static_cast<size_t>(i) * stride * D);
-        const float* xv = reinterpret_cast<const float*>(&x);
-        if (fi != 0.f) {
+      for (int i0 = 0; i0 < n; i0 += 8) {
+        // Eight partials in flight before any is used.
+        Vec x[8];
 #pragma unroll
-          for (int e = 0; e < E; ++e) acc[e] = fmaf(fi, xv[e], acc[e]);
+        for (int u = 0; u < 8; ++u)
+          if (i0 + u < n) x[u] = *reinterpret_cast<const Vec*>(src + static_cast<size_t>(i0 + u) * stride * D);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (i0 + u >= n) break;
+          const float fi = __shfl_sync(0xffffffffu, f, i0 + u);
+          const float* xv = reinterpret_cast<const float*>(&x[u]);
+          if (fi != 0.f) {
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc[e] = fmaf(fi, xv[e], acc[e]);
+          }
         }
       }
     }
