@@ -596,6 +596,48 @@ def decode_workloads(dev, stream, hbm_peak_gbs, iters=20):
     return res
 
 
+def decode_only(args):
+    """--decode BATCHxKEYS: the split-KV decode call of that shape alone, for
+    profiling captures (the same seeded inputs and split count as the decode
+    lines of the full run)."""
+    import torch
+
+    from varlen_flashattention_02_b200 import fa_varlen
+
+    batch, lk = (int(x) for x in args.decode.lower().split("x"))
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    w = synth.decode_workload(batch, lk)
+    H, Hk, D = w.heads, w.kv_heads, w.head_dim
+    t = w.tensors()
+    q, k, v = (torch.from_numpy(t[n].view(np.int16)).view(torch.bfloat16).to(dev) for n in ("q", "k", "v"))
+    cu_q = torch.from_numpy(w.cu_q).to(dev)
+    cu_k = torch.from_numpy(w.cu_k).to(dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    splits = fa_varlen.fa_varlen_splitkv_num_splits(batch, 1, H, Hk, lk, sms)
+    out = torch.empty_like(q)
+    lse = torch.empty((H, batch), dtype=torch.float32, device=dev)
+    ws = fa_varlen.new_workspace(int(fa_varlen.lib.fa_varlen_fwd_splitkv_workspace_size(batch, batch, H, Hk, D, splits)),
+                                 dev)
+    call = lambda: fa_varlen.fa_varlen_fwd_splitkv(q, k, v, cu_q, 1, lk, w.scale, True, splits, cu_seqlens_k=cu_k,
+                                                   out=out, softmax_lse=lse, workspace=ws, stream=stream)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        call()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    if fa_varlen.device_status(ws) != 0:
+        raise RuntimeError("device status not OK after the decode calls")
+    ms = a.elapsed_time(b) / args.steps
+    kv_bytes = 2 * batch * lk * Hk * D * 2
+    return {"mode": "decode", "workload": f"{batch} seqs x {lk} keys, h32 kv8 d128, 1 query token", "splits": splits,
+            "calls": args.steps, "ms_per_call": ms, "kv_gbs": kv_bytes / (ms * 1e-3) / 1e9}
+
+
 # ------------------------------------------------------------- oracle (CPU)
 def oracle_sample(w, budget_s: float, seed: int = 0):
     """Pick (sequence, head) units of ``w`` whose oracle fwd+bwd takes about
@@ -714,6 +756,9 @@ def main():
                          "heads = one workload, its heads split across the ranks (strong scaling)")
     ap.add_argument("--tokens", type=int, default=synth.TOTAL_TOKENS,
                     help="total tokens of the workload (default 16384; smaller only for profiling captures)")
+    ap.add_argument("--decode", metavar="BATCHxKEYS",
+                    help="profiling mode, one GPU: only the split-KV decode call of that shape (one query token, "
+                         "32 query heads over 8 key/value heads, d=128), --warmup untimed and --steps timed calls")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -728,6 +773,11 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
+        return
+    if args.decode:
+        if world != 1:
+            sys.exit("--decode runs on one GPU")
+        print(json.dumps(decode_only(args)), flush=True)
         return
 
     import torch
