@@ -272,7 +272,10 @@ fa_status_t fa_varlen_fwd_splitkv(const void* q, const void* k, const void* v, c
  * returns the smallest num_splits for which the units fill the SMs in
  * nearly whole waves (at least 95% of the CTA-unit slots busy, the units
  * being of equal size), keeping at least two 128-key tiles per range; if no
- * count reaches that, the one with the best fill. A query tile holds
+ * count reaches that, the one with the best fill. If that count leaves
+ * fewer than 8 key tiles per range, where a unit's fixed costs dominate, it
+ * returns instead the smallest count whose units occupy at least 85% of the
+ * SMs at once, when there is a smaller one. A query tile holds
  * tq = floor(128 / group) tokens of one sequence (group = num_heads /
  * num_heads_k), so the unit count per range is taken as
  * batch * num_heads_k * ceil(max_seqlen_q / tq).

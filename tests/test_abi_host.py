@@ -163,7 +163,9 @@ def test_splitkv_rejects(lib):
 def test_splitkv_num_splits(lib):
     """The advisory split count: smallest count whose equal-sized units keep
     at least 95% of the (SM x wave) slots busy, at least two 128-key tiles per
-    range, 1 for invalid arguments. Values worked by hand for 148 SMs."""
+    range; if that leaves fewer than 8 key tiles per range, the smallest
+    smaller count whose units occupy 85% of the SMs at once; 1 for invalid
+    arguments. Values worked by hand for 148 SMs."""
     f = lib.fa_varlen_splitkv_num_splits
     # 64 sequences x 8 kv heads = 512 units: 1 split fills 512/592 = 86%,
     # 2 splits fill 1024/1036 = 98.8%.
@@ -181,11 +183,19 @@ def test_splitkv_num_splits(lib):
     # per tile, so 128 tokens need 4 tiles (not ceil(3*128/128) = 3). With 2
     # sequences x 8 kv heads that is 64 units per split; 9 splits fill
     # 576/592 = 97.3% (3 tiles per sequence would have given 3 splits:
-    # 144/148). g = 6 packs 21 tokens: 64 tokens need 4 tiles, 3 sequences x
-    # 8 x 4 = 96 units, 3 splits fill 288/296 = 97.3%.
+    # 144/148); ceil(64/9) = 8 key tiles per range, not fewer than 8, so 9
+    # stays. g = 6 packs 21 tokens: 64 tokens need 4 tiles, 3
+    # sequences x 8 x 4 = 96 units, 3 splits fill 288/296 = 97.3%.
     assert f(2, 128, 24, 8, 8192, 148) == 9
     assert f(3, 64, 48, 8, 8192, 148) == 3
     assert f(74, 42, 24, 8, 8192, 148) == f(74, 1, 24, 8, 8192, 148)  # 42 tokens: still one tile
+    # Short ranges: 16 sequences x 8 kv heads = 128 units per split, 4096
+    # keys = 32 tiles. 8 splits fill 1024/1036 = 98.8% but leave 4 tiles per
+    # range; 1 split already occupies 128/148 = 86% of the SMs.
+    assert f(16, 1, 32, 8, 4096, 148) == 1
+    # 8 x 8 = 64 units, 16384 keys = 128 tiles: 9 splits give 15 tiles per
+    # range, long enough, so the fill rule's choice stays.
+    assert f(8, 1, 32, 8, 16384, 148) == 9
     # Invalid arguments.
     assert f(0, 1, 32, 8, 8192, 148) == 1
     assert f(4, 1, 32, 7, 8192, 148) == 1
@@ -207,5 +217,8 @@ def test_splitkv_num_splits(lib):
                             break
                         if fill > best[0]:
                             best = (fill, s)
-                    assert f(batch, 1, hk, hk, lk, sms) == (want if want is not None else best[1])
+                    got = want if want is not None else best[1]
+                    if -(-tiles // got) < 8:
+                        got = next((s for s in range(1, got) if per * s * 100 >= 85 * sms), got)
+                    assert f(batch, 1, hk, hk, lk, sms) == got
 
