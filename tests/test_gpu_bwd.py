@@ -17,6 +17,7 @@ SMALL = [
     ("empty-and-one", [0, 5, 1, 0, 130, 3], [3, 0, 1, 0, 257, 300], 2, 128),
     ("multi-tile-ragged", [513, 260, 384], [513, 260, 384], 2, 64),
     ("long-ragged", [1000, 45], [1000, 45], 1, 128),
+    ("long-d64", [2000, 130], [2000, 130], 2, 64),
 ]
 
 

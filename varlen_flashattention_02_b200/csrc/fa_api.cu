@@ -52,6 +52,21 @@ bool encode_map(CUtensorMap* map, const void* base, int rows, int cols, int box_
 // 3-D bf16 map over q viewed as [tokens, H, D]: box = 64 channels x g heads x
 // tq tokens, 128-byte swizzle; it lands the (token, head) rows of a group
 // as consecutive 128-byte rows.
+// fp32 2-D map [rows, cols] with boxes of 128 rows x 32 columns (128 bytes),
+// 128-byte swizzle: the backward's dQ accumulator at head_dim 64.
+bool encode_map_f32(CUtensorMap* map, const void* base, long long rows, int cols) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 4};
+  cuuint32_t box[2] = {32, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool encode_map_q3(CUtensorMap* map, const void* base, int tokens, int H, int D, int g, int tq) {
   auto fn = get_encode_fn();
   if (!fn) return false;
@@ -250,6 +265,11 @@ fa_status_t run_bwd(const void* dout, const void* q, const void* k, const void* 
              !encode_map(&maps.dv, dvp, krows, kcols, fa::kBwdBN)) {
     return FA_ERR_CUDA;
   }
+  std::memset(&maps.dqacc, 0, sizeof(maps.dqacc));
+  if (head_dim == 64 && total_q > 0 &&
+      !encode_map_f32(&maps.dqacc, static_cast<char*>(workspace) + L.dqacc,
+                      static_cast<long long>(num_heads) * L.tq_pad, head_dim))
+    return FA_ERR_CUDA;
 
   const int sms = sm_count();
   if (sms <= 0) return FA_ERR_CUDA;

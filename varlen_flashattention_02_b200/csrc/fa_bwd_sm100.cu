@@ -57,7 +57,23 @@ constexpr uint32_t kTmemCols = 512;
 // TMEM column map: dK, dV (D columns each), S^T (P^T at +0/+64, dS^T at
 // +32/+96 as bf16 pairs, one 64-query half per P/dS warpgroup), dP^T (then
 // dQ^T: D lanes x 128 query columns).
-constexpr int kColDK = 0, kColDV = 128, kColS = 256, kColDP = 384;
+constexpr int kColDP = 384;  // dP^T of the step, then its dQ^T
+// TMEM columns of the dK and dV accumulators and of the S^T buffer(s). At
+// head_dim 64 the accumulators take 64 columns each and a second S^T buffer
+// fits: step p uses buffer p & 1, and the next step's S^T is computed while
+// this step's dS^T is being formed, so the P/dS warps go from dS^T of one
+// step straight to P^T of the next.
+template <int D>
+struct TCols {
+  static constexpr bool kTwoS = D == 64;
+  static constexpr uint32_t dk = 0, dv = D == 64 ? 64 : 128;
+  static constexpr uint32_t s0 = D == 64 ? 128 : 256;
+  __device__ static constexpr uint32_t s(uint32_t p) { return kTwoS ? s0 + (p & 1u) * 128u : s0; }
+  // s_full barrier of step p and the parity of its wait.
+  __device__ static constexpr int sbar(uint32_t p) { return kTwoS ? static_cast<int>(p & 1u) : 0; }
+  __device__ static constexpr uint32_t spar(uint32_t p) { return kTwoS ? (p >> 1) & 1u : p & 1u; }
+};
+static_assert(TCols<64>::s0 + 256 <= kColDP && TCols<128>::s0 + 128 <= kColDP, "TMEM columns");
 constexpr int kPdsWarp0 = 4, kDrainWarp0 = 12;
 
 template <int D>
@@ -116,7 +132,7 @@ struct Bars {
   // drain hands the Q half back as soon as the first half of the step's dQ
   // reduction has read it, so the next Q load starts early.
   uint64_t q_full[3], q_empty[3], do_full[3], do_empty[3];
-  uint64_t s_full, dp_full;   // S^T, dP^T of the step in TMEM
+  uint64_t s_full[2], dp_full;  // S^T (per buffer), dP^T of the step in TMEM
   uint64_t p_full, ds_full;   // P^T (TMEM), dS^T (TMEM and shared) written
   uint64_t dq_full, dq_free;  // dQ^T in TMEM; read out by the drain group
   uint64_t dkv_full, dv_free, dk_free;
@@ -192,8 +208,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
-               const BwdArgs a) {
+               const __grid_constant__ CUtensorMap tm_dqacc, const BwdArgs a) {
   using L = BwdSmem<D>;
+  using TC = TCols<D>;
   constexpr int NQ = L::kQStages;
   extern __shared__ __align__(1024) uint8_t smem[];
   Bars& bars = *reinterpret_cast<Bars*>(smem + L::kBar);
@@ -225,7 +242,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.ld_full[i], 2);
       mbar_init(&bars.ld_empty[i], 8);
     }
-    mbar_init(&bars.s_full, 1);
+    mbar_init(&bars.s_full[0], 1);
+    mbar_init(&bars.s_full[1], 1);
     mbar_init(&bars.dp_full, 1);
     mbar_init(&bars.p_full, 8);
     mbar_init(&bars.ds_full, 8);
@@ -342,6 +360,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t kIdS = idesc_bf16_f32(BN, BM, false, false);  // S^T, dP^T: 128 x 128, K = D
     constexpr uint32_t kIdKV = idesc_bf16_f32(BN, D, false, true);   // dV, dK: 128 x D, K = 128 queries
     constexpr uint32_t kIdQ = idesc_bf16_f32(128, BM, true, true);   // dQ^T: 128 (>= D) x 128, K = 128 keys
+    // At head_dim 64, dQ itself: 128 queries x 64, K = 128 keys, A = dS from
+    // the dS^T buffer read M-major, B = K read N-major.
+    constexpr uint32_t kIdQ64 = idesc_bf16_f32(BM, 64, true, true);
     const uint64_t k_kmaj = smem_desc_sw128(smem_u32(smem + L::kK), 16, 1024);
     const uint64_t v_kmaj = smem_desc_sw128(smem_u32(smem + L::kV), 16, 1024);
     // At head_dim 64 the second 64-row half of M reads the first again
@@ -363,23 +384,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (it.n == 0) continue;
       if (!wait_bar_warp(&bars.kv_full, m & 1, ab)) goto mma_done;
       tc_fence_after();
+      // S^T of step pp into its buffer (waits for pp's Q tile).
+      auto issue_s = [&](uint32_t pp) -> bool {
+        const int qq = static_cast<int>(pp % NQ);
+        if (!wait_bar_warp(&bars.q_full[qq], (pp / NQ) & 1, ab)) return false;
+        tc_fence_after();
+        if (elect_one()) {
+          const uint64_t qk = opaque_u64(qdo_kmaj0) + static_cast<uint64_t>((2 * qq * L::kQTile) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t o = ((kk >> 2) * L::kKChunk + (kk & 3) * 32) >> 4;
+            mma_ss(tmem + TC::s(pp), opaque_u64(k_kmaj) + o, qk + o, kIdS, kk > 0);
+          }
+          mma_commit(&bars.s_full[TC::sbar(pp)]);
+        }
+        __syncwarp();
+        return true;
+      };
       for (int s = 0; s < it.n; ++s, ++p) {
         const int qs = p % NQ;
         // Descriptors are rebuilt from opaque copies where they are used, so
         // that the compiler does not keep every offset form in registers.
         const uint64_t q_kmaj = opaque_u64(qdo_kmaj0) + static_cast<uint64_t>((2 * qs * L::kQTile) >> 4);
         const uint64_t q_mn = opaque_u64(qdo_mn0) + static_cast<uint64_t>((2 * qs * L::kQTile) >> 4);
-        if (!wait_bar_warp(&bars.q_full[qs], (p / NQ) & 1, ab)) goto mma_done;
-        tc_fence_after();
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t o = ((kk >> 2) * L::kKChunk + (kk & 3) * 32) >> 4;
-            mma_ss(tmem + kColS, opaque_u64(k_kmaj) + o, q_kmaj + o, kIdS, kk > 0);
-          }
-          mma_commit(&bars.s_full);
-        }
-        __syncwarp();
+        // With two S^T buffers an item's later steps had their S^T issued
+        // during the step before.
+        if ((!TC::kTwoS || s == 0) && !issue_s(p)) goto mma_done;
         // dP^T goes where the previous step's dQ^T is until the drain group
         // has read it out.
         if (p > 0 && !wait_bar_warp(&bars.dq_free, (p - 1) & 1, ab)) goto mma_done;
@@ -405,10 +435,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           // queries 64-127 start 64 columns further), dO MN-major.
 #pragma unroll
           for (int kk = 0; kk < BM / 16; ++kk)
-            mma_ts(tmem + kColDV, tmem + kColS + (kk >> 2) * 64 + (kk & 3) * 8,
+            mma_ts(tmem + TC::dv, tmem + TC::s(p) + (kk >> 2) * 64 + (kk & 3) * 8,
                    q_mn + kQTileD + ((kk * 2048) >> 4), kIdKV, (acc | kk) ? 1u : 0u);
         }
         __syncwarp();
+        // The next step's S^T into the other buffer, while the P/dS warps
+        // form this step's dS^T (dK below reads this step's buffer).
+        if (TC::kTwoS && s + 1 < it.n && !issue_s(p + 1)) goto mma_done;
         if (!wait_bar_warp(&bars.ds_full, p & 1, ab)) goto mma_done;
         if (s == 0 && m > 0 && !wait_bar_warp(&bars.dk_free, (m - 1) & 1, ab)) goto mma_done;
         tc_fence_after();
@@ -416,13 +449,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           // dK += dS^T Q (dS^T bf16 in TMEM, 32 columns after its P^T).
 #pragma unroll
           for (int kk = 0; kk < BM / 16; ++kk)
-            mma_ts(tmem + kColDK, tmem + kColS + (kk >> 2) * 64 + 32 + (kk & 3) * 8, q_mn + ((kk * 2048) >> 4),
+            mma_ts(tmem + TC::dk, tmem + TC::s(p) + (kk >> 2) * 64 + 32 + (kk & 3) * 8, q_mn + ((kk * 2048) >> 4),
                    kIdKV, (acc | kk) ? 1u : 0u);
-          // dQ^T = K^T dS^T (dS^T from shared memory) into the dP^T columns.
+          // dQ^T = K^T dS^T (dS^T from shared memory) into the dP^T columns;
+          // at head_dim 64 dQ = dS K instead (one query row per TMEM lane, so
+          // all four drain warps read it, and N = 64 with no padded half).
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            mma_ss(tmem + kColDP, opaque_u64(k_mn) + ((kk * 2048) >> 4), opaque_u64(ds_mn) + ((kk * 2048) >> 4), kIdQ,
-                   kk > 0);
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            if constexpr (D == 64)
+              mma_ss(tmem + kColDP, opaque_u64(ds_mn) + ((kk * 2048) >> 4), opaque_u64(k_mn) + ((kk * 2048) >> 4),
+                     kIdQ64, kk > 0);
+            else
+              mma_ss(tmem + kColDP, opaque_u64(k_mn) + ((kk * 2048) >> 4), opaque_u64(ds_mn) + ((kk * 2048) >> 4),
+                     kIdQ, kk > 0);
+          }
           mma_commit(&bars.dq_full);
         }
         __syncwarp();
@@ -486,7 +526,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qh = (warp - kPdsWarp0) >> 2;
     const int kr = (threadIdx.x - kPdsWarp0 * 32) & 127;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t t_s = tmem + lane_base + kColS + qh * 64;    // S^T of my queries; P^T, dS^T after it
     const uint32_t t_dp = tmem + lane_base + kColDP + qh * 64;  // dP^T of my queries
     uint8_t* ds_row = smem + L::kDs + qh * L::kDsHalf + kr * 128;
     uint32_t p = 0, ni = 0;
@@ -502,7 +541,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int diag = it.s.lk - it.s.lq;
       for (int s = 0; s < it.n; ++s, ++p) {
         const int slot = p % NQ;
-        if (!wait_bar_warp(&bars.s_full, p & 1, ab)) goto compute_done;
+        if (!wait_bar_warp(&bars.s_full[TC::sbar(p)], TC::spar(p), ab)) goto compute_done;
+        const uint32_t t_s = tmem + lane_base + TC::s(p) + qh * 64;  // S^T of my queries; P^T, dS^T after it
         if (!wait_bar_warp(&bars.ld_full[slot], (p / NQ) & 1, ab)) goto compute_done;
         tc_fence_after();
         const float* ld = reinterpret_cast<const float*>(smem + L::kLd) + slot * 2 * BM + qh * 64;
@@ -541,8 +581,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.p_full);
-        // dS^T of the previous step has been read by its dQ^T MMAs: S^T of
-        // this step was issued after them and has completed.
+        // dS^T of the previous step has been read by its dQ^T MMAs: dP^T of
+        // this step goes where that dQ^T was and is issued only after the
+        // drain group has read it out.
         if (!wait_bar_warp(&bars.dp_full, p & 1, ab)) goto compute_done;
         tc_fence_after();
         const uint64_t* dv2p = reinterpret_cast<const uint64_t*>(ld + BM);
@@ -632,53 +673,97 @@ __global__ void __launch_bounds__(kThreads, 1)
         const size_t q0 = static_cast<size_t>(it.s.q0) + static_cast<size_t>(sp.t) * BM;
         uint32_t* cnt = qcount + static_cast<size_t>(sp.h) * a.tq_pad + q0;
         float* gdq = dqacc + (static_cast<size_t>(sp.h) * a.tq_pad + q0) * D;
-#pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
-          uint32_t v0[32], v1[32];
-          tmem_ld32(tmem + lane_base + kColDP + h * 64, v0);
-          tmem_ld32(tmem + lane_base + kColDP + h * 64 + 32, v1);
+        if constexpr (D == 64) {
+          // Thread t holds query row t of dQ (64 channels): one read frees
+          // the columns at once. The row is staged as two 128-byte-swizzled
+          // boxes of [128 rows x 32 channels] (channels 0-31 over the Q half
+          // of the stage, 32-63 over the dO half; the swizzle spreads a
+          // warp's stores over all banks) and leaves with two tensor
+          // reductions into the accumulator viewed as [H * tq_pad, 64].
+          uint32_t v[64];
+          tmem_ld32(tmem + lane_base + kColDP, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+          tmem_ld32(tmem + lane_base + kColDP + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
           tmem_wait_ld();
-          if (h == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars.dq_free);
-          }
-          float* st = stage + h * 64 * D;
-          if (t < D) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars.dq_free);
+          uint8_t* st8 = reinterpret_cast<uint8_t*>(stage) + t * 128;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) st[e * D + t] = __uint_as_float(v0[e]);
+          for (int b = 0; b < 2; ++b)
 #pragma unroll
-            for (int e = 0; e < 32; ++e) st[(32 + e) * D + t] = __uint_as_float(v1[e]);
-          }
-          if (!DET) {
-            fence_proxy_async_smem();
-            named_bar_sync(1, 128);
-            if (t == 0 && !*ab.flag) {
-              bulk_reduce_add_f32(gdq + h * 64 * D, st, 64 * D * 4);
-              bulk_commit_group();
-            }
-          }
-        }
-        if (DET) {
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(st8 + b * L::kQTile + ((c ^ (t & 7)) << 4)) =
+                  make_uint4(v[32 * b + 4 * c], v[32 * b + 4 * c + 1], v[32 * b + 4 * c + 2], v[32 * b + 4 * c + 3]);
           fence_proxy_async_smem();
           named_bar_sync(1, 128);
           if (t == 0) {
-            // This query tile's turn first (a wait that runs out raises the
-            // abort flag, and nothing more is added).
-            wait_dq_turn(cnt, static_cast<uint32_t>(it.j), ab);
+            const int y = sp.h * a.tq_pad + static_cast<int>(q0);
+            if (DET) wait_dq_turn(cnt, static_cast<uint32_t>(it.j), ab);
             if (!*ab.flag) {
-              fence_proxy_async_global();
-              bulk_reduce_add_f32(gdq, stage, BM * D * 4);
+              if (DET) fence_proxy_async_global();
+              tma_reduce_add_2d(&tm_dqacc, stage, 0, y);
+              if (!DET) bulk_commit_group();
+              tma_reduce_add_2d(&tm_dqacc, reinterpret_cast<uint8_t*>(stage) + L::kQTile, 32, y);
               bulk_commit_group();
-              // Pass the previous step's turn on once its addition has been
-              // performed (it was issued a step ago, so this rarely waits);
-              // this step's turn passes on at the next step or item end.
-              if (det_prev) {
-                bulk_wait_group1();
-                fence_proxy_async_global();
-                st_release_gpu(det_prev, static_cast<uint32_t>(it.j) + 1u);
+              if (DET) {
+                if (det_prev) {
+                  bulk_wait_group1();
+                  fence_proxy_async_global();
+                  st_release_gpu(det_prev, static_cast<uint32_t>(it.j) + 1u);
+                }
+                det_prev = cnt;
               }
-              det_prev = cnt;
+            }
+          }
+        } else {
+  #pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            uint32_t v0[32], v1[32];
+            tmem_ld32(tmem + lane_base + kColDP + h * 64, v0);
+            tmem_ld32(tmem + lane_base + kColDP + h * 64 + 32, v1);
+            tmem_wait_ld();
+            if (h == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bars.dq_free);
+            }
+            float* st = stage + h * 64 * D;
+            if (t < D) {
+  #pragma unroll
+              for (int e = 0; e < 32; ++e) st[e * D + t] = __uint_as_float(v0[e]);
+  #pragma unroll
+              for (int e = 0; e < 32; ++e) st[(32 + e) * D + t] = __uint_as_float(v1[e]);
+            }
+            if (!DET) {
+              fence_proxy_async_smem();
+              named_bar_sync(1, 128);
+              if (t == 0 && !*ab.flag) {
+                bulk_reduce_add_f32(gdq + h * 64 * D, st, 64 * D * 4);
+                bulk_commit_group();
+              }
+            }
+          }
+          if (DET) {
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            if (t == 0) {
+              // This query tile's turn first (a wait that runs out raises the
+              // abort flag, and nothing more is added).
+              wait_dq_turn(cnt, static_cast<uint32_t>(it.j), ab);
+              if (!*ab.flag) {
+                fence_proxy_async_global();
+                bulk_reduce_add_f32(gdq, stage, BM * D * 4);
+                bulk_commit_group();
+                // Pass the previous step's turn on once its addition has been
+                // performed (it was issued a step ago, so this rarely waits);
+                // this step's turn passes on at the next step or item end.
+                if (det_prev) {
+                  bulk_wait_group1();
+                  fence_proxy_async_global();
+                  st_release_gpu(det_prev, static_cast<uint32_t>(it.j) + 1u);
+                }
+                det_prev = cnt;
+              }
             }
           }
         }
@@ -720,7 +805,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll 1
         for (int g = 0; g < 2; ++g) {  // g = 0: dV, g = 1: dK (times scale)
-          const int col = g == 0 ? kColDV : kColDK;
+          const int col = g == 0 ? TC::dv : TC::dk;
           const float sc = g == 0 ? 1.f : a.scale;
           __nv_bfloat16* gdst = static_cast<__nv_bfloat16*>(g == 0 ? a.dv : a.dk) + krow * D;
           uint8_t* box = stage + g * L::kQTile;  // bf16 boxes of [128 rows x 64 columns], 16 KB apart
@@ -902,11 +987,12 @@ __global__ void __launch_bounds__(256) bwd_convert_kernel(const BwdArgs a) {
 template <int D, bool CAUSAL, bool DET>
 cudaError_t launch_main(const BwdArgs& a, const BwdMaps& m, cudaStream_t stream) {
   using L = BwdSmem<D>;
+  using TC = TCols<D>;
   auto kern = bwd_kernel<D, CAUSAL, DET>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
   if (e != cudaSuccess) return e;
   return launch_kernel(kern, a.grid, kThreads, L::kBytes, stream, a.chained != 0, m.q, m.k, m.v, m.dout, m.dk, m.dv,
-                       a);
+                       m.dqacc, a);
 }
 
 }  // namespace

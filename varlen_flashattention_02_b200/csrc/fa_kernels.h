@@ -109,8 +109,11 @@ struct BwdArgs {
 // swizzle and 64-column boxes: q / dout over [rows, H*D] with 128-row boxes
 // (loads); k / v over [rows, Hk*D] with 128-row boxes (loads); dk / dv over
 // [rows, Hk*D] with 128-row boxes (stores of whole key tiles).
+// At head_dim 64 dQ leaves through tensor reductions: dqacc is an fp32 map
+// over the accumulator viewed as [H * tq_pad rows, 64], boxes of 128 rows x
+// 32 columns (128 bytes) with 128-byte swizzle (unused at head_dim 128).
 struct BwdMaps {
-  CUtensorMap q, k, v, dout, dk, dv;
+  CUtensorMap q, k, v, dout, dk, dv, dqacc;
 };
 // head_dim 256: a dV pass (q / dout maps with 128-row boxes) and a dK/dQ
 // pass (q / dout maps with 64-row boxes); k, v with 128-row boxes. Both take
