@@ -257,7 +257,13 @@ typedef struct {
  *    (num_splits = 1 writes out directly).
  * head_dim 64 or 128 (FA_ERR_UNSUPPORTED otherwise). The workspace must
  * hold fa_varlen_fwd_splitkv_workspace_size(...) bytes (0 = invalid sizes).
- * Layout-specific checks are those of the matching entry point. */
+ * Layout-specific checks are those of the matching entry point. When
+ * max_seqlen_q <= floor(128 / g) (every sequence fits one tile: decoding)
+ * the call builds no work list: it resets the workspace's status word and
+ * work counters with one cudaMemsetAsync and the decode kernel checks each
+ * sequence as it takes its work; a sequence that fails a check is skipped
+ * and FA_ERR_BAD_SEQLENS is recorded (the outputs are then undefined, as
+ * for every device-side error). */
 size_t fa_varlen_fwd_splitkv_workspace_size(int batch, int total_q, int num_heads, int num_heads_k, int head_dim,
                                             int num_splits);
 fa_status_t fa_varlen_fwd_splitkv(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,

@@ -155,3 +155,79 @@ def test_splitkv_workspace_reused():
         torch.cuda.synchronize()
         ref_out, ref_lse = oracle.fwd(t["q"], t["k"], t["v"], w.cu_q, w.cu_k, w.scale, True)
         _check(t["q"], w.cu_q, out, lse, ref_out, ref_lse, H, D, True)
+
+
+# Decode calls (at most one query tile per sequence) run without a work list:
+# the decode kernel checks every sequence itself. Each case breaks one check.
+# (name, layout, cu_q, max_seqlen_q, key description)
+BAD = [
+    ("cu_q-decreasing", "packed", [0, 2, 1, 3], 4, None),
+    ("cu_q-end", "packed", [0, 1, 2, 2], 4, None),
+    ("lq-over-max", "packed", [0, 3, 4, 5], 2, None),
+    ("cu_k-end", "packed", [0, 1, 2, 3], 4, "cu_k_end"),
+    ("slots-leftpad", "slots", [0, 1, 2, 3], 4, "leftpad"),
+    ("slots-rows", "slots", [0, 1, 2, 3], 4, "rows"),
+    ("paged-page", "paged", [0, 1, 2, 3], 4, "page"),
+    ("paged-len", "paged", [0, 1, 2, 3], 4, "len"),
+]
+
+
+@pytest.mark.parametrize("case", BAD, ids=[c[0] for c in BAD])
+def test_splitkv_bad_sequences_reported(case):
+    """A malformed sequence is reported as FA_ERR_BAD_SEQLENS; the same
+    workspace then serves a well-formed call, which matches the oracle."""
+    import torch
+
+    from varlen_flashattention_02_b200 import fa_varlen
+
+    name, layout, cu_q, max_q, kind = case
+    rng = np.random.default_rng(861)
+    H, Hk, D, batch, Tq = 8, 2, 128, 3, cu_q[-1] if name != "cu_q-end" else 3
+    q = pu.to_dev(synth.bf16_normal(rng, (Tq, H, D)))
+    cq = _dev(np.array(cu_q, dtype=np.int32))
+    scale = 1.0 / np.sqrt(D)
+    ws = fa_varlen.new_workspace(int(fa_varlen.lib.fa_varlen_fwd_splitkv_workspace_size(batch, Tq, H, Hk, D, 4)), "cuda")
+    if layout == "packed":
+        ck_np = np.array([0, 300, 500, 900], dtype=np.int32)
+        if kind == "cu_k_end":
+            ck_np[-1] = 800  # the keys' offsets end short of total_k (900 rows)
+        k = pu.to_dev(synth.bf16_normal(rng, (900, Hk, D)))
+        v = pu.to_dev(synth.bf16_normal(rng, (900, Hk, D)))
+        kw = dict(cu_seqlens_k=_dev(ck_np))
+        max_k = 400
+    elif layout == "slots":
+        rows = 512
+        k = pu.to_dev(synth.bf16_normal(rng, (batch, rows, Hk, D)))
+        v = pu.to_dev(synth.bf16_normal(rng, (batch, rows, Hk, D)))
+        sl = np.array([300, 200, 512], dtype=np.int32)
+        lp = np.array([0, 10, 5], dtype=np.int32)
+        if kind == "leftpad":
+            lp[1] = 250  # left padding past the sequence end
+        else:
+            sl[2] = 600  # more rows than the cache slot has
+        kw = dict(seqlens_k=_dev(sl), leftpad_k=_dev(lp))
+        max_k = 1024
+    else:
+        ps, n_pages = 256, 6
+        k = pu.to_dev(synth.bf16_normal(rng, (n_pages, ps, Hk, D)))
+        v = pu.to_dev(synth.bf16_normal(rng, (n_pages, ps, Hk, D)))
+        bt = np.array([[0, 1], [2, 3], [4, 5]], dtype=np.int32)
+        sl = np.array([300, 256, 400], dtype=np.int32)
+        if kind == "page":
+            bt[2, 1] = 7  # a page outside the 6-page pool
+        else:
+            sl[1] = 600  # more keys than two pages hold
+        kw = dict(seqlens_k=_dev(sl), block_table=_dev(bt))
+        max_k = 1024
+    fa_varlen.fa_varlen_fwd_splitkv(q, k, v, cq, max_q, max_k, scale, True, 4, workspace=ws, **kw)
+    assert fa_varlen.device_status(ws) == 5  # FA_ERR_BAD_SEQLENS
+    # A well-formed call on the same workspace.
+    good = synth.make_workload("bad-then-good", [1, 1, 1], [300, 200, 400], heads=H, head_dim=D, causal=True,
+                               seed=862, heads_k=Hk)
+    t = good.tensors()
+    out, lse = fa_varlen.fa_varlen_fwd_splitkv(pu.to_dev(t["q"]), pu.to_dev(t["k"]), pu.to_dev(t["v"]),
+                                               pu.cu_dev(good.cu_q), 1, 400, good.scale, True, 4,
+                                               cu_seqlens_k=pu.cu_dev(good.cu_k), workspace=ws)
+    assert fa_varlen.device_status(ws) == 0
+    ref_out, ref_lse = oracle.fwd(t["q"], t["k"], t["v"], good.cu_q, good.cu_k, good.scale, True)
+    _check(t["q"], good.cu_q, out, lse, ref_out, ref_lse, H, D, True)

@@ -421,9 +421,18 @@ fa_status_t fa_varlen_fwd_splitkv(const void* q, const void* k, const void* v, c
                          kv->cache_rows, kv->block_table, kv->max_pages_per_seq, kv->page_size};
 
   t_events.next = 0;
-  fa::SchedArgs sa{cu_seqlens_q, keys, batch, total_q, total_k, max_seqlen_q, max_seqlen_k,
-                   causal ? 1 : 0, 0, L.tq, 0, workspace, L.seq_off, L.pairs, L.max_pairs};
-  if (timed_launch(stream, [&] { return fa::launch_sched_prep(sa, stream); }) != cudaSuccess) return FA_ERR_CUDA;
+  // Decoding and other calls whose sequences have at most one query tile need
+  // no work list: the decode kernel takes item idx as (sequence idx / (Hk *
+  // splits), its only tile) and checks each sequence itself, and the call
+  // only resets the header's status word and work counters.
+  const bool inline_list = max_seqlen_q <= L.tq;
+  if (inline_list) {
+    if (cudaMemsetAsync(workspace, 0, 4 * sizeof(uint32_t), stream) != cudaSuccess) return FA_ERR_CUDA;
+  } else {
+    fa::SchedArgs sa{cu_seqlens_q, keys, batch, total_q, total_k, max_seqlen_q, max_seqlen_k,
+                     causal ? 1 : 0, 0, L.tq, 0, workspace, L.seq_off, L.pairs, L.max_pairs};
+    if (timed_launch(stream, [&] { return fa::launch_sched_prep(sa, stream); }) != cudaSuccess) return FA_ERR_CUDA;
+  }
   if (total_q == 0) return FA_OK;
 
   const int g = num_heads / num_heads_k;
@@ -439,7 +448,7 @@ fa_status_t fa_varlen_fwd_splitkv(const void* q, const void* k, const void* v, c
 
   const int sms = sm_count();
   if (sms <= 0) return FA_ERR_CUDA;
-  const long long items = static_cast<long long>(L.max_pairs) * num_heads_k * num_splits;
+  const long long items = static_cast<long long>(inline_list ? batch : L.max_pairs) * num_heads_k * num_splits;
   fa::DecodeArgs d{};
   d.cu_q = cu_seqlens_q;
   d.keys = keys;
@@ -461,9 +470,18 @@ fa_status_t fa_varlen_fwd_splitkv(const void* q, const void* k, const void* v, c
   d.scale_log2 = softmax_scale * 1.4426950408889634f;
   d.grid = static_cast<int>(items < sms ? items : sms);
   d.wait_ns = t_hooks.wait_ns;
-  d.chained = chained() ? 1 : 0;
+  d.inline_list = inline_list ? 1 : 0;
+  d.batch = batch;
+  d.total_k = total_k;
+  d.max_seqlen_q = max_seqlen_q;
+  d.max_seqlen_k = max_seqlen_k;
+  // After the header reset the decode kernel is the call's first kernel: a
+  // plain launch. The combine is chained to it.
+  fa::DecodeArgs dc = d;
+  d.chained = chained() && !inline_list ? 1 : 0;
+  dc.chained = chained() ? 1 : 0;
   if (timed_launch(stream, [&] { return fa::launch_decode(d, tq3, tk, tv, stream); }) != cudaSuccess ||
-      timed_launch(stream, [&] { return fa::launch_decode_combine(d, stream); }) != cudaSuccess)
+      timed_launch(stream, [&] { return fa::launch_decode_combine(dc, stream); }) != cudaSuccess)
     return FA_ERR_CUDA;
   return FA_OK;
 }

@@ -68,7 +68,25 @@ struct Item {
   int b, hk, t, split;  // t: tile of tq query tokens
   SeqInfo s;
   int j0, j1;           // key tiles [j0, j1) of this split
+  bool bad;             // inline list: the sequence failed its checks (the item does nothing)
 };
+
+// Without a work list, the checks the work-list kernel makes on sequence b:
+// its query rows lie inside [0, total_q) and number at most max_seqlen_q,
+// and its keys lie inside their layout's bounds (packed: inside [0,
+// total_k); cache slots: 0 <= leftpad <= seqlens <= cache_rows; pages: at
+// most max_pages * page_size keys) and number at most max_seqlen_k.
+template <int KL>
+__device__ __forceinline__ bool seq_ok(const DecodeArgs& a, int b, const SeqInfo& s) {
+  if (s.q0 < 0 || s.lq < 0 || s.lq > a.max_seqlen_q || s.q0 + s.lq > a.total_q) return false;
+  if (s.lk < 0 || s.lk > a.max_seqlen_k) return false;
+  if (KL == kKeysPaged) return s.lk <= a.keys.max_pages * a.keys.page_size;
+  if (KL == kKeysSlots) {
+    const int lp = a.keys.leftpad_k ? __ldg(a.keys.leftpad_k + b) : 0;
+    return lp >= 0 && lp + s.lk <= a.keys.cache_rows;
+  }
+  return s.k0 >= 0 && s.k0 + s.lk <= a.total_k;
+}
 
 template <int KL>
 __device__ __forceinline__ Item get_item(const DecodeArgs& a, const int2* pairs, int idx) {
@@ -76,15 +94,42 @@ __device__ __forceinline__ Item get_item(const DecodeArgs& a, const int2* pairs,
   it.split = idx % a.splits;
   const int rest = idx / a.splits;
   it.hk = rest % a.Hk;
-  const int2 pr = pairs[rest / a.Hk];
-  it.b = pr.x;
-  it.t = pr.y;
+  if (a.inline_list) {
+    it.b = rest / a.Hk;
+    it.t = 0;
+  } else {
+    const int2 pr = pairs[rest / a.Hk];
+    it.b = pr.x;
+    it.t = pr.y;
+  }
   it.s = seq_info_l<KL>(a.cu_q, a.keys, it.b);
+  it.bad = a.inline_list && !seq_ok<KL>(a, it.b, it.s);
+  if (a.inline_list && (it.bad || it.s.lq == 0)) {  // no rows: nothing to load, nothing to write
+    it.s.lq = 0;
+    it.j0 = it.j1 = 0;
+    return it;
+  }
   const int nk = fwd_k_tiles((it.t + 1) * a.tq, it.s.lq, it.s.lk, a.causal != 0);
   const int per = (nk + a.splits - 1) / a.splits;
   it.j0 = min(nk, it.split * per);
   it.j1 = min(nk, it.j0 + per);
   return it;
+}
+
+// Row of key tile j of the item in the key/value tensor. With an inline list
+// the block-table entries have not been checked: a page outside the pool
+// gives row 0 and clears `ok`.
+template <int KL>
+__device__ __forceinline__ int tile_row(const DecodeArgs& a, const Item& it, int j, bool& ok) {
+  if (KL != kKeysPaged) return it.s.k0 + j * BN;
+  if (!a.inline_list) return key_tile_row(a.keys, it.b, it.s, j);
+  const int pos = j * BN;
+  const int page = __ldg(a.keys.block_table + static_cast<size_t>(it.b) * a.keys.max_pages + pos / a.keys.page_size);
+  if (page < 0 || page >= a.total_k / a.keys.page_size) {
+    ok = false;
+    return 0;
+  }
+  return page * a.keys.page_size + pos % a.keys.page_size;
 }
 
 template <int D, bool CAUSAL, int KL>
@@ -143,16 +188,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
   const Abort ab{&bars.abort_flag, &hdr->status, a.wait_ns};
-  const int n_items = (hdr->status == FA_OK) ? static_cast<int>(hdr->n_pairs) * a.Hk * a.splits : 0;
+  const int n_pairs = a.inline_list ? a.batch : static_cast<int>(hdr->n_pairs);
+  const int n_items = (hdr->status == FA_OK) ? n_pairs * a.Hk * a.splits : 0;
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ Q and K producer
+    if (a.inline_list && blockIdx.x == 0) {
+      // The whole-batch checks of the work-list kernel: the offsets start at
+      // 0 and end at the totals.
+      bool ok = __ldg(a.cu_q) == 0 && __ldg(a.cu_q + a.batch) == a.total_q;
+      if (KL == kKeysPacked) ok = ok && __ldg(a.keys.cu_k) == 0 && __ldg(a.keys.cu_k + a.batch) == a.total_k;
+      if (!ok) atomicCAS(&hdr->status, static_cast<uint32_t>(FA_OK), static_cast<uint32_t>(FA_ERR_BAD_SEQLENS));
+    }
     uint32_t kc = 0, nq = 0, ni = 0;
     for (;;) {
       int idx;
       if (!publish_item(bars.items, ni, &hdr->work_counter, n_items, idx, ab)) goto kproducer_done;
       if (idx < 0) break;
       const Item it = get_item<KL>(a, pairs, idx);
+      if (it.bad) atomicCAS(&hdr->status, static_cast<uint32_t>(FA_OK), static_cast<uint32_t>(FA_ERR_BAD_SEQLENS));
       if (it.j0 >= it.j1) continue;
       if (nq > 0 && !wait_bar(&bars.q_empty, (nq - 1) & 1, ab)) goto kproducer_done;
       // Rows (token, head): tq tokens from the tile's first, the group's g
@@ -167,7 +221,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = it.j0; j < it.j1; ++j, ++kc) {
         const int st = kc % NK;
         const uint32_t use = kc / NK;
-        const int krow = KL == kKeysPaged ? key_tile_row(a.keys, it.b, it.s, j) : it.s.k0 + j * BN;
+        bool page_ok = true;
+        const int krow = tile_row<KL>(a, it, j, page_ok);
+        if (!page_ok)
+          atomicCAS(&hdr->status, static_cast<uint32_t>(FA_OK), static_cast<uint32_t>(FA_ERR_BAD_SEQLENS));
         if (use > 0 && !wait_bar(&bars.k_empty[st], (use - 1) & 1, ab)) goto kproducer_done;
         mbar_arrive_expect_tx(&bars.k_full[st], L::kTileBytes);
         for (int c = 0; c < L::kChunks; ++c)
@@ -190,7 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = it.j0; j < it.j1; ++j, ++vc) {
         const int st = vc % NV;
         const uint32_t use = vc / NV;
-        const int vrow = KL == kKeysPaged ? key_tile_row(a.keys, it.b, it.s, j) : it.s.k0 + j * BN;
+        bool page_ok = true;  // reported by the K producer
+        const int vrow = tile_row<KL>(a, it, j, page_ok);
         if (use > 0 && !wait_bar(&bars.v_empty[st], (use - 1) & 1, ab)) goto vproducer_done;
         mbar_arrive_expect_tx(&bars.v_full[st], L::kTileBytes);
         for (int c = 0; c < L::kChunks; ++c)

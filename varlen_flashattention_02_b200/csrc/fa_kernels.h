@@ -77,6 +77,12 @@ struct DecodeArgs {
   int grid;
   uint64_t wait_ns;  // time limit of every pipeline wait
   int chained;       // decode chained to the work-list kernel, combine to decode
+  // 1: no work list. Every sequence has at most one query tile, so item idx
+  // is (sequence idx / (Hk * splits), its only tile); the kernel checks each
+  // item's sequence itself (the checks of the work-list kernel) and the
+  // call resets the header instead of running that kernel.
+  int inline_list;
+  int batch, total_k, max_seqlen_q, max_seqlen_k;
 };
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tm_q3, const CUtensorMap& tm_k,
                           const CUtensorMap& tm_v, cudaStream_t stream);
