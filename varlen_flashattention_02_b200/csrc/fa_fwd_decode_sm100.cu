@@ -19,9 +19,12 @@
 //    different CTAs; each writes its normalised partial output and its
 //    logsumexp, and the combine kernel merges them:
 //      lse = log sum_s exp(lse_s),  out = sum_s exp(lse_s - lse) * out_s.
-// Roles: one warp loads Q and K (and hands out items), one loads V, one
-// issues the MMAs, four (one thread per tile row) run the softmax and the
-// epilogue; S is double-buffered in TMEM, O accumulates in TMEM.
+// Items come from the work list, or, when every sequence fits one query tile
+// (decoding), straight from their index, each sequence then checked by the
+// kernel itself. Roles: one warp loads Q and K (and hands out items), one
+// loads V, one issues the MMAs, four (one thread per tile row) run the
+// softmax and the epilogue; S is double-buffered in TMEM, O accumulates in
+// TMEM.
 #include "fa_common.cuh"
 #include "fa_kernels.h"
 
