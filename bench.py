@@ -596,6 +596,37 @@ def decode_workloads(dev, stream, hbm_peak_gbs, iters=20):
     return res
 
 
+def fwd_only(args):
+    """--fwd-only N[:D]: the forward of standard workload N alone, for
+    profiling captures (the same seeded inputs as the forward lines of the
+    full run)."""
+    import torch
+
+    from varlen_flashattention_02_b200 import fa_varlen
+
+    n, _, d = args.fwd_only.partition(":")
+    w = synth.standard_workload(int(n), head_dim=int(d) if d else None)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    t = w.tensors()
+    q, k, v = (torch.from_numpy(t[x].view(np.int16)).view(torch.bfloat16).to(dev) for x in ("q", "k", "v"))
+    cq, ck = torch.from_numpy(w.cu_q).to(dev), torch.from_numpy(w.cu_k).to(dev)
+    call = lambda: fa_varlen.fa_varlen_fwd(q, k, v, cq, ck, w.max_seqlen_q, w.max_seqlen_k, w.scale, w.causal,
+                                           stream=stream)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        call()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b) / args.steps
+    return {"mode": "fwd-only", "workload": w.name, "calls": args.steps, "ms_per_call": ms,
+            "tflops": fwd_flops(w.cu_q, w.cu_k, w.heads, w.head_dim, w.causal) / (ms * 1e-3) / 1e12}
+
+
 def decode_only(args):
     """--decode BATCHxKEYS: the split-KV decode call of that shape alone, for
     profiling captures (the same seeded inputs and split count as the decode
@@ -756,6 +787,9 @@ def main():
                          "heads = one workload, its heads split across the ranks (strong scaling)")
     ap.add_argument("--tokens", type=int, default=synth.TOTAL_TOKENS,
                     help="total tokens of the workload (default 16384; smaller only for profiling captures)")
+    ap.add_argument("--fwd-only", metavar="N[:D]",
+                    help="profiling mode, one GPU: only the forward of standard workload N (1-5) at head_dim D, "
+                         "--warmup untimed and --steps timed calls")
     ap.add_argument("--decode", metavar="BATCHxKEYS",
                     help="profiling mode, one GPU: only the split-KV decode call of that shape (one query token, "
                          "32 query heads over 8 key/value heads, d=128), --warmup untimed and --steps timed calls")
@@ -778,6 +812,11 @@ def main():
         if world != 1:
             sys.exit("--decode runs on one GPU")
         print(json.dumps(decode_only(args)), flush=True)
+        return
+    if args.fwd_only:
+        if world != 1:
+            sys.exit("--fwd-only runs on one GPU")
+        print(json.dumps(fwd_only(args)), flush=True)
         return
 
     import torch
