@@ -133,7 +133,7 @@ fa_status_t check_sizes(int batch, int total_q, int total_k, int max_sq, int max
   if (batch < 1 || total_q < 0 || total_k < 0 || max_sq < 0 || max_sk < 0 || H < 1) return FA_ERR_INVALID_ARGUMENT;
   if (Hk < 1 || Hk > H || H % Hk != 0) return FA_ERR_INVALID_ARGUMENT;
   if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARGUMENT;
-  if (D != 64 && D != 128 && D != 256) return FA_ERR_UNSUPPORTED;  // 256: forward only
+  if (D != 64 && D != 128 && D != 256) return FA_ERR_UNSUPPORTED;
   // Row indices and TMA coordinates are int32; element offsets are 64-bit.
   const long long hd = static_cast<long long>(H) * D;
   if (hd > (1ll << 31) - 1 || static_cast<long long>(total_q) + 2 * fa::kFwdBM > (1ll << 31) - 1 ||
