@@ -10,12 +10,25 @@ from varlen_flashattention_02_b200 import synth
 pytestmark = pytest.mark.gpu
 
 
-def _read_pairs(ws, backward, batch, total_q, total_k):
+def _read_pairs(ws, backward, batch, total_q, total_k, with_classes=False):
     lay = sr.layout(batch, total_q, total_k, backward)
     raw = ws.cpu().numpy()
     status, n_pairs = (int(x) for x in raw[:8].view(np.uint32))
     pairs = raw[lay["pairs"]:lay["pairs"] + 8 * n_pairs].view(np.int32).reshape(-1, 2)
+    if with_classes:
+        # header words 4..15: number of pairs of cost >= 2^k, k = 0..11
+        return status, pairs, raw[16:64].view(np.uint32).astype(np.int64)
     return status, pairs
+
+
+def _check_order(pairs, want, class_end):
+    cost = {(b, t): c for b, t, c in want}
+    got = [(int(b), int(t)) for b, t in pairs]
+    assert sorted(got) == sorted(cost)  # same multiset, no padding tiles
+    costs = [cost[p] for p in got]
+    assert all(costs[i] >= costs[i + 1] for i in range(len(costs) - 1))  # longest first
+    clamped = np.minimum(np.array(costs, dtype=np.int64), 2047)
+    assert [int(x) for x in class_end] == [int(np.sum(clamped >= (1 << k))) for k in range(12)]
 
 
 @pytest.mark.parametrize("causal", [False, True])
@@ -27,14 +40,30 @@ def test_fwd_work_list(wl, causal):
     w.causal = causal
     ws = fa_varlen.new_workspace(fa_varlen.fwd_workspace_size(w.batch, w.total_q, w.heads, w.head_dim), "cuda")
     pu.run_fwd(w, workspace=ws)
-    status, pairs = _read_pairs(ws, False, w.batch, w.total_q, w.total_k)
+    status, pairs, class_end = _read_pairs(ws, False, w.batch, w.total_q, w.total_k, with_classes=True)
     assert status == 0
-    want = sr.work_list(w.cu_q, w.cu_k, causal)
-    cost = {(b, t): c for b, t, c in want}
-    got = [(int(b), int(t)) for b, t in pairs]
-    assert sorted(got) == sorted(cost)  # same multiset, no padding tiles
-    costs = [cost[p] for p in got]
-    assert all(costs[i] >= costs[i + 1] for i in range(len(costs) - 1))  # longest first
+    _check_order(pairs, sr.work_list(w.cu_q, w.cu_k, causal), class_end)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("wl", [3, 5])
+def test_bwd_work_list(wl, causal):
+    """The backward's list (key tiles, ordered by the query tiles that see
+    them) and its cost-class boundaries, which set the backward's work
+    order."""
+    from varlen_flashattention_02_b200 import fa_varlen
+
+    w = synth.standard_workload(wl)
+    w.causal = causal
+    (q, k, v), out, lse = pu.run_fwd(w)
+    ws = fa_varlen.new_workspace(fa_varlen.bwd_workspace_size(w.batch, w.total_q, w.total_k, w.heads, w.head_dim),
+                                 "cuda")
+    do = pu.to_dev(w.tensors()["dout"])
+    fa_varlen.fa_varlen_bwd(do, q, k, v, out, lse, pu.cu_dev(w.cu_q), pu.cu_dev(w.cu_k), w.max_seqlen_q,
+                            w.max_seqlen_k, w.scale, causal, workspace=ws)
+    status, pairs, class_end = _read_pairs(ws, True, w.batch, w.total_q, w.total_k, with_classes=True)
+    assert status == 0
+    _check_order(pairs, sr.work_list(w.cu_q, w.cu_k, causal, backward=True), class_end)
 
 
 @pytest.mark.parametrize("cu_q,cu_k,max_q", [

@@ -111,10 +111,36 @@ struct Item {
   int n;       // steps: nt * group
 };
 
-__device__ __forceinline__ Item get_item(const BwdArgs& a, const int2* pairs, int idx) {
+// Work order. The items are the work list's (sequence, key tile) pairs,
+// most query tiles first, each for every key/value head, claimed in index
+// order. Plain order: item idx is pair idx / Hk of head idx % Hk, so the
+// longest items of all heads start first. Class order (CLASSES): the pairs
+// fall into cost classes [2^k, 2^(k+1)) (class_end from the work-list
+// kernel); the classes are taken longest first, and within a class head by
+// head. Concurrent items then mostly share a head, whose Q/dO tiles and part
+// of the fp32 dQ accumulator stay in L2 while they are read and reduced
+// into, while no item can start much later than one twice as long.
+template <bool CLASSES>
+__device__ __forceinline__ Item get_item(const BwdArgs& a, const int2* pairs, int idx, int n_pairs,
+                                         const uint32_t* class_end) {
   Item it;
-  const int2 pr = pairs[idx / a.Hk];
-  it.hk = idx % a.Hk;
+  int pair = idx / a.Hk, hk = idx % a.Hk;
+  if constexpr (CLASSES) {
+    int lo = 0;  // pairs of the classes before this one
+#pragma unroll
+    for (int k = kCostClasses - 1; k >= -1; --k) {
+      const int hi = k >= 0 ? static_cast<int>(class_end[k]) : n_pairs;
+      if (idx < hi * a.Hk) {
+        const int n = hi - lo, local = idx - lo * a.Hk;
+        hk = local / n;
+        pair = lo + local % n;
+        break;
+      }
+      lo = hi;
+    }
+  }
+  const int2 pr = pairs[pair];
+  it.hk = hk;
   it.h0 = it.hk * a.group;
   it.b = pr.x;
   it.j = pr.y;
@@ -283,7 +309,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
   const Abort ab{&bars.abort_flag, &hdr->status, a.wait_ns};
-  const int n_items = (hdr->status == FA_OK) ? static_cast<int>(hdr->n_pairs) * a.Hk : 0;
+  const int n_pairs = static_cast<int>(hdr->n_pairs);
+  const int n_items = (hdr->status == FA_OK) ? n_pairs * a.Hk : 0;
+  // Class order outside the deterministic mode (whose list is in tile
+  // order, and whose query tiles take their dQ turns in key-tile order).
+  constexpr bool kClassOrder = !DET;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -294,6 +324,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // for the K/V buffer, so an item's first step starts without an
       // exposed load.
       uint32_t m = 0, p = 0, ni = 0;
+      uint32_t class_end[kCostClasses];
+#pragma unroll
+      for (int k = 0; k < kCostClasses; ++k) class_end[k] = kClassOrder ? hdr->class_end[k] : 0u;
       auto load_qdo = [&](const Item& it, int s) -> bool {
         const int st = p % NQ;
         const Step sp = item_step(it, s);
@@ -316,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int idx;
         Item it;
         auto decode = [&](int slot, int v) {
-          it = get_item(a, pairs, v);
+          it = get_item<kClassOrder>(a, pairs, v, n_pairs, class_end);
           bars.item_data[slot] = it;
         };
         if (!publish_item_decoded(bars.items, ni, &hdr->work_counter, n_items, idx, ab, decode)) goto producer_done;

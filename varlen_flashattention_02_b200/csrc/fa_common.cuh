@@ -27,12 +27,18 @@ constexpr int kBwdBN = 128;
 constexpr int kBwdBM = 128;
 
 // Per-call device state at the start of the workspace.
+constexpr int kCostClasses = 12;  // cost classes [1, 2), [2, 4), ..., [2^11, inf)
+
 struct WsHeader {
   uint32_t status;         // fa_status_t of the device side of the call
   uint32_t n_pairs;        // number of (sequence, tile) pairs in `pairs`
   uint32_t work_counter;   // next work item to hand out (reset by the scheduler)
   uint32_t work_counter2;  // the same, for a second kernel over the same list (head_dim 256 backward)
-  uint32_t reserved[60];
+  // Cost-ordered lists: class_end[k] = number of pairs whose cost (visible
+  // tiles on the other side) is at least 2^k; the pairs of cost class
+  // [2^k, 2^(k+1)) are pairs[class_end[k+1] .. class_end[k]).
+  uint32_t class_end[kCostClasses];
+  uint32_t reserved[60 - kCostClasses];
 };
 static_assert(sizeof(WsHeader) == 256, "header is one 256-byte block");
 

@@ -212,6 +212,11 @@ __global__ void __launch_bounds__(kThreads) sched_prep_kernel(SchedArgs a) {
   }
   __syncthreads();
 
+  // Cost classes: s_hist[c] now counts the pairs of cost above c.
+  static_assert(kBins == 1 << (kCostClasses - 1), "the top class starts at the last bucket");
+  const int class_end = tid < kCostClasses ? s_hist[(1 << tid) - 1] : 0;
+  __syncthreads();
+
   // Scatter.
   for (int p = tid; p < n_pairs; p += kThreads) {
     const int b = find_seq(seq_off, a.batch, p);
@@ -221,6 +226,7 @@ __global__ void __launch_bounds__(kThreads) sched_prep_kernel(SchedArgs a) {
     const int pos = atomicAdd(&s_hist[c], 1);
     pairs[pos] = make_int2(b, t);
   }
+  if (tid < kCostClasses) hdr->class_end[tid] = tile_major ? 0u : static_cast<uint32_t>(class_end);
   if (tid == 0) {
     hdr->status = FA_OK;
     hdr->n_pairs = static_cast<uint32_t>(n_pairs);
