@@ -50,10 +50,31 @@ struct Item {
   int i0, nt, h0, n;
 };
 
-__device__ __forceinline__ Item get_item(const BwdArgs& a, const int2* pairs, int idx, int bm) {
+// Work order, as in the head_dim 64/128 backward: outside the deterministic
+// mode the items are taken by cost class (longest class first, the work
+// list's class_end) and head by head within a class, so that concurrent
+// items mostly share a head whose Q/dO tiles and dQ accumulator rows stay in
+// L2; the deterministic mode takes pair idx / Hk of head idx % Hk.
+__device__ __forceinline__ Item get_item(const BwdArgs& a, const int2* pairs, int idx, int bm, int n_pairs,
+                                         const uint32_t (&class_end)[kCostClasses]) {
   Item it;
-  const int2 pr = pairs[idx / a.Hk];
-  it.hk = idx % a.Hk;
+  int pair = idx / a.Hk, hk = idx % a.Hk;
+  if (!a.deterministic) {
+    int lo = 0;  // pairs of the classes before this one
+#pragma unroll
+    for (int k = kCostClasses - 1; k >= -1; --k) {
+      const int hi = k >= 0 ? static_cast<int>(class_end[k]) : n_pairs;
+      if (idx < hi * a.Hk) {
+        const int n = hi - lo, local = idx - lo * a.Hk;
+        hk = local / n;
+        pair = lo + local % n;
+        break;
+      }
+      lo = hi;
+    }
+  }
+  const int2 pr = pairs[pair];
+  it.hk = hk;
   it.h0 = it.hk * a.group;
   it.b = pr.x;
   it.j = pr.y;
@@ -204,11 +225,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       // K once per item, then Q of each step once the previous step's S^T
       // has read the single Q buffer.
       uint32_t m = 0, p = 0, ni = 0;
+      const int n_pairs = static_cast<int>(hdr->n_pairs);
+      uint32_t class_end[kCostClasses];
+#pragma unroll
+      for (int k = 0; k < kCostClasses; ++k) class_end[k] = hdr->class_end[k];
       for (;;) {
         int idx;
         Item it;
         auto decode = [&](int slot, int v) {
-          it = get_item(a, pairs, v, BM);
+          it = get_item(a, pairs, v, BM, n_pairs, class_end);
           bars.item_data[slot] = it;
         };
         if (!publish_item_decoded(bars.items, ni, counter, n_items, idx, ab, decode)) goto k_done;
@@ -537,11 +562,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Per item K and V; per step dO (free once the previous dP^T is done)
       // and then Q (free once the previous dK MMA is done).
       uint32_t m = 0, nq = 0, nd = 0, ni = 0;  // K/V, Q and dO loads issued
+      const int n_pairs = static_cast<int>(hdr->n_pairs);
+      uint32_t class_end[kCostClasses];
+#pragma unroll
+      for (int k = 0; k < kCostClasses; ++k) class_end[k] = hdr->class_end[k];
       for (;;) {
         int idx;
         Item it;
         auto decode = [&](int slot, int v) {
-          it = get_item(a, pairs, v, BM);
+          it = get_item(a, pairs, v, BM, n_pairs, class_end);
           bars.item_data[slot] = it;
         };
         if (!publish_item_decoded(bars.items, ni, counter, n_items, idx, ab, decode)) goto loads_done;
