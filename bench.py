@@ -84,6 +84,46 @@ def shard_heads(tensors: dict, h0: int, h1: int, kv_group: int = 1) -> dict:
     return out
 
 
+def sequence_split(cu_q, cu_k, world: int) -> list:
+    """Sequences of each rank when the sequences of one problem are split
+    across ``world`` GPUs, balanced by attention work: sequence b costs
+    lq_b * lk_b (a causal mask halves every cost alike), and the sequences,
+    largest first, go one by one to the rank with the least work so far (ties
+    to the lower rank, then to the lower sequence index). Each rank's list is
+    in sequence order. Every (sequence, head) unit is independent in both
+    directions, so the ranks exchange nothing."""
+    lq = np.diff(np.asarray(cu_q, dtype=np.int64))
+    lk = np.diff(np.asarray(cu_k, dtype=np.int64))
+    if world < 1 or len(lq) < world:
+        raise ValueError(f"cannot split {len(lq)} sequences over {world} ranks")
+    cost = lq * lk
+    load = [0] * world
+    parts = [[] for _ in range(world)]
+    for b in sorted(range(len(cost)), key=lambda i: (-int(cost[i]), i)):
+        r = min(range(world), key=lambda i: (load[i], i))
+        parts[r].append(b)
+        load[r] += int(cost[b])
+    return [sorted(x) for x in parts]
+
+
+def shard_sequences(tensors: dict, cu_q, cu_k, seqs) -> tuple:
+    """This rank's problem: the rows of sequences ``seqs`` (in that order)
+    packed back to back, query-side arrays (q, dout) from cu_q and key/value
+    arrays from cu_k, with their own cumulative offsets."""
+    cu_q = np.asarray(cu_q, dtype=np.int64)
+    cu_k = np.asarray(cu_k, dtype=np.int64)
+
+    def rows(cu):
+        return np.concatenate([np.arange(cu[b], cu[b + 1]) for b in seqs]).astype(np.int64)
+
+    def offsets(cu):
+        return np.concatenate([[0], np.cumsum([cu[b + 1] - cu[b] for b in seqs])]).astype(np.int32)
+
+    rq, rk = rows(cu_q), rows(cu_k)
+    out = {n: np.ascontiguousarray(a[rq if n in ("q", "dout") else rk]) for n, a in tensors.items()}
+    return out, offsets(cu_q), offsets(cu_k)
+
+
 def weak_scaling_value(world: int, flops_per_rank: float, max_ms_per_step: float) -> float:
     """Whole-job TFLOP/s: every rank did ``flops_per_rank`` per step; the job's
     step time is the slowest rank's."""
@@ -208,15 +248,21 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = bench_workload(args.tokens)
-    split_heads = args.split == "heads" and world > 1
-    heads_job = w.heads
+    split_heads = args.split in ("heads", "sequences") and world > 1  # one problem over the ranks
+    heads_job, batch_job, tokens_job = w.heads, w.batch, w.total_q
     if split_heads:
+        F_job = fwd_flops(w.cu_q, w.cu_k, w.heads, w.head_dim, w.causal)
+    if split_heads and args.split == "heads":
         # One problem, its heads split across the ranks: every rank draws the
         # same seeded batch and keeps its contiguous slice of heads.
-        F_job = fwd_flops(w.cu_q, w.cu_k, w.heads, w.head_dim, w.causal)
         h0, h1 = head_range(w.heads, world, rank)
         t = shard_heads(w.tensors(), h0, h1)
         w.heads = h1 - h0
+    elif split_heads:
+        # One problem, its sequences split across the ranks by work: every
+        # rank draws the same seeded batch and keeps its sequences, repacked.
+        seqs = sequence_split(w.cu_q, w.cu_k, world)[rank]
+        t, w.cu_q, w.cu_k = shard_sequences(w.tensors(), w.cu_q, w.cu_k, seqs)
     else:
         w.seed = w.seed + 1000 * rank  # same shape, own data per rank
         t = w.tensors()
@@ -407,12 +453,14 @@ def run_ours(args, rank, world, local_rank):
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong" if split_heads else "weak",
         "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded bf16 N(0,1); lengths from numpy default_rng)",
-        "config": {"workload": WORKLOAD, "total_tokens": w.total_q, "batch": w.batch, "heads": heads_job,
+        "config": {"workload": WORKLOAD, "total_tokens": tokens_job, "batch": batch_job, "heads": heads_job,
                    "head_dim": D, "causal": True, "max_seqlen": w.max_seqlen_q,
                    "flops_fwd": F, "flop_convention": "fwd+bwd = 3.5 * F_fwd (bwd = 2.5 * F_fwd); causal halved",
                    "l2": "256 MiB buffer written between steps (and step inputs exceed L2)",
                    "parallelism": (f"strong: heads split over {world} ranks (contiguous slices, cu_seqlens "
-                                   f"replicated, no data-path collective)" if split_heads else
+                                   f"replicated, no data-path collective)" if split_heads and args.split == "heads"
+                                   else f"strong: sequences split over {world} ranks, balanced by lq*lk (each "
+                                   f"rank's sequences repacked, no data-path collective)" if split_heads else
                                    f"weak: {world} independent replicas of the workload, no data-path collective")},
         "fwd_tflops": F / (statistics.mean(fwd_call_ms) * 1e-3) / 1e12,
         "bwd_tflops": 2.5 * F / (statistics.mean(bwd_call_ms) * 1e-3) / 1e12,
@@ -782,9 +830,10 @@ def main():
     ap.add_argument("--no-aux", action="store_true", help="skip the forward-only workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--split", choices=("replicas", "heads"), default="replicas",
+    ap.add_argument("--split", choices=("replicas", "heads", "sequences"), default="replicas",
                     help="N > 1: replicas = every rank runs the whole workload on its own data (weak scaling); "
-                         "heads = one workload, its heads split across the ranks (strong scaling)")
+                         "heads = one workload, its heads split across the ranks; sequences = one workload, its "
+                         "sequences split across the ranks balanced by lq*lk (strong scaling)")
     ap.add_argument("--tokens", type=int, default=synth.TOTAL_TOKENS,
                     help="total tokens of the workload (default 16384; smaller only for profiling captures)")
     ap.add_argument("--fwd-only", metavar="N[:D]",

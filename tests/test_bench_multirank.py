@@ -117,6 +117,103 @@ def test_head_split_reassembles_bitwise_gloo():
     assert out["ok"] == [True] * 5
 
 
+def _seq_split_worker(rank, world, port, out):
+    """One rank of a sequence-split problem: its sequences, repacked, through
+    the oracle; the pieces gathered over gloo and put back in place on rank 0."""
+    import numpy as np
+    import torch.distributed as dist
+
+    import bench
+    import oracle
+    from varlen_flashattention_02_b200 import synth
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = synth.make_workload("seqsplit", [70, 130, 1, 45, 200], [90, 130, 4, 45, 150], heads=2, head_dim=64,
+                                causal=True, seed=78)
+        seqs = bench.sequence_split(w.cu_q, w.cu_k, world)[rank]
+        t, cq, ck = bench.shard_sequences(w.tensors(), w.cu_q, w.cu_k, seqs)
+        o, l = oracle.fwd(t["q"], t["k"], t["v"], cq, ck, w.scale, True)
+        g = oracle.bwd(t["q"], t["k"], t["v"], t["dout"], cq, ck, w.scale, True)
+        pieces = [None] * world
+        dist.all_gather_object(pieces, (seqs, o, l) + tuple(g))
+        if rank == 0:
+            full_o, full_l = oracle.fwd(*(w.tensors()[n] for n in ("q", "k", "v")), w.cu_q, w.cu_k, w.scale, True)
+            full_g = oracle.bwd(*(w.tensors()[n] for n in ("q", "k", "v", "dout")), w.cu_q, w.cu_k, w.scale, True)
+            got = [np.full_like(x, np.nan) for x in (full_o, full_l) + tuple(full_g)]
+            for seq_list, po, pl, pdq, pdk, pdv in pieces:
+                rq = rk = 0
+                for b in seq_list:
+                    nq = int(w.cu_q[b + 1] - w.cu_q[b])
+                    nk = int(w.cu_k[b + 1] - w.cu_k[b])
+                    sq = slice(int(w.cu_q[b]), int(w.cu_q[b + 1]))
+                    sk = slice(int(w.cu_k[b]), int(w.cu_k[b + 1]))
+                    got[0][sq], got[1][:, sq], got[2][sq] = po[rq:rq + nq], pl[:, rq:rq + nq], pdq[rq:rq + nq]
+                    got[3][sk], got[4][sk] = pdk[rk:rk + nk], pdv[rk:rk + nk]
+                    rq, rk = rq + nq, rk + nk
+            want = (full_o, full_l) + tuple(full_g)
+            out["ok"] = [np.array_equal(a, b) for a, b in zip(got, want)]
+            out["parts"] = [list(p[0]) for p in pieces]
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sequence_split_reassembles_bitwise_gloo():
+    """Two gloo ranks split the sequences of one problem (bench.py --split
+    sequences), balanced by lq*lk: each rank's repacked problem, gathered and
+    put back at the original offsets, equals the whole problem bit for bit."""
+    import oracle
+
+    oracle.build()
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_seq_split_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0
+    assert out["ok"] == [True] * 5
+    assert sorted(sum(out["parts"], [])) == [0, 1, 2, 3, 4]  # every sequence exactly once
+
+
+def test_sequence_split_balance():
+    import numpy as np
+
+    import bench
+
+    cu = np.array([0, 5664, 12359, 13044, 16384], dtype=np.int32)  # the fwd+bwd workload's lengths
+    assert bench.sequence_split(cu, cu, 2) == [[1], [0, 2, 3]]  # 44.8M vs 43.7M of lq*lk
+    assert bench.sequence_split(cu, cu, 1) == [[0, 1, 2, 3]]
+    assert bench.sequence_split(cu, cu, 4) == [[1], [0], [3], [2]]
+    lq = np.array([5, 4, 3, 3, 3, 2])
+    cq = np.concatenate([[0], np.cumsum(lq)])
+    parts = bench.sequence_split(cq, cq, 2)  # greedy by lq^2: 25 | 16 9 | 9 (to 25) ...
+    loads = [sum(int(lq[b]) ** 2 for b in p) for p in parts]
+    assert sorted(sum(parts, [])) == list(range(6)) and abs(loads[0] - loads[1]) <= 9
+    with pytest.raises(ValueError):
+        bench.sequence_split(cu, cu, 5)
+
+
+def test_shard_sequences():
+    import numpy as np
+
+    import bench
+
+    cq = np.array([0, 2, 5, 6])
+    ck = np.array([0, 1, 4, 8])
+    q = np.arange(6 * 2).reshape(6, 1, 2)
+    k = np.arange(8 * 2).reshape(8, 1, 2) + 100
+    t, nq, nk = bench.shard_sequences({"q": q, "k": k, "v": k, "dout": q}, cq, ck, [0, 2])
+    assert np.array_equal(t["q"], q[[0, 1, 5]]) and np.array_equal(t["k"], k[[0, 4, 5, 6, 7]])
+    assert list(nq) == [0, 2, 3] and list(nk) == [0, 1, 5]
+
+
 def test_head_range():
     import bench
 
