@@ -113,3 +113,19 @@ def test_bwd_gradient_sums():
         assert float((dvs - dos).norm() / dos.norm()) < 2e-2
         dks = dk[sk].double().sum(0).cpu()
         assert float(dks.norm() / dk[sk].double().norm().cpu()) < 5e-2
+
+
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+def test_bwd_many_short_sequences(causal):
+    """2000 sequences of 1 to 64 queries and 1 to 96 keys (seeded): thousands
+    of one-tile backward items. Every gradient against the oracle."""
+    rng = np.random.default_rng(13)
+    lq = rng.integers(1, 65, 2000).tolist()
+    lk = rng.integers(1, 97, 2000).tolist()
+    w = synth.make_workload("many-short", lq, lk, heads=2, head_dim=128, causal=causal, seed=14)
+    dq, dk, dv = _run_bwd(w)
+    t = w.tensors()
+    rq, rk, rv = oracle.bwd(t["q"], t["k"], t["v"], t["dout"], w.cu_q, w.cu_k, w.scale, w.causal)
+    _check("dq", dq, rq)
+    _check("dk", dk, rk)
+    _check("dv", dv, rv)
