@@ -79,3 +79,41 @@ def test_offsets_beyond_2_31_elements():
             assert err <= pu.GRAD_REL_L2, f"{name}[{s},{h}] rel-L2 {err:.3e}"
     del big, out, lse, dq, dk, dv
     torch.cuda.empty_cache()
+
+
+def test_single_sequence_of_262144_tokens():
+    """One causal sequence of 262,144 tokens (2048 tiles of 128: the work
+    list's cost histogram clamps the longest items, and key tile 0's item has
+    2048 steps). The forward is checked against the oracle on sampled rows of
+    both heads; the backward, too long for the fp64 oracle, against what holds
+    at any size: every row of P sums to one, so sum_j dV_j = sum_i dO_i, and
+    every row of dS sums to zero, so sum_j dK_j = 0 (up to rounding)."""
+    import torch
+
+    from varlen_flashattention_02_b200 import fa_varlen
+
+    n = 262144
+    w = synth.make_workload("one-long", [n], heads=2, head_dim=64, causal=True, seed=910)
+    t = w.tensors()
+    q, k, v, do = (pu.to_dev(t[x]) for x in ("q", "k", "v", "dout"))
+    cu = pu.cu_dev(w.cu_q)
+    out, lse = fa_varlen.fa_varlen_fwd(q, k, v, cu, cu, n, n, w.scale, True)
+    dq, dk, dv = fa_varlen.fa_varlen_bwd(do, q, k, v, out, lse, cu, cu, n, n, w.scale, True)
+    torch.cuda.synchronize()
+    step = 8191  # rows 0, 8191, ... : both ends of tiles, early and late in the sequence
+    ref_out, ref_lse = oracle.fwd(t["q"], t["k"], t["v"], w.cu_q, w.cu_q, w.scale, True, row_step=step)
+    rows = np.arange(0, n, step)
+    rows_dev = torch.as_tensor(rows, device="cuda")
+    for h in range(w.heads):
+        got = pu.bf16_dev_to_f64(out[rows_dev, h])
+        assert float(np.max(np.abs(got - ref_out[rows, h]))) <= pu.OUT_MAX_ABS
+        assert pu.rel_l2(got, ref_out[rows, h]) <= pu.OUT_REL_L2
+        gl = lse[h, rows_dev].cpu().numpy().astype(np.float64)
+        assert float(np.max(np.abs(gl - ref_lse[h, rows]))) <= pu.LSE_MAX_ABS
+    for x in (out, dq, dk, dv):
+        assert bool(torch.isfinite(x.float()).all())
+    dvs, dos = dv.double().sum(0), do.double().sum(0)
+    assert float((dvs - dos).norm() / dos.norm()) < 2e-2
+    assert float(dk.double().sum(0).norm() / dk.double().norm()) < 5e-2
+    del q, k, v, do, out, lse, dq, dk, dv
+    torch.cuda.empty_cache()
